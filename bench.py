@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Throughput of the Muon weight update on B200: full Mamba-2 130M optimizer steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload mamba2-130m|mamba2-2k]
+
+One step = the whole hot path over every in_proj (24 x 3352 x 768) and
+out_proj (24 x 768 x 1536) matrix of a Mamba-2 130M model, in one
+muon_step_groups call: momentum + Nesterov + Frobenius norm, 5 quintic
+Newton-Schulz iterations (three tensor-core products each), shape scale and
+decoupled weight decay applied to W.  Gradients are synthetic (Gaussian bulk
++ rank-4 spike, bf16), redrawn per step from a pool of pre-generated sets
+resident in HBM; W and M persist across steps.
+
+Multi-GPU (torchrun): every rank runs its own full step on its own GPU (the
+matrices of different models/ranks are independent -- weak scaling, no
+collective on the data path); time is the max over ranks.
+
+Prints ONE JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
+(the baseline arm) on rank 0 over a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Muon steps/s and Newton-Schulz TFLOP/s (% of bf16 peak), Mamba-2 130M shapes"
+UNIT = "steps/s"
+QUINTIC = (3.4445, -4.7750, 2.0315)
+K_ITERS = 5
+HP = dict(lr=0.02, beta=0.95, weight_decay=0.1, eps=1e-7)
+GRAD_SETS = 4
+
+WORKLOADS = {
+    # name: list of (label, count, rows, cols)
+    "mamba2-130m": [("out_proj", 24, 768, 1536), ("in_proj", 24, 3352, 768)],
+    "mamba2-2k": [("out_proj", 48, 2048, 4096), ("in_proj", 48, 8768, 2048)],
+}
+WORKLOAD_NAMES = {
+    "mamba2-130m": "full Mamba-2 130M Muon step: in_proj 24x3352x768 + out_proj 24x768x1536 bf16, "
+                   "5 quintic NS iterations, one muon_step_groups call",
+    "mamba2-2k": "scaled Mamba-2-style d_model 2048: in_proj 48x8768x2048 + out_proj 48x2048x4096 bf16, "
+                 "5 quintic NS iterations",
+}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- work counts
+def ns_flops(groups, k=K_ITERS):
+    """Algorithmic NS flops: per iteration m^2 n (symmetric Gram) + m^3 (symmetric A^2) + 2 m^2 n (B X)."""
+    tot = 0
+    for _, L, R, C in groups:
+        m, n = min(R, C), max(R, C)
+        tot += L * k * (3 * m * m * n + m ** 3)
+    return tot
+
+
+def ns_dense_flops(groups, k=K_ITERS):
+    tot = 0
+    for _, L, R, C in groups:
+        m, n = min(R, C), max(R, C)
+        tot += L * k * (4 * m * m * n + 2 * m ** 3)
+    return tot
+
+
+def elements(groups):
+    return sum(L * R * C for _, L, R, C in groups)
+
+
+def momentum_bytes(groups):
+    """Algorithmic bytes of the momentum pass: G 2 + M 4 (read) + M 4 + U 2 (write) per element."""
+    return 12 * elements(groups)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def gemm_source_hash():
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "device_utils.cuh", "internal.h"):
+        with open(os.path.join(ROOT, "spectral_optimizer_state_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it matches the current kernel source."""
+    path = os.path.join(ROOT, "profiles", f"ns_gemm_kernel.{workload}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("gemm_source_sha256") != gemm_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.lines = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", self.gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- inputs
+def make_inputs(groups, device, sets=GRAD_SETS, pinned_host=False):
+    import torch
+
+    from synthetic import group_inputs, group_weights
+    Ws, Ms, Gsets, Ghost = [], [], [], []
+    for g, (_, L, R, C) in enumerate(groups):
+        Ws.append([torch.from_numpy(w).to(torch.bfloat16).to(device) for w in group_weights(3, g, L, R, C)])
+        Ms.append([torch.zeros((R, C), dtype=torch.float32, device=device) for _ in range(L)])
+    for s in range(sets):
+        per_group, per_group_host = [], []
+        for g, (_, L, R, C) in enumerate(groups):
+            gs = group_inputs(3, s, g, L, R, C)
+            per_group.append([torch.from_numpy(x).to(torch.bfloat16).to(device) for x in gs])
+            if pinned_host and s == 0:
+                per_group_host.append([torch.from_numpy(x).to(torch.bfloat16).pin_memory() for x in gs])
+        Gsets.append(per_group)
+        if pinned_host and s == 0:
+            Ghost = per_group_host
+    return Ws, Ms, Gsets, Ghost
+
+
+# ---------------------------------------------------------------- oracle arm
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads") for d in threadpool_info() if d.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_sample(groups, budget_s=12.0, max_per_group=4):
+    """Time the fp64 oracle on whole matrices of one step until ~budget_s; returns steps/s and a label."""
+    import oracle
+    from synthetic import group_inputs, group_weights
+    coeffs = [QUINTIC] * K_ITERS
+    done = {lbl: 0 for lbl, *_ in groups}
+    t_total = 0.0
+    frac = 0.0
+    total_mats = sum(L for _, L, _, _ in groups)
+    for i in range(max_per_group):
+        for g, (lbl, L, R, C) in enumerate(groups):
+            G = group_inputs(3, 0, g, 1, R, C)[0].astype(np.float64)
+            W = group_weights(3, g, 1, R, C)[0].astype(np.float64)
+            M = np.zeros((R, C))
+            t0 = time.perf_counter()
+            oracle.muon_step(W, G, M, coeffs, **HP)
+            t_total += time.perf_counter() - t0
+            done[lbl] += 1
+            frac += 1.0 / total_mats
+        if t_total >= budget_s:
+            break
+    sample = " + ".join(f"{n} {lbl}" for lbl, n in done.items()) + " matrices of one step (oracle.muon_step, fp64 NumPy)"
+    return frac / t_total, sample, t_total
+
+
+def run_reference(args, groups, rank):
+    if rank != 0:
+        return
+    per_step = []
+    labels = None
+    coeffs = [QUINTIC] * K_ITERS
+    import oracle
+    from synthetic import group_inputs, group_weights
+    total_mats = sum(L for _, L, _, _ in groups)
+    mats = []
+    for g, (lbl, L, R, C) in enumerate(groups):
+        mats.append((g, lbl, R, C, group_inputs(3, 0, g, 1, R, C)[0].astype(np.float64),
+                     group_weights(3, g, 1, R, C)[0].astype(np.float64)))
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        for (g, lbl, R, C, G, W) in mats:  # one matrix of each group per step
+            oracle.muon_step(W, G, np.zeros((R, C)), coeffs, **HP)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            per_step.append(dt)
+    frac = len(mats) / total_mats
+    value = frac * len(per_step) / sum(per_step)
+    labels = " + ".join(f"1 {m[1]}" for m in mats) + " matrix per step (oracle.muon_step, fp64 NumPy)"
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": labels},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(args):
+    return {"workload": WORKLOAD_NAMES[args.workload], "ns_iterations": K_ITERS,
+            "coefficients": list(QUINTIC), "hparams": HP, "parallelism": f"replicas x{args.gpus} (independent matrices)",
+            "grad_sets_in_hbm": GRAD_SETS,
+            "l2": "inputs larger than L2: each step streams G, M and W (%.2f GB)" % (
+                elements(WORKLOADS[args.workload]) * 8 / 1e9)}
+
+
+# ---------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="mamba2-130m")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    groups = WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, groups, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from spectral_optimizer_state_b200 import Muon
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+
+    # cpu baseline first (rank 0, N = 1), before any pools or threads touch the GPU
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample, spent = oracle_sample(groups)
+        cpu = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample,
+               "seconds": round(spent, 2)}
+
+    mu = Muon(local)
+    mu.set_coeffs([QUINTIC] * K_ITERS)
+    Ws, Ms, Gsets, Ghost = make_inputs(groups, device, pinned_host=True)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        mu.step_groups([(Ws[g], Gsets[i % GRAD_SETS][g], Ms[g]) for g in range(len(groups))], stream=stream, **HP)
+
+    for i in range(args.warmup):
+        step(i)
+    st, flags = mu.status()
+    assert st == 0, f"device status {st}"
+
+    peaks, peak_src = load_peaks()
+    uuid = str(torch.cuda.get_device_properties(device).uuid)
+    clocks = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+
+    mu.profile_read(reset=True)
+    mu.profile_enable(True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.25)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    mu.profile_enable(False)
+    prof = mu.profile_read(reset=True)
+    st, flags = mu.status()
+    assert st == 0, f"device status {st}"
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # e2e through the host-gradient entry point (pinned host G in, norms + flags out)
+    e2e_steps = max(3, min(args.e2e_steps, args.steps))
+    for i in range(2):
+        mu.step_groups_host([(Ws[g], Ghost[g], Ms[g]) for g in range(len(groups))], stream=stream, **HP)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        mu.step_groups_host([(Ws[g], Ghost[g], Ms[g]) for g in range(len(groups))], stream=stream, **HP)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    n_mats = sum(L for _, L, _, _ in groups)
+    steps_per_s = world * args.steps / (ms / 1e3)
+    gemm_launches = sum(prof[k][0] for k in ("gram", "poly", "update"))
+    gemm_ms = sum(prof[k][1] for k in ("gram", "poly", "update"))
+    flops_timed = ns_flops(groups) * args.steps
+    achieved_tf = flops_timed / (gemm_ms / 1e3) / 1e12
+    burst, sustained = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+    traffic = recorded_traffic(args.workload)
+    mom_launches, mom_ms = prof["momentum"]
+    mom_gbs = momentum_bytes(groups) * args.steps / (mom_ms / 1e3) / 1e9 if mom_ms > 0 else None
+    h2d = sum(L * R * C * 2 for _, L, R, C in groups)
+    d2h = n_mats * 8
+
+    line = {
+        "metric": METRIC, "value": steps_per_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(args),
+        "matrices_per_s": steps_per_s * n_mats,
+        "ns_tflops": achieved_tf,
+        "ns_frac_of_bf16_peak": {"burst": achieved_tf / burst, "sustained": achieved_tf / sustained,
+                                 "source": peak_src},
+        "ns_dense_equivalent_tflops": ns_dense_flops(groups) * args.steps / (gemm_ms / 1e3) / 1e12,
+        "roofline": {"bound": "tensor", "kernel": "ns_gemm_kernel", "achieved": achieved_tf, "peak": burst,
+                     "unit": "TFLOP/s", "frac": achieved_tf / burst,
+                     "peak_kind": f"{peak_src} bf16 burst (cuBLAS 8192^3)",
+                     "traffic": traffic,
+                     "flops_per_launch": flops_timed / max(gemm_launches, 1),
+                     "avg_launch_ms": gemm_ms / max(gemm_launches, 1), "launches": gemm_launches},
+        "momentum_kernel": {"bound": "hbm", "achieved_gbs": mom_gbs, "peak_gbs": peaks["hbm_gbs"],
+                            "frac": (mom_gbs / peaks["hbm_gbs"]) if mom_gbs else None,
+                            "bytes_per_element": 12, "launches": mom_launches},
+        "kernel_ms_per_step": {k: v[1] / args.steps for k, v in prof.items()},
+        "cpu_baseline": cpu,
+        "clocks": clk,
+        "e2e": {"value": world * e2e_steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "entry": "muon_step_groups_host (pinned host G -> device, norms + flags -> host)"},
+        "gpu_launches": sum(v[0] for v in prof.values()),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    mu.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

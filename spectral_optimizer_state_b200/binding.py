@@ -1,0 +1,298 @@
+"""ctypes binding of libmuon (include/muon.h): argument marshalling only.
+
+Every step of the Muon update runs in the CUDA kernels of libmuon.so; this
+module turns torch tensors into raw device pointers and the current CUDA
+stream into a cudaStream_t, and raises on any non-OK status.  There is no
+CPU fallback: without the built library, or without an sm_100 device, every
+call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Iterable, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmuon.so")
+
+MUON_OK = 0
+STATUS_NAMES = {
+    0: "MUON_OK", 1: "MUON_ERR_INVALID_ARG", 2: "MUON_ERR_UNSUPPORTED_SHAPE", 3: "MUON_ERR_DTYPE",
+    4: "MUON_ERR_CUDA", 5: "MUON_ERR_NONFINITE", 6: "MUON_ERR_TIMEOUT", 7: "MUON_ERR_NO_DEVICE",
+    8: "MUON_ERR_ALLOC",
+}
+MUON_BF16, MUON_F32 = 0, 1
+SCALE_SQRT_RATIO, SCALE_NONE, SCALE_RMS_MATCH = 0, 1, 2
+FLAG_NONFINITE = 1
+MAX_BATCH = 256
+MAX_ITERS = 32
+MAX_GROUPS = 8
+QUINTIC = (3.4445, -4.7750, 2.0315)
+CUBIC = (1.5, -0.5, 0.0)
+
+# Every symbol include/muon.h declares.
+EXPORTS = (
+    "muon_abi_version", "muon_status_string", "muon_last_cuda_error", "muon_create", "muon_destroy",
+    "muon_set_coeffs", "muon_get_coeffs", "muon_step", "muon_step_groups", "muon_step_groups_host",
+    "muon_ns_orthogonalize", "muon_get_status", "muon_get_norms", "muon_workspace_bytes",
+    "muon_profile_enable", "muon_profile_read",
+)
+KERNEL_KINDS = ("momentum", "gram", "poly", "update")
+
+
+class MuonError(RuntimeError):
+    def __init__(self, status: int, what: str, detail: str = ""):
+        self.status = status
+        msg = f"{what}: {STATUS_NAMES.get(status, status)}"
+        if detail:
+            msg += f" ({detail})"
+        super().__init__(msg)
+
+
+class Hparams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta", ctypes.c_float), ("weight_decay", ctypes.c_float),
+                ("eps", ctypes.c_float), ("nesterov", ctypes.c_int), ("scale_mode", ctypes.c_int)]
+
+
+class Profile(ctypes.Structure):
+    _fields_ = [("launches", ctypes.c_int * 4), ("ms", ctypes.c_double * 4)]
+
+
+class Group(ctypes.Structure):
+    _fields_ = [("W", ctypes.POINTER(ctypes.c_void_p)), ("G", ctypes.POINTER(ctypes.c_void_p)),
+                ("M", ctypes.POINTER(ctypes.c_void_p)), ("batch", ctypes.c_int),
+                ("rows", ctypes.c_int), ("cols", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+_lib = None
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load libmuon.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(f"libmuon.so not built at {p}: run `python -m spectral_optimizer_state_b200.build`")
+    lib = ctypes.CDLL(p)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    pvp = ctypes.POINTER(ctypes.c_void_p)
+    sig = {
+        "muon_abi_version": (i, []),
+        "muon_status_string": (ctypes.c_char_p, [i]),
+        "muon_last_cuda_error": (ctypes.c_char_p, []),
+        "muon_create": (i, [ctypes.POINTER(vp), i]),
+        "muon_destroy": (i, [vp]),
+        "muon_set_coeffs": (i, [vp, ctypes.POINTER(f), i]),
+        "muon_get_coeffs": (i, [vp, ctypes.POINTER(f), ctypes.POINTER(i)]),
+        "muon_step": (i, [vp, pvp, pvp, pvp, i, i, i, i, ctypes.POINTER(Hparams), vp]),
+        "muon_step_groups": (i, [vp, ctypes.POINTER(Group), i, ctypes.POINTER(Hparams), vp]),
+        "muon_step_groups_host": (i, [vp, ctypes.POINTER(Group), i, ctypes.POINTER(Hparams),
+                                      ctypes.POINTER(f), ctypes.POINTER(i), vp]),
+        "muon_ns_orthogonalize": (i, [vp, pvp, pvp, i, i, i, i, f, vp]),
+        "muon_get_status": (i, [vp, ctypes.POINTER(i), i, ctypes.POINTER(i)]),
+        "muon_get_norms": (i, [vp, ctypes.POINTER(f), i, ctypes.POINTER(i)]),
+        "muon_workspace_bytes": (sz, [vp]),
+        "muon_profile_enable": (i, [vp, i]),
+        "muon_profile_read": (i, [vp, ctypes.POINTER(Profile), i]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _ptrs(tensors: Sequence) -> ctypes.Array:
+    return (ctypes.c_void_p * len(tensors))(*[t.data_ptr() for t in tensors])
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return MUON_BF16
+    if t.dtype == torch.float32:
+        return MUON_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; libmuon takes bfloat16 or float32")
+
+
+def _check_same(ts: Sequence, shape, dtype, device_type: str, what: str):
+    if len(ts) == 0:
+        raise ValueError(f"{what}: empty list")
+    for t in ts:
+        if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+            raise ValueError(f"{what}: every matrix must be {tuple(shape)} {dtype}, got {tuple(t.shape)} {t.dtype}")
+        if t.device.type != device_type:
+            raise ValueError(f"{what}: expected {device_type} tensors, got {t.device}")
+        if not t.is_contiguous():
+            raise ValueError(f"{what}: tensors must be contiguous (row-major)")
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(int(s.cuda_stream))
+
+
+class Muon:
+    """A libmuon context on one CUDA device (owns the workspace and the coefficient table)."""
+
+    def __init__(self, device: int = 0, coeffs: Iterable | None = None):
+        self.lib = load_library()
+        self.device = device
+        h = ctypes.c_void_p()
+        st = self.lib.muon_create(ctypes.byref(h), device)
+        self._check(st, "muon_create")
+        self.handle = h
+        self._keep = []
+        if coeffs is not None:
+            self.set_coeffs(coeffs)
+
+    # -------------------------------------------------------------- helpers
+    def _check(self, st: int, what: str):
+        if st != MUON_OK:
+            detail = ""
+            if st == 4:
+                detail = self.lib.muon_last_cuda_error().decode()
+            raise MuonError(st, what, detail)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            self.lib.muon_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    # -------------------------------------------------------------- coefficients
+    def set_coeffs(self, coeffs: Iterable):
+        flat = [float(v) for abc in coeffs for v in abc]
+        k = len(flat) // 3
+        arr = (ctypes.c_float * len(flat))(*flat)
+        self._check(self.lib.muon_set_coeffs(self.handle, arr, k), "muon_set_coeffs")
+
+    def get_coeffs(self):
+        arr = (ctypes.c_float * (3 * MAX_ITERS))()
+        k = ctypes.c_int()
+        self._check(self.lib.muon_get_coeffs(self.handle, arr, ctypes.byref(k)), "muon_get_coeffs")
+        return [tuple(arr[3 * i:3 * i + 3]) for i in range(k.value)]
+
+    # -------------------------------------------------------------- steps
+    @staticmethod
+    def hparams(lr=0.02, beta=0.95, weight_decay=0.1, eps=1e-7, nesterov=True, scale_mode=SCALE_SQRT_RATIO):
+        return Hparams(float(lr), float(beta), float(weight_decay), float(eps), int(bool(nesterov)), int(scale_mode))
+
+    def _group(self, W, G, M, g_device_type="cuda"):
+        import torch
+        shape, dt = tuple(W[0].shape), W[0].dtype
+        if len(shape) != 2:
+            raise ValueError("matrices must be 2-D")
+        if not (len(W) == len(G) == len(M)):
+            raise ValueError("W, G and M must have the same length")
+        _check_same(W, shape, dt, "cuda", "W")
+        _check_same(G, shape, dt, g_device_type, "G")
+        _check_same(M, shape, torch.float32, "cuda", "M")
+        pw, pg, pm = _ptrs(W), _ptrs(G), _ptrs(M)
+        self._keep = [pw, pg, pm]
+        return Group(pw, pg, pm, len(W), shape[0], shape[1], _dtype_code(W[0])), (pw, pg, pm)
+
+    def step(self, W, G, M, stream=None, **hp):
+        """One Muon step on same-shape matrices W[l] (updated), G[l], M[l] (fp32, updated)."""
+        self.step_groups([(W, G, M)], stream=stream, **hp)
+
+    def step_groups(self, groups, stream=None, **hp):
+        """groups: list of (W list, G list, M list), one entry per shape."""
+        gs, keep = [], []
+        for (W, G, M) in groups:
+            g, k = self._group(W, G, M)
+            gs.append(g)
+            keep.append(k)
+        arr = (Group * len(gs))(*gs)
+        h = self.hparams(**hp)
+        st = self.lib.muon_step_groups(self.handle, arr, len(gs), ctypes.byref(h), _stream_handle(stream))
+        self._check(st, "muon_step_groups")
+
+    def step_groups_host(self, groups, stream=None, **hp):
+        """Like step_groups, but every G is a (pinned) CPU tensor; copies happen inside the call.
+
+        Returns (nu, flags) per matrix in group order, after the stream has completed.
+        """
+        gs, keep = [], []
+        for (W, G, M) in groups:
+            g, k = self._group(W, G, M, g_device_type="cpu")
+            gs.append(g)
+            keep.append(k)
+        n = sum(g.batch for g in gs)
+        nu = (ctypes.c_float * n)()
+        flags = (ctypes.c_int * n)()
+        arr = (Group * len(gs))(*gs)
+        h = self.hparams(**hp)
+        st = self.lib.muon_step_groups_host(self.handle, arr, len(gs), ctypes.byref(h), nu, flags,
+                                            _stream_handle(stream))
+        if st not in (MUON_OK, 5):
+            self._check(st, "muon_step_groups_host")
+        return list(nu), list(flags)
+
+    def ns_orthogonalize(self, X, Out, eps=1e-7, stream=None):
+        """Out[l] = NS_k(X[l] / (||X[l]||_F + eps)) for same-shape matrices (bf16 or fp32)."""
+        shape, dt = tuple(X[0].shape), X[0].dtype
+        _check_same(X, shape, dt, "cuda", "X")
+        _check_same(Out, shape, dt, "cuda", "Out")
+        if len(X) != len(Out):
+            raise ValueError("X and Out must have the same length")
+        px, po = _ptrs(X), _ptrs(Out)
+        st = self.lib.muon_ns_orthogonalize(self.handle, px, po, len(X), shape[0], shape[1],
+                                            _dtype_code(X[0]), float(eps), _stream_handle(stream))
+        self._check(st, "muon_ns_orthogonalize")
+
+    # -------------------------------------------------------------- status
+    def status(self):
+        """(status code, per-matrix flags) of the last call; synchronises its stream."""
+        cap = 8 * MAX_BATCH * MAX_GROUPS
+        flags = (ctypes.c_int * cap)()
+        cnt = ctypes.c_int()
+        st = self.lib.muon_get_status(self.handle, flags, cap, ctypes.byref(cnt))
+        if st not in (MUON_OK, 5, 6):
+            self._check(st, "muon_get_status")
+        return st, list(flags[:cnt.value])
+
+    def norms(self):
+        cap = 8 * MAX_BATCH * MAX_GROUPS
+        nu = (ctypes.c_float * cap)()
+        cnt = ctypes.c_int()
+        self._check(self.lib.muon_get_norms(self.handle, nu, cap, ctypes.byref(cnt)), "muon_get_norms")
+        return list(nu[:cnt.value])
+
+    def workspace_bytes(self) -> int:
+        return int(self.lib.muon_workspace_bytes(self.handle))
+
+    def profile_enable(self, on: bool = True):
+        self._check(self.lib.muon_profile_enable(self.handle, int(bool(on))), "muon_profile_enable")
+
+    def profile_read(self, reset: bool = True):
+        """{kind: (launches, total device ms)} since the last reset; synchronises on the events."""
+        p = Profile()
+        self._check(self.lib.muon_profile_read(self.handle, ctypes.byref(p), int(bool(reset))), "muon_profile_read")
+        return {k: (p.launches[i], p.ms[i]) for i, k in enumerate(KERNEL_KINDS)}
+
+
+def shape_scale(rows: int, cols: int, mode: int = SCALE_SQRT_RATIO) -> float:
+    """The scale the library applies (mirrors the C side, for callers' bookkeeping)."""
+    if mode == SCALE_NONE:
+        return 1.0
+    if mode == SCALE_RMS_MATCH:
+        return 0.2 * math.sqrt(max(rows, cols))
+    return math.sqrt(max(1.0, rows / cols))

@@ -1,0 +1,474 @@
+// The three matrix products of a Newton-Schulz iteration on the tensor cores
+// of sm_100a (tcgen05 + TMEM, operands staged by TMA):
+//
+//   Gram     A = X X^T            M = N = m, K = n, symmetric output
+//   poly     B = b A + c A A      M = N = K = m,   symmetric output
+//   update   X' = a X + B X       M = m, N = n, K = m (B operand MN-major)
+//
+// (MuonSSM: Orthogonalizing State Space Models, section on the lightweight
+// Newton-Schulz step: the orthogonalisation is matrix products only, no SVD;
+// Muon Meets Mamba, abstract: one orthogonalised update per weight matrix.)
+//
+// One persistent kernel serves all three: a CTA owns a 128-row M tile and up
+// to 256 N columns, loops over a static round-robin list of tiles (every
+// matrix of one or two same-phase problems), and runs
+//   warp 0      TMA producer (one thread) into a 4-stage ring of 48 KB stages,
+//   warp 1      TMEM allocation + UMMA issuer (one thread),
+//   warps 2..5  epilogue: TMEM -> registers -> fused arithmetic -> global.
+// Two TMEM accumulators (2 x 256 fp32 columns) let the epilogue of one tile
+// overlap the main loop of the next.  Symmetric outputs are computed on the
+// upper 128 x 128 blocks only (tiles start at the diagonal block) and mirrored.
+// The fp32 path passes three bf16 planes per operand; six plane products
+// (small terms first) are accumulated in the same TMEM tile.
+//
+// Every wait is bounded; a CTA that runs out sets the device status word and
+// unwinds after draining its own copies and MMAs, then frees its TMEM.
+#include <cuda_bf16.h>
+
+#include "device_utils.cuh"
+#include "internal.h"
+
+namespace muon {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int BN = 256;
+constexpr int STAGES = 4;
+constexpr uint32_t A_BYTES = BM * BK * 2;     // 16 KB
+constexpr uint32_t B_BYTES = BN * BK * 2;     // 32 KB
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t KMAJ_BOX_BYTES = 128 * BK * 2;  // box {64 K, 128 rows}
+constexpr uint32_t MNMAJ_BOX_BYTES = 64 * BK * 2;  // box {64 N, 64 K rows}
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COLS = 256;
+constexpr int NUM_BARS = 2 * STAGES + 5;
+constexpr uint32_t BAR_BYTES = 8 * NUM_BARS + 16;
+constexpr uint64_t kDrainLimitNs = 200000000ull;
+
+struct Tile {
+  int pi, l, m0, n0, nw;
+};
+
+__device__ __forceinline__ Tile decode_tile(const GemmParams& P, int t) {
+  Tile ti;
+  ti.pi = (P.nprob > 1 && t >= P.prob[1].tile_base) ? 1 : 0;
+  const GemmProblem& q = P.prob[ti.pi];
+  const int local = t - q.tile_base;
+  ti.l = local / q.tiles_per_matrix;
+  int r = local - ti.l * q.tiles_per_matrix;
+  if (q.sym) {
+    int mb = 0;
+    for (;;) {
+      const int cnt = (q.M - BM * mb + BN - 1) / BN;
+      if (r < cnt) break;
+      r -= cnt;
+      ++mb;
+    }
+    ti.m0 = BM * mb;
+    ti.n0 = BM * mb + BN * r;
+  } else {
+    const int tn = (q.N + BN - 1) / BN;
+    const int mb = r / tn;
+    ti.m0 = BM * mb;
+    ti.n0 = (r - mb * tn) * BN;
+  }
+  const int nw = ((q.N - ti.n0 + 63) / 64) * 64;
+  ti.nw = nw < BN ? nw : BN;
+  return ti;
+}
+
+// Plane pairs of the split products, smallest first: mid*mid, hi*lo, lo*hi,
+// hi*mid, mid*hi, hi*hi (plane 0 = hi, 1 = mid, 2 = lo).
+__device__ __forceinline__ void segment_planes(int nseg, int seg, int& pa, int& pb) {
+  if (nseg == 1) {
+    pa = 0;
+    pb = 0;
+    return;
+  }
+  // nibble seg of each constant: a planes {1,0,2,0,1,0}, b planes {1,2,0,1,0,0}
+  pa = (0x10201 >> (4 * seg)) & 0xF;
+  pb = (0x01021 >> (4 * seg)) & 0xF;
+}
+
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kDrainLimitNs) return false;
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ epilogue
+__device__ __forceinline__ void unpack_bf16x8(uint4 q, float* v) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  return static_cast<uint32_t>(float_to_bf16_bits(a)) |
+         (static_cast<uint32_t>(float_to_bf16_bits(b)) << 16);
+}
+
+// v[t] += beta * sum_p cin_p(row, j0 + t) for t < nv
+__device__ __forceinline__ void add_cin(const GemmProblem& q, int l, int row, int j0, int nv,
+                                        float (&v)[32]) {
+  float c[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) c[t] = 0.f;
+  for (int p = 0; p < q.planes; ++p) {
+    const uint16_t* src = q.cin + p * q.cin_plane + l * q.cin_mat +
+                          static_cast<long long>(row) * q.cin_pitch + j0;
+    if (nv == 32) {
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        float f[8];
+        unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(src) + h), f);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) c[8 * h + t] += f[t];
+      }
+    } else {
+#pragma unroll
+      for (int t = 0; t < 32; ++t)
+        if (t < nv) c[t] += bf16_bits_to_float(src[t]);
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < 32; ++t) v[t] = fmaf(q.beta, c[t], v[t]);
+}
+
+template <int PLANES>
+__device__ __forceinline__ void store_tile_row(const GemmProblem& q, int l, int row, int j0, int nv,
+                                               const float (&v)[32], bool mirror) {
+  uint16_t* base = q.out + l * q.out_mat;
+  if (nv == 32) {
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      uint32_t w[PLANES][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint16_t a[PLANES], b[PLANES];
+        split_planes<PLANES>(v[8 * h + 2 * i], a);
+        split_planes<PLANES>(v[8 * h + 2 * i + 1], b);
+#pragma unroll
+        for (int p = 0; p < PLANES; ++p)
+          w[p][i] = static_cast<uint32_t>(a[p]) | (static_cast<uint32_t>(b[p]) << 16);
+      }
+#pragma unroll
+      for (int p = 0; p < PLANES; ++p) {
+        uint16_t* dst = base + p * q.out_plane + static_cast<long long>(row) * q.out_pitch + j0 + 8 * h;
+        *reinterpret_cast<uint4*>(dst) = make_uint4(w[p][0], w[p][1], w[p][2], w[p][3]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      if (t >= nv) continue;
+      uint16_t a[PLANES];
+      split_planes<PLANES>(v[t], a);
+#pragma unroll
+      for (int p = 0; p < PLANES; ++p)
+        base[p * q.out_plane + static_cast<long long>(row) * q.out_pitch + j0 + t] = a[p];
+    }
+  }
+  if (mirror) {
+    // (row, j) -> (j, row): lanes hold consecutive rows, so each store is coalesced.
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      if (t >= nv) continue;
+      uint16_t a[PLANES];
+      split_planes<PLANES>(v[t], a);
+#pragma unroll
+      for (int p = 0; p < PLANES; ++p)
+        base[p * q.out_plane + static_cast<long long>(j0 + t) * q.out_pitch + row] = a[p];
+    }
+  }
+}
+
+// W (or Out) element of wide position (row, j).
+__device__ __forceinline__ long long w_index(const GemmProblem& q, int row, int j) {
+  return q.transposed ? static_cast<long long>(j) * q.wcols + row
+                      : static_cast<long long>(row) * q.wcols + j;
+}
+
+__device__ __forceinline__ void write_caller(const GemmProblem& q, int l, int row, int j0, int nv,
+                                             const float (&v)[32], bool apply) {
+  void* w = q.wtab[l];
+  const bool vec = q.w_vec && !q.transposed && nv == 32;
+  if (q.w_f32) {
+    float* W = static_cast<float*>(w);
+    if (vec) {
+      float4* p4 = reinterpret_cast<float4*>(W + w_index(q, row, j0));
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        float4 o = make_float4(v[4 * h], v[4 * h + 1], v[4 * h + 2], v[4 * h + 3]);
+        if (apply) {
+          const float4 c = p4[h];
+          o.x = fmaf(q.decay, c.x, -q.lrs * o.x);
+          o.y = fmaf(q.decay, c.y, -q.lrs * o.y);
+          o.z = fmaf(q.decay, c.z, -q.lrs * o.z);
+          o.w = fmaf(q.decay, c.w, -q.lrs * o.w);
+        }
+        p4[h] = o;
+      }
+    } else {
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        if (t >= nv) continue;
+        const long long e = w_index(q, row, j0 + t);
+        W[e] = apply ? fmaf(q.decay, W[e], -q.lrs * v[t]) : v[t];
+      }
+    }
+  } else {
+    uint16_t* W = static_cast<uint16_t*>(w);
+    if (vec) {
+      uint4* p4 = reinterpret_cast<uint4*>(W + w_index(q, row, j0));
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        float o[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) o[t] = v[8 * h + t];
+        if (apply) {
+          float c[8];
+          unpack_bf16x8(p4[h], c);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) o[t] = fmaf(q.decay, c[t], -q.lrs * o[t]);
+        }
+        p4[h] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                           pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+      }
+    } else {
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        if (t >= nv) continue;
+        const long long e = w_index(q, row, j0 + t);
+        const float o = apply ? fmaf(q.decay, bf16_bits_to_float(W[e]), -q.lrs * v[t]) : v[t];
+        W[e] = float_to_bf16_bits(o);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void epilogue_chunk(const GemmProblem& q, const Tile& ti, int row,
+                                               int j0, const uint32_t (&r)[32], float sl,
+                                               bool skip) {
+  if (row >= q.M || j0 >= q.N) return;
+  const int nv = min(32, q.N - j0);
+  float v[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) v[t] = q.alpha * __uint_as_float(r[t]);
+  if (q.cin != nullptr) add_cin(q, ti.l, row, j0, nv, v);
+#pragma unroll
+  for (int t = 0; t < 32; ++t) v[t] *= sl;
+  if (q.epi == EPI_STORE) {
+    const bool mirror = q.sym && (j0 >= ti.m0 + BM);
+    if (q.planes == 3) store_tile_row<3>(q, ti.l, row, j0, nv, v, mirror);
+    else store_tile_row<1>(q, ti.l, row, j0, nv, v, mirror);
+  } else if (!skip) {
+    write_caller(q, ti.l, row, j0, nv, v, q.epi == EPI_APPLY);
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+__global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_constant__ GemmParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t bar0 = base + STAGES * STAGE_BYTES;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 8 * NUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 128);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < P.nprob; ++i) {
+      tma_prefetch_map(&P.prob[i].tmA);
+      tma_prefetch_map(&P.prob[i].tmB);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < P.total_tiles; t += gridDim.x) {
+        const Tile ti = decode_tile(P, t);
+        const GemmProblem& q = P.prob[ti.pi];
+        const int nk = q.k_tiles * q.nseg;
+        const uint32_t bbytes = q.b_mn_major ? static_cast<uint32_t>(ti.nw / 64) * MNMAJ_BOX_BYTES
+                                             : static_cast<uint32_t>((ti.nw + 127) / 128) * KMAJ_BOX_BYTES;
+        for (int kk = 0; kk < nk; ++kk, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, P.status)) {
+            ok = false;
+            break;
+          }
+          const int seg = kk / q.k_tiles;
+          const int kb = kk - seg * q.k_tiles;
+          int pa, pb;
+          segment_planes(q.nseg, seg, pa, pb);
+          const uint32_t sa = base + s * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+          mbar_arrive_expect_tx(full_bar(s), A_BYTES + bbytes);
+          tma_load_4d(sa, &q.tmA, full_bar(s), kb * BK, ti.m0, ti.l, pa);
+          if (q.b_mn_major) {
+            for (int c = 0; c < ti.nw / 64; ++c)
+              tma_load_4d(sb + c * MNMAJ_BOX_BYTES, &q.tmB, full_bar(s), ti.n0 + 64 * c, kb * BK, ti.l, pb);
+          } else {
+            for (int h = 0; h < (ti.nw + 127) / 128; ++h)
+              tma_load_4d(sb + h * KMAJ_BOX_BYTES, &q.tmB, full_bar(s), kb * BK, ti.n0 + 128 * h, ti.l, pb);
+          }
+        }
+      }
+      if (!ok) {
+        // Let the copies this thread started land before the CTA exits.
+        const uint32_t n = it < STAGES ? it : STAGES;
+        for (uint32_t j = it - n; j < it; ++j) wait_drain(full_bar(j % STAGES), (j / STAGES) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      uint32_t it = 0;
+      int local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < P.total_tiles; t += gridDim.x, ++local) {
+        const Tile ti = decode_tile(P, t);
+        const GemmProblem& q = P.prob[ti.pi];
+        const int acc = local & 1;
+        const uint32_t aph = (local >> 1) & 1;
+        if (!mbar_wait_bounded(tempty_bar(acc), aph ^ 1u, abort_flag, P.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        const uint32_t idesc = instr_desc_bf16(BM, ti.nw, q.b_mn_major != 0);
+        const int nk = q.k_tiles * q.nseg;
+        for (int kk = 0; kk < nk; ++kk, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, P.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base + s * STAGE_BYTES;
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int k4 = 0; k4 < BK / 16; ++k4) {
+            const uint64_t ad = smem_desc_sw128(sa + 32u * k4, 16u, 1024u);
+            const uint64_t bd = q.b_mn_major ? smem_desc_sw128(sb + 2048u * k4, MNMAJ_BOX_BYTES, 1024u)
+                                             : smem_desc_sw128(sb + 32u * k4, 16u, 1024u);
+            tc_mma_bf16(d_tmem, ad, bd, idesc, (kk | k4) != 0 ? 1u : 0u);
+          }
+          tc_commit(empty_bar(s));
+        }
+        if (ok) tc_commit(tfull_bar(acc));
+      }
+      if (!ok) {
+        tc_commit(drain_bar);
+        wait_drain(drain_bar, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5)
+    const int quarter = warp & 3;  // TMEM lanes this warp may read
+    int local = 0;
+    for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++local) {
+      const Tile ti = decode_tile(P, t);
+      const GemmProblem& q = P.prob[ti.pi];
+      const int acc = local & 1;
+      const uint32_t aph = (local >> 1) & 1;
+      if (!mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, P.status)) break;
+      tc_fence_after();
+      const int row = ti.m0 + 32 * quarter + lane;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * ACC_COLS;
+      const float sl = q.mat_scale != nullptr ? q.mat_scale[ti.l] : 1.0f;
+      const bool skip = q.epi == EPI_APPLY && q.flags != nullptr && q.flags[q.flag_offset + ti.l] != 0;
+      for (int c = 0; c < ti.nw; c += 32) {
+        uint32_t r[32];
+        __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the guarded stores
+        tmem_load_32cols(tbase + c, r);
+        tmem_load_wait();
+        epilogue_chunk(q, ti, row, ti.n0 + c, r, sl, skip);
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+size_t gemm_smem_bytes() { return STAGES * STAGE_BYTES + BAR_BYTES + 1024; }
+
+int gemm_tiles_per_matrix(int M, int N, int sym) {
+  if (sym) {
+    int n = 0;
+    for (int mb = 0; mb * BM < M; ++mb) n += (M - BM * mb + BN - 1) / BN;
+    return n;
+  }
+  return ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+}
+
+cudaError_t launch_gemm(const GemmParams& p, int grid, cudaStream_t stream) {
+  static int configured_device = -1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (configured_device != dev) {
+    e = cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(gemm_smem_bytes()));
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  ns_gemm_kernel<<<grid, THREADS, gemm_smem_bytes(), stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace muon

@@ -1,0 +1,96 @@
+// Structures shared by the host side of libmuon and its kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/muon.h"
+
+namespace muon {
+
+// ------------------------------------------------------------------ K1
+// Momentum + Nesterov + Frobenius norm, writes X0 (un-normalised U) in the
+// wide orientation into the workspace as PLANES bf16 planes.
+struct MomentumParams {
+  const void* g[MUON_MAX_BATCH];  // rows x cols, bf16 or fp32
+  float* m[MUON_MAX_BATCH];       // rows x cols fp32 (null when no momentum)
+  uint16_t* x;                    // [planes][batch][mrows][pitch] bf16 bits
+  long long x_plane;              // elements between planes
+  long long x_mat;                // elements between matrices
+  int pitch;                      // wide row pitch (elements), multiple of 8
+  int rows, cols;                 // of G / M (row-major)
+  float beta;
+  int nesterov;
+  float eps;
+  int nblk;                       // blocks per matrix (gridDim.x)
+  float* partials;                // [batch][nblk]
+  unsigned int* counters;         // [batch], zero between calls
+  float* nu;                      // [batch] ||U||_F
+  float* scale1;                  // [batch] 1/(nu+eps)
+  float* scale2;                  // [batch] scale1^2
+  int* flags;                     // [batch]
+};
+
+// Launch K1 for one group; mode bits choose the kernel instance.
+cudaError_t launch_momentum(const MomentumParams& p, int batch, bool g_is_f32, bool momentum,
+                            int planes, cudaStream_t stream);
+
+// Number of blocks per matrix K1 uses for a rows x cols matrix.
+int momentum_blocks_per_matrix(int rows, int cols);
+
+// ------------------------------------------------------------------ GEMM
+enum EpilogueKind : int {
+  EPI_STORE = 0,  // out = s_l * (alpha*acc + beta*cin), written as planes (and mirrored if sym)
+  EPI_APPLY = 1,  // O = s_l*(alpha*acc + beta*cin); W <- decay*W - lrs*O (oriented)
+  EPI_OUT = 2,    // O as above written to a caller matrix (oriented)
+};
+
+constexpr int kMaxProblems = 2;
+
+struct alignas(64) GemmProblem {
+  CUtensorMap tmA;  // A operand [planes][L][M][K], K contiguous, box {64, 128}
+  CUtensorMap tmB;  // B operand: K-major [planes][L][N][K] box {64,128}, or
+                    //            MN-major [planes][L][K][N] box {64, 64}
+  int M, N, K, L;
+  int nseg;          // 1 (bf16) or 6 (three-plane split)
+  int b_mn_major;    // 0: B stored N x K; 1: B stored K x N
+  int sym;           // output symmetric: compute upper tiles only, mirror the rest
+  int epi;           // EpilogueKind
+  int tiles_per_matrix;
+  int tile_base;     // first global tile index of this problem
+  int k_tiles;       // ceil(K / 64)
+  int planes;        // planes of out / cin (1 or 3)
+  float alpha, beta;
+  const float* mat_scale;  // per-matrix factor s_l, or null for 1
+  uint16_t* out;           // [planes][L][M][out_pitch] (EPI_STORE)
+  long long out_plane, out_mat;
+  int out_pitch;
+  const uint16_t* cin;     // [planes][L][M][cin_pitch], null when beta == 0
+  long long cin_plane, cin_mat;
+  int cin_pitch;
+  // EPI_APPLY / EPI_OUT: caller matrices, rows x cols row-major (W dims)
+  int wrows, wcols;
+  int transposed;          // wide O(i,j) lands at W(j,i)
+  int w_f32;               // 1: fp32 W/Out, 0: bf16
+  int w_vec;               // rows of W are 16-byte aligned for vector access
+  float decay, lrs;        // W <- decay*W - lrs*O
+  const int* flags;        // skip matrices whose flag is set (EPI_APPLY)
+  int flag_offset;
+  void* wtab[MUON_MAX_BATCH];
+};
+
+struct GemmParams {
+  GemmProblem prob[kMaxProblems];
+  int nprob;
+  int total_tiles;
+  int* status;
+};
+
+size_t gemm_smem_bytes();
+cudaError_t launch_gemm(const GemmParams& p, int grid, cudaStream_t stream);
+
+// Tiles one matrix of this problem shape contributes.
+int gemm_tiles_per_matrix(int M, int N, int sym);
+
+}  // namespace muon

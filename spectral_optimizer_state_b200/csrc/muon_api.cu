@@ -1,0 +1,672 @@
+// C-ABI of libmuon: argument checks, workspace, tensor maps and the launch
+// sequence of one Muon step (momentum pass, k Newton-Schulz iterations of
+// three tensor-core products each, the last one applying the update).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/muon.h"
+#include "device_utils.cuh"
+#include "internal.h"
+
+using namespace muon;
+
+namespace {
+
+// ------------------------------------------------------------------ errors
+char g_cuda_error[256] = "";
+std::mutex g_err_mu;
+
+muon_status cuda_fail(cudaError_t e, const char* what) {
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  std::snprintf(g_cuda_error, sizeof(g_cuda_error), "%s: %s", what, cudaGetErrorString(e));
+  return MUON_ERR_CUDA;
+}
+
+#define MUON_CUDA(call, what)                          \
+  do {                                                 \
+    cudaError_t _e = (call);                           \
+    if (_e != cudaSuccess) return cuda_fail(_e, what); \
+  } while (0)
+
+// ------------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 buffer [planes][L][rows][pitch] viewed as 4-D {cols, rows, L, planes};
+// box {box_cols, box_rows}, 128-byte swizzle, out-of-range reads give zeros.
+bool encode_map(CUtensorMap* map, const void* base, int cols, int rows, int L, int planes,
+                int pitch, int box_cols, int box_rows) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(planes)};
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(pitch) * 2;
+  cuuint64_t strides[3] = {row_bytes, row_bytes * rows, row_bytes * rows * L};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+constexpr float kQuintic[3] = {3.4445f, -4.7750f, 2.0315f};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int round8(int x) { return (x + 7) / 8 * 8; }
+
+// One group as the kernels see it.
+struct GroupPlan {
+  const void* const* g;  // device pointers (G or X)
+  float* const* m;       // null for orthogonalise-only
+  void* const* w;        // W (step) or Out (orthogonalise)
+  int batch, rows, cols, f32, planes;
+  int m_rows, n_cols, transposed, pitch_n, pitch_m, nblk;
+  long long x_mat, x_plane, a_mat, a_plane;  // elements
+  size_t off_x[2], off_a, off_b;             // bytes into the workspace
+  int mat_off, part_off;
+};
+
+}  // namespace
+
+struct muon_ctx {
+  int device = 0;
+  int sm_count = 148;
+  float coeffs[3 * MUON_MAX_ITERS];
+  int k = 5;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  // per-matrix arrays
+  int cap_mats = 0;
+  size_t cap_parts = 0;
+  float* d_nu = nullptr;
+  float* d_s1 = nullptr;
+  float* d_s2 = nullptr;
+  int* d_flags = nullptr;
+  unsigned* d_counters = nullptr;
+  float* d_partials = nullptr;
+  int* d_status = nullptr;
+  int last_count = 0;
+  cudaStream_t last_stream = nullptr;
+  bool pending = false;
+  // device staging for gradients that arrive from host memory
+  void* d_stage = nullptr;
+  size_t stage_bytes = 0;
+  // per-launch timing
+  bool profiling = false;
+  std::vector<cudaEvent_t> events;  // pool, two per recorded launch
+  std::vector<int> rec_kind;        // kind of recorded launch i (events 2i, 2i+1)
+};
+
+namespace {
+
+// Record the start event of a profiled launch; returns the slot or -1.
+int prof_begin(muon_ctx* c, int kind, cudaStream_t s) {
+  if (!c->profiling) return -1;
+  const size_t slot = c->rec_kind.size();
+  while (c->events.size() < 2 * (slot + 1)) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return -1;
+    c->events.push_back(e);
+  }
+  c->rec_kind.push_back(kind);
+  cudaEventRecord(c->events[2 * slot], s);
+  return static_cast<int>(slot);
+}
+
+void prof_end(muon_ctx* c, int slot, cudaStream_t s) {
+  if (slot >= 0) cudaEventRecord(c->events[2 * slot + 1], s);
+}
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    if (prev != dev) cudaSetDevice(dev);
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+bool finite(float x) { return std::isfinite(x); }
+
+muon_status check_hparams(const muon_hparams* hp) {
+  if (!hp) return MUON_ERR_INVALID_ARG;
+  if (!finite(hp->lr) || !finite(hp->beta) || !finite(hp->weight_decay) || !finite(hp->eps))
+    return MUON_ERR_INVALID_ARG;
+  if (hp->eps < 0.f) return MUON_ERR_INVALID_ARG;
+  if (hp->scale_mode < MUON_SCALE_SQRT_RATIO || hp->scale_mode > MUON_SCALE_RMS_MATCH)
+    return MUON_ERR_INVALID_ARG;
+  return MUON_OK;
+}
+
+muon_status check_group(const muon_group& g, bool need_m) {
+  if (g.dtype != MUON_BF16 && g.dtype != MUON_F32) return MUON_ERR_DTYPE;
+  if (g.batch < 1 || g.batch > MUON_MAX_BATCH) return MUON_ERR_INVALID_ARG;
+  if (g.rows < 1 || g.cols < 1) return MUON_ERR_INVALID_ARG;
+  if (g.rows > 32768 || g.cols > 32768 || std::min(g.rows, g.cols) > 8192)
+    return MUON_ERR_UNSUPPORTED_SHAPE;
+  if (!g.W || !g.G || (need_m && !g.M)) return MUON_ERR_INVALID_ARG;
+  for (int l = 0; l < g.batch; ++l) {
+    if (!g.W[l] || !g.G[l] || (need_m && !g.M[l])) return MUON_ERR_INVALID_ARG;
+  }
+  return MUON_OK;
+}
+
+float shape_scale(int rows, int cols, int mode) {
+  switch (mode) {
+    case MUON_SCALE_NONE: return 1.0f;
+    case MUON_SCALE_RMS_MATCH: return 0.2f * std::sqrt(static_cast<float>(std::max(rows, cols)));
+    default: return std::sqrt(std::max(1.0f, static_cast<float>(rows) / static_cast<float>(cols)));
+  }
+}
+
+// Make sure the workspace and the per-matrix arrays can hold `plans`.
+muon_status reserve(muon_ctx* c, std::vector<GroupPlan>& plans, cudaStream_t s) {
+  size_t bytes = 0;
+  int mats = 0;
+  size_t parts = 0;
+  for (auto& p : plans) {
+    const size_t xb = static_cast<size_t>(p.x_plane) * p.planes * 2;
+    const size_t ab = static_cast<size_t>(p.a_plane) * p.planes * 2;
+    p.off_x[0] = bytes; bytes = align_up(bytes + xb, 256);
+    p.off_x[1] = bytes; bytes = align_up(bytes + xb, 256);
+    p.off_a = bytes; bytes = align_up(bytes + ab, 256);
+    p.off_b = bytes; bytes = align_up(bytes + ab, 256);
+    p.mat_off = mats;
+    mats += p.batch;
+    p.part_off = static_cast<int>(parts);
+    parts += static_cast<size_t>(p.batch) * p.nblk;
+  }
+  if (bytes > c->ws_bytes) {
+    MUON_CUDA(cudaDeviceSynchronize(), "sync before workspace growth");
+    if (c->ws) cudaFree(c->ws);
+    c->ws = nullptr;
+    c->ws_bytes = 0;
+    if (cudaMalloc(&c->ws, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return MUON_ERR_ALLOC;
+    }
+    c->ws_bytes = bytes;
+  }
+  if (mats > c->cap_mats || parts > c->cap_parts) {
+    MUON_CUDA(cudaDeviceSynchronize(), "sync before array growth");
+    cudaFree(c->d_nu); cudaFree(c->d_s1); cudaFree(c->d_s2); cudaFree(c->d_flags);
+    cudaFree(c->d_counters); cudaFree(c->d_partials);
+    c->d_nu = c->d_s1 = c->d_s2 = c->d_partials = nullptr;
+    c->d_flags = nullptr;
+    c->d_counters = nullptr;
+    const int cm = std::max(mats, c->cap_mats);
+    const size_t cp = std::max(parts, c->cap_parts);
+    bool ok = cudaMalloc(&c->d_nu, cm * sizeof(float)) == cudaSuccess &&
+              cudaMalloc(&c->d_s1, cm * sizeof(float)) == cudaSuccess &&
+              cudaMalloc(&c->d_s2, cm * sizeof(float)) == cudaSuccess &&
+              cudaMalloc(&c->d_flags, cm * sizeof(int)) == cudaSuccess &&
+              cudaMalloc(&c->d_counters, cm * sizeof(unsigned)) == cudaSuccess &&
+              cudaMalloc(&c->d_partials, cp * sizeof(float)) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      c->cap_mats = 0;
+      c->cap_parts = 0;
+      return MUON_ERR_ALLOC;
+    }
+    MUON_CUDA(cudaMemset(c->d_counters, 0, cm * sizeof(unsigned)), "clear counters");
+    MUON_CUDA(cudaMemset(c->d_flags, 0, cm * sizeof(int)), "clear flags");
+    c->cap_mats = cm;
+    c->cap_parts = cp;
+  }
+  return MUON_OK;
+}
+
+GroupPlan plan_group(const muon_group& g) {
+  GroupPlan p{};
+  p.g = g.G;
+  p.m = g.M;
+  p.w = g.W;
+  p.batch = g.batch;
+  p.rows = g.rows;
+  p.cols = g.cols;
+  p.f32 = g.dtype == MUON_F32;
+  p.planes = p.f32 ? 3 : 1;
+  p.transposed = g.rows > g.cols;
+  p.m_rows = std::min(g.rows, g.cols);
+  p.n_cols = std::max(g.rows, g.cols);
+  p.pitch_n = round8(p.n_cols);
+  p.pitch_m = round8(p.m_rows);
+  p.nblk = momentum_blocks_per_matrix(g.rows, g.cols);
+  p.x_mat = static_cast<long long>(p.m_rows) * p.pitch_n;
+  p.x_plane = p.x_mat * p.batch;
+  p.a_mat = static_cast<long long>(p.m_rows) * p.pitch_m;
+  p.a_plane = p.a_mat * p.batch;
+  return p;
+}
+
+uint16_t* ws_at(muon_ctx* c, size_t off) {
+  return reinterpret_cast<uint16_t*>(static_cast<char*>(c->ws) + off);
+}
+
+enum Phase { PH_GRAM, PH_POLY, PH_UPDATE };
+
+// Fill one GEMM problem for group p, phase ph of iteration `it`.
+bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, bool last, bool step,
+                  const muon_hparams* hp, GemmProblem& q) {
+  std::memset(static_cast<void*>(&q), 0, sizeof(q));
+  const float a = c->coeffs[3 * it], b = c->coeffs[3 * it + 1], cc = c->coeffs[3 * it + 2];
+  const int src = it & 1, dst = (it + 1) & 1;
+  uint16_t* X = ws_at(c, p.off_x[src]);
+  uint16_t* Xn = ws_at(c, p.off_x[dst]);
+  uint16_t* A = ws_at(c, p.off_a);
+  uint16_t* B = ws_at(c, p.off_b);
+  const int m = p.m_rows, n = p.n_cols;
+  q.L = p.batch;
+  q.nseg = p.planes == 3 ? 6 : 1;
+  q.planes = p.planes;
+  q.flags = c->d_flags;
+  q.flag_offset = p.mat_off;
+  switch (ph) {
+    case PH_GRAM:
+      if (!encode_map(&q.tmA, X, n, m, p.batch, p.planes, p.pitch_n, 64, 128)) return false;
+      q.tmB = q.tmA;
+      q.M = m; q.N = m; q.K = n;
+      q.b_mn_major = 0; q.sym = 1; q.epi = EPI_STORE;
+      q.alpha = 1.f; q.beta = 0.f;
+      q.mat_scale = it == 0 ? c->d_s2 + p.mat_off : nullptr;
+      q.out = A; q.out_plane = p.a_plane; q.out_mat = p.a_mat; q.out_pitch = p.pitch_m;
+      break;
+    case PH_POLY:
+      if (!encode_map(&q.tmA, A, m, m, p.batch, p.planes, p.pitch_m, 64, 128)) return false;
+      q.tmB = q.tmA;
+      q.M = m; q.N = m; q.K = m;
+      q.b_mn_major = 0; q.sym = 1; q.epi = EPI_STORE;
+      q.alpha = cc; q.beta = b;
+      q.cin = A; q.cin_plane = p.a_plane; q.cin_mat = p.a_mat; q.cin_pitch = p.pitch_m;
+      q.out = B; q.out_plane = p.a_plane; q.out_mat = p.a_mat; q.out_pitch = p.pitch_m;
+      break;
+    case PH_UPDATE: {
+      const bool have_poly = cc != 0.f;
+      if (!encode_map(&q.tmA, have_poly ? B : A, m, m, p.batch, p.planes, p.pitch_m, 64, 128)) return false;
+      if (!encode_map(&q.tmB, X, n, m, p.batch, p.planes, p.pitch_n, 64, 64)) return false;
+      q.M = m; q.N = n; q.K = m;
+      q.b_mn_major = 1; q.sym = 0;
+      q.alpha = have_poly ? 1.f : b;
+      q.beta = a;
+      q.mat_scale = it == 0 ? c->d_s1 + p.mat_off : nullptr;
+      q.cin = X; q.cin_plane = p.x_plane; q.cin_mat = p.x_mat; q.cin_pitch = p.pitch_n;
+      if (!last) {
+        q.epi = EPI_STORE;
+        q.out = Xn; q.out_plane = p.x_plane; q.out_mat = p.x_mat; q.out_pitch = p.pitch_n;
+      } else {
+        q.epi = step ? EPI_APPLY : EPI_OUT;
+        q.wrows = p.rows; q.wcols = p.cols; q.transposed = p.transposed; q.w_f32 = p.f32;
+        bool vec = (p.cols % (p.f32 ? 4 : 8)) == 0;
+        for (int l = 0; l < p.batch; ++l) {
+          q.wtab[l] = p.w[l];
+          if (reinterpret_cast<uintptr_t>(p.w[l]) % 16) vec = false;
+        }
+        q.w_vec = vec;
+        if (step) {
+          q.decay = 1.0f - hp->lr * hp->weight_decay;
+          q.lrs = hp->lr * shape_scale(p.rows, p.cols, hp->scale_mode);
+        }
+      }
+      break;
+    }
+  }
+  q.tiles_per_matrix = gemm_tiles_per_matrix(q.M, q.N, q.sym);
+  q.k_tiles = (q.K + 63) / 64;
+  return true;
+}
+
+muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* hp, bool step,
+                float eps, cudaStream_t s) {
+  muon_status st = reserve(c, plans, s);
+  if (st != MUON_OK) return st;
+  int total = 0;
+  for (auto& p : plans) total += p.batch;
+  MUON_CUDA(cudaMemsetAsync(c->d_status, 0, sizeof(int), s), "clear status");
+
+  // K1: momentum / look-ahead / norm, one launch per group.
+  for (auto& p : plans) {
+    MomentumParams mp;
+    std::memset(static_cast<void*>(&mp), 0, sizeof(mp));
+    for (int l = 0; l < p.batch; ++l) {
+      mp.g[l] = p.g[l];
+      mp.m[l] = step ? p.m[l] : nullptr;
+    }
+    mp.x = ws_at(c, p.off_x[0]);
+    mp.x_plane = p.x_plane;
+    mp.x_mat = p.x_mat;
+    mp.pitch = p.pitch_n;
+    mp.rows = p.rows;
+    mp.cols = p.cols;
+    mp.beta = step ? hp->beta : 0.f;
+    mp.nesterov = step ? hp->nesterov : 0;
+    mp.eps = eps;
+    mp.nblk = p.nblk;
+    mp.partials = c->d_partials + p.part_off;
+    mp.counters = c->d_counters + p.mat_off;
+    mp.nu = c->d_nu + p.mat_off;
+    mp.scale1 = c->d_s1 + p.mat_off;
+    mp.scale2 = c->d_s2 + p.mat_off;
+    mp.flags = c->d_flags + p.mat_off;
+    const int slot = prof_begin(c, MUON_KERNEL_MOMENTUM, s);
+    MUON_CUDA(launch_momentum(mp, p.batch, p.f32 != 0, step, p.planes, s), "momentum kernel");
+    prof_end(c, slot, s);
+  }
+
+  // k Newton-Schulz iterations; each phase covers up to two groups per launch.
+  GemmParams gp;
+  for (int it = 0; it < c->k; ++it) {
+    const bool last = it == c->k - 1;
+    const bool have_poly = c->coeffs[3 * it + 2] != 0.f;
+    for (int ph = PH_GRAM; ph <= PH_UPDATE; ++ph) {
+      if (ph == PH_POLY && !have_poly) continue;
+      for (size_t g0 = 0; g0 < plans.size(); g0 += kMaxProblems) {
+        std::memset(static_cast<void*>(&gp), 0, sizeof(gp));
+        gp.status = c->d_status;
+        int tiles = 0;
+        for (size_t g = g0; g < std::min(plans.size(), g0 + kMaxProblems); ++g) {
+          GemmProblem& q = gp.prob[gp.nprob];
+          if (!fill_problem(c, plans[g], static_cast<Phase>(ph), it, last, step, hp, q))
+            return cuda_fail(cudaErrorInvalidValue, "tensor map encoding");
+          q.tile_base = tiles;
+          tiles += q.tiles_per_matrix * q.L;
+          ++gp.nprob;
+        }
+        gp.total_tiles = tiles;
+        const int grid = std::min(tiles, c->sm_count);
+        const int slot = prof_begin(c, MUON_KERNEL_GRAM + (ph - PH_GRAM), s);
+        MUON_CUDA(launch_gemm(gp, grid, s), "newton-schulz gemm");
+        prof_end(c, slot, s);
+      }
+    }
+  }
+  c->last_count = total;
+  c->last_stream = s;
+  c->pending = true;
+  return MUON_OK;
+}
+
+muon_status validate_and_plan(muon_ctx* c, const muon_group* groups, int ngroups, bool step,
+                              std::vector<GroupPlan>& plans) {
+  if (!c || !groups || ngroups < 1 || ngroups > MUON_MAX_GROUPS) return MUON_ERR_INVALID_ARG;
+  plans.clear();
+  for (int i = 0; i < ngroups; ++i) {
+    muon_status st = check_group(groups[i], step);
+    if (st != MUON_OK) return st;
+    plans.push_back(plan_group(groups[i]));
+  }
+  return MUON_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+int muon_abi_version(void) { return MUON_ABI_VERSION; }
+
+const char* muon_status_string(muon_status s) {
+  switch (s) {
+    case MUON_OK: return "MUON_OK";
+    case MUON_ERR_INVALID_ARG: return "MUON_ERR_INVALID_ARG";
+    case MUON_ERR_UNSUPPORTED_SHAPE: return "MUON_ERR_UNSUPPORTED_SHAPE";
+    case MUON_ERR_DTYPE: return "MUON_ERR_DTYPE";
+    case MUON_ERR_CUDA: return "MUON_ERR_CUDA";
+    case MUON_ERR_NONFINITE: return "MUON_ERR_NONFINITE";
+    case MUON_ERR_TIMEOUT: return "MUON_ERR_TIMEOUT";
+    case MUON_ERR_NO_DEVICE: return "MUON_ERR_NO_DEVICE";
+    case MUON_ERR_ALLOC: return "MUON_ERR_ALLOC";
+  }
+  return "MUON_ERR_UNKNOWN";
+}
+
+const char* muon_last_cuda_error(void) { return g_cuda_error; }
+
+muon_status muon_create(muon_ctx** out, int device) {
+  if (!out) return MUON_ERR_INVALID_ARG;
+  *out = nullptr;
+  int n = 0;
+  if (cudaGetDeviceCount(&n) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return MUON_ERR_NO_DEVICE;
+  }
+  if (device < 0 || device >= n) return MUON_ERR_INVALID_ARG;
+  cudaDeviceProp prop;
+  MUON_CUDA(cudaGetDeviceProperties(&prop, device), "device properties");
+  if (prop.major != 10) return MUON_ERR_NO_DEVICE;
+  if (!get_encoder()) return MUON_ERR_NO_DEVICE;
+  DeviceGuard guard(device);
+  muon_ctx* c = new muon_ctx();
+  c->device = device;
+  c->sm_count = prop.multiProcessorCount;
+  for (int i = 0; i < 5; ++i) std::memcpy(&c->coeffs[3 * i], kQuintic, sizeof(kQuintic));
+  c->k = 5;
+  if (cudaMalloc(&c->d_status, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    delete c;
+    return MUON_ERR_ALLOC;
+  }
+  cudaMemset(c->d_status, 0, sizeof(int));
+  *out = c;
+  return MUON_OK;
+}
+
+muon_status muon_destroy(muon_ctx* c) {
+  if (!c) return MUON_OK;
+  DeviceGuard guard(c->device);
+  cudaDeviceSynchronize();
+  cudaFree(c->ws);
+  cudaFree(c->d_nu);
+  cudaFree(c->d_s1);
+  cudaFree(c->d_s2);
+  cudaFree(c->d_flags);
+  cudaFree(c->d_counters);
+  cudaFree(c->d_partials);
+  cudaFree(c->d_status);
+  cudaFree(c->d_stage);
+  for (cudaEvent_t e : c->events) cudaEventDestroy(e);
+  delete c;
+  return MUON_OK;
+}
+
+muon_status muon_set_coeffs(muon_ctx* c, const float* abc, int k) {
+  if (!c || !abc || k < 1 || k > MUON_MAX_ITERS) return MUON_ERR_INVALID_ARG;
+  for (int i = 0; i < 3 * k; ++i)
+    if (!std::isfinite(abc[i])) return MUON_ERR_INVALID_ARG;
+  std::memcpy(c->coeffs, abc, sizeof(float) * 3 * k);
+  c->k = k;
+  return MUON_OK;
+}
+
+muon_status muon_get_coeffs(const muon_ctx* c, float* abc, int* k) {
+  if (!c || !abc || !k) return MUON_ERR_INVALID_ARG;
+  std::memcpy(abc, c->coeffs, sizeof(float) * 3 * c->k);
+  *k = c->k;
+  return MUON_OK;
+}
+
+muon_status muon_step_groups(muon_ctx* c, const muon_group* groups, int ngroups,
+                             const muon_hparams* hp, void* stream) {
+  std::vector<GroupPlan> plans;
+  muon_status st = validate_and_plan(c, groups, ngroups, true, plans);
+  if (st != MUON_OK) return st;
+  st = check_hparams(hp);
+  if (st != MUON_OK) return st;
+  DeviceGuard guard(c->device);
+  return run(c, plans, hp, true, hp->eps, static_cast<cudaStream_t>(stream));
+}
+
+muon_status muon_step(muon_ctx* c, void* const* W, const void* const* G, float* const* M,
+                      int batch, int rows, int cols, int dtype, const muon_hparams* hp,
+                      void* stream) {
+  muon_group g;
+  g.W = W;
+  g.G = G;
+  g.M = M;
+  g.batch = batch;
+  g.rows = rows;
+  g.cols = cols;
+  g.dtype = dtype;
+  return muon_step_groups(c, &g, 1, hp, stream);
+}
+
+muon_status muon_ns_orthogonalize(muon_ctx* c, const void* const* X, void* const* Out, int batch,
+                                  int rows, int cols, int dtype, float eps, void* stream) {
+  if (!std::isfinite(eps) || eps < 0.f) return MUON_ERR_INVALID_ARG;
+  muon_group g;
+  g.W = Out;
+  g.G = X;
+  g.M = nullptr;
+  g.batch = batch;
+  g.rows = rows;
+  g.cols = cols;
+  g.dtype = dtype;
+  std::vector<GroupPlan> plans;
+  muon_status st = validate_and_plan(c, &g, 1, false, plans);
+  if (st != MUON_OK) return st;
+  for (int l = 0; l < batch; ++l)
+    if (Out[l] == X[l]) return MUON_ERR_INVALID_ARG;
+  DeviceGuard guard(c->device);
+  return run(c, plans, nullptr, false, eps, static_cast<cudaStream_t>(stream));
+}
+
+muon_status muon_get_status(muon_ctx* c, int* flags, int capacity, int* count) {
+  if (!c || capacity < 0) return MUON_ERR_INVALID_ARG;
+  DeviceGuard guard(c->device);
+  if (count) *count = c->last_count;
+  if (!c->pending) return MUON_OK;
+  MUON_CUDA(cudaStreamSynchronize(c->last_stream), "stream synchronize");
+  int status = 0;
+  MUON_CUDA(cudaMemcpy(&status, c->d_status, sizeof(int), cudaMemcpyDeviceToHost), "read status");
+  std::vector<int> f(c->last_count);
+  if (c->last_count > 0)
+    MUON_CUDA(cudaMemcpy(f.data(), c->d_flags, sizeof(int) * c->last_count, cudaMemcpyDeviceToHost),
+              "read flags");
+  if (flags) std::memcpy(flags, f.data(), sizeof(int) * std::min(capacity, c->last_count));
+  if (status & kStatusTimeout) return MUON_ERR_TIMEOUT;
+  for (int v : f)
+    if (v & MUON_FLAG_NONFINITE) return MUON_ERR_NONFINITE;
+  return MUON_OK;
+}
+
+muon_status muon_get_norms(muon_ctx* c, float* nu, int capacity, int* count) {
+  if (!c || !nu || capacity < 0) return MUON_ERR_INVALID_ARG;
+  DeviceGuard guard(c->device);
+  if (count) *count = c->last_count;
+  if (!c->pending || c->last_count == 0) return MUON_OK;
+  MUON_CUDA(cudaStreamSynchronize(c->last_stream), "stream synchronize");
+  MUON_CUDA(cudaMemcpy(nu, c->d_nu, sizeof(float) * std::min(capacity, c->last_count),
+                       cudaMemcpyDeviceToHost),
+            "read norms");
+  return MUON_OK;
+}
+
+muon_status muon_step_groups_host(muon_ctx* c, const muon_group* groups, int ngroups,
+                                  const muon_hparams* hp, float* nu_host, int* flags_host,
+                                  void* stream) {
+  if (!c || !groups || ngroups < 1 || ngroups > MUON_MAX_GROUPS) return MUON_ERR_INVALID_ARG;
+  muon_status st = check_hparams(hp);
+  if (st != MUON_OK) return st;
+  size_t need = 0;
+  for (int i = 0; i < ngroups; ++i) {
+    st = check_group(groups[i], true);
+    if (st != MUON_OK) return st;
+    const size_t eb = groups[i].dtype == MUON_F32 ? 4 : 2;
+    need += align_up(static_cast<size_t>(groups[i].rows) * groups[i].cols * eb, 256) * groups[i].batch;
+  }
+  DeviceGuard guard(c->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (need > c->stage_bytes) {
+    MUON_CUDA(cudaStreamSynchronize(s), "sync before staging growth");
+    cudaFree(c->d_stage);
+    c->d_stage = nullptr;
+    c->stage_bytes = 0;
+    if (cudaMalloc(&c->d_stage, need) != cudaSuccess) {
+      cudaGetLastError();
+      return MUON_ERR_ALLOC;
+    }
+    c->stage_bytes = need;
+  }
+  // Device-side copies of the groups whose G pointers now point into the staging buffer.
+  std::vector<std::vector<const void*>> gptr(ngroups);
+  std::vector<muon_group> dev(groups, groups + ngroups);
+  size_t off = 0;
+  for (int i = 0; i < ngroups; ++i) {
+    const size_t eb = groups[i].dtype == MUON_F32 ? 4 : 2;
+    const size_t bytes = static_cast<size_t>(groups[i].rows) * groups[i].cols * eb;
+    gptr[i].resize(groups[i].batch);
+    for (int l = 0; l < groups[i].batch; ++l) {
+      void* dst = static_cast<char*>(c->d_stage) + off;
+      MUON_CUDA(cudaMemcpyAsync(dst, groups[i].G[l], bytes, cudaMemcpyHostToDevice, s), "gradient upload");
+      gptr[i][l] = dst;
+      off += align_up(bytes, 256);
+    }
+    dev[i].G = gptr[i].data();
+  }
+  std::vector<GroupPlan> plans;
+  st = validate_and_plan(c, dev.data(), ngroups, true, plans);
+  if (st != MUON_OK) return st;
+  st = run(c, plans, hp, true, hp->eps, s);
+  if (st != MUON_OK) return st;
+  if (nu_host)
+    MUON_CUDA(cudaMemcpyAsync(nu_host, c->d_nu, sizeof(float) * c->last_count, cudaMemcpyDeviceToHost, s),
+              "norm download");
+  if (flags_host)
+    MUON_CUDA(cudaMemcpyAsync(flags_host, c->d_flags, sizeof(int) * c->last_count, cudaMemcpyDeviceToHost, s),
+              "flag download");
+  MUON_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+  return muon_get_status(c, nullptr, 0, nullptr);
+}
+
+size_t muon_workspace_bytes(const muon_ctx* c) {
+  if (!c) return 0;
+  return c->ws_bytes + c->stage_bytes;
+}
+
+muon_status muon_profile_enable(muon_ctx* c, int on) {
+  if (!c) return MUON_ERR_INVALID_ARG;
+  c->profiling = on != 0;
+  return MUON_OK;
+}
+
+muon_status muon_profile_read(muon_ctx* c, muon_profile* out, int reset) {
+  if (!c || !out) return MUON_ERR_INVALID_ARG;
+  DeviceGuard guard(c->device);
+  std::memset(out, 0, sizeof(*out));
+  for (size_t i = 0; i < c->rec_kind.size(); ++i) {
+    MUON_CUDA(cudaEventSynchronize(c->events[2 * i + 1]), "profile event");
+    float ms = 0.f;
+    MUON_CUDA(cudaEventElapsedTime(&ms, c->events[2 * i], c->events[2 * i + 1]), "profile elapsed");
+    out->launches[c->rec_kind[i]] += 1;
+    out->ms[c->rec_kind[i]] += ms;
+  }
+  if (reset) c->rec_kind.clear();
+  return MUON_OK;
+}
+
+}  // extern "C"

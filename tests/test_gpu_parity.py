@@ -1,0 +1,330 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C-ABI (needs a B200).
+
+Tolerances (relative Frobenius error per matrix): bf16 path <= 2e-2, fp32 path
+<= 1e-4.  Small cases span several 128 x 256 tiles and ragged tails; the
+Mamba-2 130M groups run at full size and are compared on sampled matrices.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from synthetic import (MAMBA2_130M_IN_PROJ, MAMBA2_130M_OUT_PROJ, draw, group_inputs, group_weights,
+                       rng_for, round_bf16)
+from tests.gpu_common import (BF16_TOL, F32_TOL, dominant_subspace_error, half_ulp_bf16, rel_f,
+                              to_device, to_numpy)
+
+pytestmark = pytest.mark.gpu
+
+QUINTIC5 = [oracle.QUINTIC] * 5
+CUBIC10 = [oracle.CUBIC] * 10
+HP = dict(lr=0.02, beta=0.95, weight_decay=0.1, eps=1e-7)
+
+
+@pytest.fixture(scope="module")
+def ctx():
+    import torch
+    from spectral_optimizer_state_b200 import Muon
+    assert torch.cuda.is_available()
+    m = Muon(0)
+    yield m
+    m.close()
+
+
+def _inputs(shape, count, seed, kind="spike", dtype="bf16"):
+    out = []
+    for l in range(count):
+        g = draw(kind, rng_for(seed, l), *shape).astype(np.float32)
+        out.append(np.asarray(g, np.float32) if dtype == "f32" else round_bf16(g))
+    return out
+
+
+SMALL_SHAPES = [(64, 96), (128, 128), (200, 328), (328, 200), (257, 700), (96, 1000), (1000, 96), (37, 53),
+                (53, 37), (768, 1536)]
+
+
+# ---------------------------------------------------------------- orthogonalisation only
+@pytest.mark.parametrize("shape", SMALL_SHAPES)
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_ns_orthogonalize_small(ctx, shape, dtype):
+    import torch
+    Gs = _inputs(shape, 3, seed=hash(shape) % 1000, kind="gauss", dtype=dtype)
+    X = [to_device(g, dtype) for g in Gs]
+    Out = [torch.empty_like(x) for x in X]
+    ctx.set_coeffs(QUINTIC5)
+    ctx.ns_orthogonalize(X, Out, eps=1e-7)
+    st, flags = ctx.status()
+    assert st == 0 and flags == [0, 0, 0]
+    tol = BF16_TOL if dtype == "bf16" else F32_TOL
+    for g, o in zip(Gs, Out):
+        ref, _ = oracle.orthogonalize(g.astype(np.float64), QUINTIC5, eps=1e-7)
+        assert rel_f(to_numpy(o), ref) <= tol, (shape, dtype, rel_f(to_numpy(o), ref))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_cubic_without_polynomial_product(ctx, dtype):
+    """c = 0 skips the A^2 product; 10 cubic steps on the 128 x 64 case."""
+    import torch
+    G = _inputs((128, 64), 1, seed=0, kind="gauss", dtype=dtype)[0]
+    X = [to_device(G, dtype)]
+    Out = [torch.empty_like(X[0])]
+    ctx.set_coeffs(CUBIC10)
+    ctx.ns_orthogonalize(X, Out, eps=1e-7)
+    ref, _ = oracle.orthogonalize(G.astype(np.float64), CUBIC10, eps=1e-7)
+    tol = BF16_TOL if dtype == "bf16" else F32_TOL
+    assert rel_f(to_numpy(Out[0]), ref) <= tol
+    ctx.set_coeffs(QUINTIC5)
+
+
+@pytest.mark.parametrize("k", [1, 2, 7])
+def test_iteration_counts(ctx, k):
+    import torch
+    coeffs = [(3.0, -3.2, 1.2)] * k
+    G = _inputs((300, 520), 2, seed=5, kind="gauss", dtype="f32")
+    X = [to_device(g, "f32") for g in G]
+    Out = [torch.empty_like(x) for x in X]
+    ctx.set_coeffs(coeffs)
+    assert ctx.get_coeffs() == [tuple(np.float32(v) for v in c) for c in coeffs]
+    ctx.ns_orthogonalize(X, Out, eps=1e-7)
+    for g, o in zip(G, Out):
+        ref, _ = oracle.orthogonalize(g.astype(np.float64), [tuple(float(np.float32(v)) for v in c) for c in coeffs])
+        assert rel_f(to_numpy(o), ref) <= F32_TOL
+    ctx.set_coeffs(QUINTIC5)
+
+
+# ---------------------------------------------------------------- full step
+def _step_case(ctx, shape, count, dtype, steps, kind="spike", w_zero=False, nesterov=True,
+               scale_mode=oracle.SCALE_SQRT_RATIO, check=None):
+    import torch
+    R, C = shape
+    check = list(range(count)) if check is None else check
+    W0 = [np.zeros(shape, np.float32) for _ in range(count)] if w_zero else \
+        _inputs(shape, count, seed=77, kind="gauss", dtype=dtype)
+    W0 = [w * (0 if w_zero else 0.02) for w in W0]
+    if dtype == "bf16":
+        W0 = [round_bf16(w) for w in W0]
+    W = [to_device(w, dtype) for w in W0]
+    M = [torch.zeros(shape, dtype=torch.float32, device="cuda") for _ in range(count)]
+    ctx.set_coeffs(QUINTIC5)
+    grads = []
+    for s in range(steps):
+        Gs = _inputs(shape, count, seed=1000 + 10 * s, kind=kind, dtype=dtype)
+        grads.append(Gs)
+        ctx.step(W, [to_device(g, dtype) for g in Gs], M, nesterov=nesterov, scale_mode=scale_mode, **HP)
+        st, flags = ctx.status()
+        assert st == 0, st
+    for l in check:
+        Wr, Mr, Or, nur = oracle_replay(W0[l], [grads[s][l] for s in range(steps)], nesterov, scale_mode)
+        Wg, Mg = to_numpy(W[l]), to_numpy(M[l])
+        assert rel_f(Mg, Mr) <= 1e-6
+        dW = Wr - W0[l]
+        if dtype == "f32":
+            assert rel_f(Wg - W0[l], dW) <= F32_TOL, rel_f(Wg - W0[l], dW)
+        else:
+            bound = BF16_TOL * np.linalg.norm(dW) + np.linalg.norm(half_ulp_bf16(Wr))
+            assert np.linalg.norm(Wg - Wr) <= bound, (np.linalg.norm(Wg - Wr), bound)
+    return W, M
+
+
+def oracle_replay(W0, Gs, nesterov=True, scale_mode=oracle.SCALE_SQRT_RATIO):
+    W = W0.astype(np.float64)
+    M = np.zeros_like(W)
+    r = None
+    for G in Gs:
+        r = oracle.muon_step(W, G.astype(np.float64), M, QUINTIC5, nesterov=nesterov, scale_mode=scale_mode, **HP)
+        W, M = r["W"], r["M"]
+    return W, M, r["O"], r["nu"]
+
+
+@pytest.mark.parametrize("shape", [(200, 328), (328, 200), (53, 37), (37, 53), (768, 1536)])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_step_small(ctx, shape, dtype):
+    _step_case(ctx, shape, 3, dtype, steps=3)
+
+
+@pytest.mark.parametrize("shape", [(200, 328), (1000, 96)])
+def test_step_bf16_zero_weights_measures_update(ctx, shape):
+    """W = 0 and wd irrelevant: W_after = -lr s O rounded to bf16, so O is compared at 2e-2."""
+    import torch
+    count = 2
+    W = [torch.zeros(shape, dtype=torch.bfloat16, device="cuda") for _ in range(count)]
+    M = [torch.zeros(shape, dtype=torch.float32, device="cuda") for _ in range(count)]
+    Gs = _inputs(shape, count, seed=3, kind="spike")
+    ctx.set_coeffs(QUINTIC5)
+    ctx.step(W, [to_device(g, "bf16") for g in Gs], M, **HP)
+    s = oracle.shape_scale(*shape)
+    for l in range(count):
+        O_ref, _ = oracle.orthogonalize((1 + HP["beta"]) * Gs[l].astype(np.float64), QUINTIC5, eps=HP["eps"])
+        O_gpu = -to_numpy(W[l]) / (HP["lr"] * s)
+        assert rel_f(O_gpu, O_ref) <= BF16_TOL + 4e-3
+
+
+@pytest.mark.parametrize("nesterov,scale_mode", [(False, oracle.SCALE_NONE), (True, oracle.SCALE_RMS_MATCH)])
+def test_step_options(ctx, nesterov, scale_mode):
+    _step_case(ctx, (300, 140), 2, "f32", steps=2, nesterov=nesterov, scale_mode=scale_mode)
+
+
+def test_norms_reported(ctx):
+    import torch
+    shape = (257, 700)
+    Gs = _inputs(shape, 2, seed=9, kind="spike", dtype="f32")
+    W = [torch.zeros(shape, device="cuda") for _ in Gs]
+    M = [torch.zeros(shape, device="cuda") for _ in Gs]
+    ctx.step(W, [to_device(g, "f32") for g in Gs], M, **HP)
+    nu = ctx.norms()
+    for g, n in zip(Gs, nu):
+        assert abs(n - (1 + HP["beta"]) * np.linalg.norm(g.astype(np.float64))) <= 1e-5 * n
+
+
+# ---------------------------------------------------------------- edge cases
+def test_zero_gradient_decays_only(ctx):
+    import torch
+    shape = (130, 260)
+    W0 = np.full(shape, 0.5, np.float32)
+    W = [to_device(W0, "f32")]
+    M = [torch.zeros(shape, device="cuda")]
+    ctx.step(W, [torch.zeros(shape, device="cuda")], M, **HP)
+    st, flags = ctx.status()
+    assert st == 0 and flags == [0]
+    assert np.array_equal(to_numpy(W[0]), (W0 * np.float32(1 - HP["lr"] * HP["weight_decay"])).astype(np.float64))
+
+
+def test_nonfinite_gradient_leaves_weights(ctx):
+    import torch
+    shape = (96, 160)
+    W0 = _inputs(shape, 2, seed=4, kind="gauss")
+    W = [to_device(w * 0.02, "bf16") for w in W0]
+    before = [w.clone() for w in W]
+    G = [to_device(g, "bf16") for g in _inputs(shape, 2, seed=5, kind="gauss")]
+    G[1][3, 7] = float("inf")
+    M = [torch.zeros(shape, device="cuda") for _ in range(2)]
+    ctx.step(W, G, M, **HP)
+    st, flags = ctx.status()
+    assert st == 5 and flags == [0, 1]
+    assert torch.equal(W[1], before[1])
+    assert not torch.equal(W[0], before[0])
+
+
+def test_deterministic_and_canaries(ctx):
+    import torch
+    shape = (331, 517)
+    n = shape[0] * shape[1]
+    results = []
+    for rep in range(2):
+        bufW = torch.full((n + 4096,), 7.0, dtype=torch.bfloat16, device="cuda")
+        bufM = torch.full((n + 4096,), -3.0, dtype=torch.float32, device="cuda")
+        W = [bufW[:n].view(shape)]
+        M = [bufM[:n].view(shape)]
+        W[0].copy_(to_device(_inputs(shape, 1, seed=8, kind="gauss")[0] * 0.02, "bf16"))
+        M[0].zero_()
+        G = [to_device(_inputs(shape, 1, seed=9, kind="spike")[0], "bf16")]
+        ctx.step(W, G, M, **HP)
+        ctx.status()
+        assert torch.all(bufW[n:] == 7.0) and torch.all(bufM[n:] == -3.0)
+        results.append((W[0].clone(), M[0].clone()))
+    assert torch.equal(results[0][0], results[1][0]) and torch.equal(results[0][1], results[1][1])
+
+
+def test_host_gradient_entry_matches_device_entry(ctx):
+    import torch
+    shape = (200, 328)
+    Gs = _inputs(shape, 3, seed=21, kind="spike")
+    W0 = [to_device(w * 0.02, "bf16") for w in _inputs(shape, 3, seed=22, kind="gauss")]
+    Wa = [w.clone() for w in W0]
+    Wb = [w.clone() for w in W0]
+    Ma = [torch.zeros(shape, device="cuda") for _ in Gs]
+    Mb = [torch.zeros(shape, device="cuda") for _ in Gs]
+    ctx.step_groups([(Wa, [to_device(g, "bf16") for g in Gs], Ma)], **HP)
+    ctx.status()
+    host = [torch.from_numpy(g).to(torch.bfloat16).pin_memory() for g in Gs]
+    nu, flags = ctx.step_groups_host([(Wb, host, Mb)], **HP)
+    assert flags == [0, 0, 0]
+    for a, b in zip(Wa, Wb):
+        assert torch.equal(a, b)
+    for g, n in zip(Gs, nu):
+        assert abs(n - 1.95 * np.linalg.norm(g.astype(np.float64))) <= 1e-5 * n
+
+
+def test_bad_arguments_raise(ctx):
+    import torch
+    from spectral_optimizer_state_b200 import MuonError
+    W = [torch.zeros(8, 8, dtype=torch.bfloat16, device="cuda")]
+    with pytest.raises(MuonError):
+        ctx.step(W, [torch.zeros(8, 8, dtype=torch.bfloat16, device="cuda")], [torch.zeros(8, 8, device="cuda")],
+                 lr=float("nan"))
+    with pytest.raises(MuonError):
+        ctx.set_coeffs([])
+    with pytest.raises(MuonError):
+        ctx.ns_orthogonalize(W, W)  # Out aliases X
+
+
+# ---------------------------------------------------------------- Mamba-2 130M groups, full size
+@pytest.mark.parametrize("name,shape", [("out_proj", MAMBA2_130M_OUT_PROJ), ("in_proj", MAMBA2_130M_IN_PROJ)])
+def test_mamba2_130m_group_full_size(ctx, name, shape):
+    """24 matrices per group in one call; matrices 0, 11 and 23 checked against the oracle."""
+    import torch
+    group = 0 if name == "out_proj" else 1
+    Gs = group_inputs(1 + group, 0, group, 24, *shape)
+    W0 = group_weights(1 + group, group, 24, *shape)
+    W = [to_device(w, "bf16") for w in W0]
+    M = [torch.zeros(shape, device="cuda") for _ in range(24)]
+    ctx.set_coeffs(QUINTIC5)
+    ctx.step(W, [to_device(g, "bf16") for g in Gs], M, **HP)
+    st, flags = ctx.status()
+    assert st == 0 and flags == [0] * 24
+    # the orthogonalised update itself, same launch shapes, through muon_ns_orthogonalize
+    U = [to_device(np.float32(1 + HP["beta"]) * g, "f32").to(torch.bfloat16) for g in Gs]
+    Out = [torch.empty_like(u) for u in U]
+    ctx.ns_orthogonalize(U, Out, eps=HP["eps"])
+    for l in (0, 11, 23):
+        O_ref, _ = oracle.orthogonalize(to_numpy(U[l]), QUINTIC5, eps=HP["eps"])
+        assert rel_f(to_numpy(Out[l]), O_ref) <= BF16_TOL
+        r = oracle.muon_step(W0[l], Gs[l], np.zeros(shape), QUINTIC5, **HP)
+        assert rel_f(to_numpy(M[l]), r["M"]) <= 1e-6
+        bound = BF16_TOL * np.linalg.norm(r["W"] - W0[l]) + np.linalg.norm(half_ulp_bf16(r["W"]))
+        assert np.linalg.norm(to_numpy(W[l]) - r["W"]) <= bound
+
+
+def test_mamba2_130m_both_groups_ten_steps(ctx):
+    """in_proj + out_proj in one call, 10 steps, persistent momentum, redrawn gradients."""
+    import torch
+    shapes = [MAMBA2_130M_OUT_PROJ, MAMBA2_130M_IN_PROJ]
+    W0 = [group_weights(3, g, 24, *shapes[g]) for g in range(2)]
+    W = [[to_device(w, "bf16") for w in W0[g]] for g in range(2)]
+    M = [[torch.zeros(shapes[g], device="cuda") for _ in range(24)] for g in range(2)]
+    sample = {0: [0, 23], 1: [5, 17]}
+    hist = {(g, l): [] for g in range(2) for l in sample[g]}
+    ctx.set_coeffs(QUINTIC5)
+    for step in range(10):
+        G = [group_inputs(3, step, g, 24, *shapes[g]) for g in range(2)]
+        for g in range(2):
+            for l in sample[g]:
+                hist[(g, l)].append(G[g][l])
+        ctx.step_groups([(W[g], [to_device(x, "bf16") for x in G[g]], M[g]) for g in range(2)], **HP)
+        st, _ = ctx.status()
+        assert st == 0
+    for (g, l), grads in hist.items():
+        Wr, Mr, _, _ = oracle_replay(W0[g][l], grads)
+        assert rel_f(to_numpy(M[g][l]), Mr) <= 1e-5
+        bound = BF16_TOL * np.linalg.norm(Wr - W0[g][l]) + np.linalg.norm(half_ulp_bf16(Wr))
+        assert np.linalg.norm(to_numpy(W[g][l]) - Wr) <= bound
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_ill_conditioned_variant(ctx, dtype):
+    """Singular values log-uniform in [1e-6, 1]: fp32 path on the full matrix; bf16 path on
+    the input's dominant subspace (normalised sigma >= 1e-2), full error reported."""
+    import torch
+    shape = MAMBA2_130M_OUT_PROJ
+    Gs = group_inputs(3, 0, 0, 2, *shape, kind="ill", dtype=dtype)
+    X = [to_device(g, dtype) for g in Gs]
+    Out = [torch.empty_like(x) for x in X]
+    ctx.set_coeffs(QUINTIC5)
+    ctx.ns_orthogonalize(X, Out, eps=HP["eps"])
+    for g, o in zip(Gs, Out):
+        ref, _ = oracle.orthogonalize(g.astype(np.float64), QUINTIC5, eps=HP["eps"])
+        full = rel_f(to_numpy(o), ref)
+        if dtype == "f32":
+            assert full <= F32_TOL, full
+        else:
+            assert dominant_subspace_error(to_numpy(o), ref, g) <= BF16_TOL
+            assert full < 0.15  # reported; single-pass bf16 cannot resolve sigma ~1e-6 directions

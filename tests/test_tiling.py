@@ -1,0 +1,87 @@
+"""Host-side check of the GEMM tile schedule (mirrors the kernel's tile decode, no GPU).
+
+For the shapes the library runs, every output element of the symmetric
+(Gram / polynomial) and plain (update) products must be written exactly once,
+directly or by the mirror store; every TMA load must start at an x coordinate
+that is a multiple of 64 elements (128 bytes); every store must stay inside
+its [rows][pitch] buffer.
+"""
+import numpy as np
+import pytest
+
+BM, BN = 128, 256
+
+
+def tiles_per_matrix(M, N, sym):
+    if sym:
+        return sum((M - BM * mb + BN - 1) // BN for mb in range((M + BM - 1) // BM))
+    return ((M + BM - 1) // BM) * ((N + BN - 1) // BN)
+
+
+def decode(M, N, sym, r):
+    if sym:
+        mb = 0
+        while True:
+            cnt = (M - BM * mb + BN - 1) // BN
+            if r < cnt:
+                break
+            r -= cnt
+            mb += 1
+        m0, n0 = BM * mb, BM * mb + BN * r
+    else:
+        tn = (N + BN - 1) // BN
+        mb = r // tn
+        m0, n0 = BM * mb, (r - mb * tn) * BN
+    nw = min(BN, (N - n0 + 63) // 64 * 64)
+    return m0, n0, nw
+
+
+SHAPES = [(64, 96), (128, 128), (200, 328), (257, 700), (96, 1000), (37, 53), (768, 1536), (768, 3352),
+          (2048, 4096), (2048, 8768), (8192, 8192), (1, 1), (130, 260)]
+
+
+@pytest.mark.parametrize("m,n", SHAPES)
+def test_symmetric_cover_exactly_once(m, n):
+    if m > 2048:
+        pytest.skip("large")
+    pitch = (m + 7) // 8 * 8
+    hits = np.zeros((m, pitch), np.int32)
+    for r in range(tiles_per_matrix(m, m, 1)):
+        m0, n0, nw = decode(m, m, 1, r)
+        assert n0 % 64 == 0 and nw % 64 == 0 and 64 <= nw <= 256 and n0 >= m0
+        rows = np.arange(m0, min(m0 + BM, m))
+        for c in range(0, nw, 32):
+            j0 = n0 + c
+            if j0 >= m:
+                continue
+            cols = np.arange(j0, min(j0 + 32, m))
+            hits[np.ix_(rows, cols)] += 1
+            if j0 >= m0 + BM:  # mirror store
+                hits[np.ix_(cols, rows)] += 1
+    assert np.all(hits[:, :m] == 1)
+    assert np.all(hits[:, m:] == 0)
+
+
+@pytest.mark.parametrize("m,n", SHAPES)
+def test_update_cover_exactly_once(m, n):
+    if m * n > 2048 * 8768:
+        pytest.skip("large")
+    hits = np.zeros((m, n), np.int32)
+    for r in range(tiles_per_matrix(m, n, 0)):
+        m0, n0, nw = decode(m, n, 0, r)
+        assert n0 % 64 == 0 and nw % 64 == 0 and nw <= 256
+        assert n0 + nw <= (n + 63) // 64 * 64
+        rows = slice(m0, min(m0 + BM, m))
+        hits[rows, n0:min(n0 + nw, n)] += 1
+    assert np.all(hits == 1)
+
+
+@pytest.mark.parametrize("m,n", SHAPES)
+def test_tma_coordinates_aligned(m, n):
+    for sym, N, K in ((1, m, n), (1, m, m), (0, n, m)):
+        for r in range(min(tiles_per_matrix(m, N, sym), 4000)):
+            m0, n0, nw = decode(m, N, sym, r)
+            for kb in range((K + 63) // 64):
+                assert (kb * 64 * 2) % 16 == 0  # A / K-major B: x = k
+            for c in range(nw // 64):
+                assert ((n0 + 64 * c) * 2) % 16 == 0  # MN-major B: x = n
