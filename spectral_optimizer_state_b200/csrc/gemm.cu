@@ -14,10 +14,14 @@
 // matrix of one or two same-phase problems), and runs
 //   warp 0      TMA producer (one thread) into a 4-stage ring of 48 KB stages,
 //   warp 1      TMEM allocation + UMMA issuer (one thread),
-//   warps 2..5  epilogue: TMEM -> registers -> fused arithmetic -> global.
+//   warps 2..9  epilogue: TMEM -> registers -> fused arithmetic -> 32 x 32
+//               swizzled shared-memory tiles -> TMA tensor stores.
 // Two TMEM accumulators (2 x 256 fp32 columns) let the epilogue of one tile
 // overlap the main loop of the next.  Symmetric outputs are computed on the
-// upper 128 x 128 blocks only (tiles start at the diagonal block) and mirrored.
+// upper 128 x 128 blocks only (tiles start at the diagonal block); the lower
+// blocks are written by transposing the staged tile (a second TMA store).
+// The update's aX term is folded into the polynomial (B' = aI + bA + cA^2),
+// so the update epilogue only scales, converts and stores.
 // The fp32 path passes three bf16 planes per operand; six plane products
 // (small terms first) are accumulated in the same TMEM tile.
 //
@@ -41,7 +45,9 @@ constexpr uint32_t B_BYTES = BN * BK * 2;     // 32 KB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t KMAJ_BOX_BYTES = 128 * BK * 2;  // box {64 K, 128 rows}
 constexpr uint32_t MNMAJ_BOX_BYTES = 64 * BK * 2;  // box {64 N, 64 K rows}
-constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
+constexpr uint32_t STAGING_BYTES_PER_WARP = 2 * 2048;  // two 32 x 32 bf16 store tiles
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COLS = 256;
 constexpr int NUM_BARS = 2 * STAGES + 5;
@@ -116,7 +122,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
          (static_cast<uint32_t>(float_to_bf16_bits(b)) << 16);
 }
 
-// v[t] += beta * sum_p cin_p(row, j0 + t) for t < nv
+// v[t] += beta * sum_p cin_p(row, j0 + t) for t < nv (caller guarantees row < M, j0 < N)
 __device__ __forceinline__ void add_cin(const GemmProblem& q, int l, int row, int j0, int nv,
                                         float (&v)[32]) {
   float c[32];
@@ -143,52 +149,59 @@ __device__ __forceinline__ void add_cin(const GemmProblem& q, int l, int row, in
   for (int t = 0; t < 32; ++t) v[t] = fmaf(q.beta, c[t], v[t]);
 }
 
-template <int PLANES>
-__device__ __forceinline__ void store_tile_row(const GemmProblem& q, int l, int row, int j0, int nv,
-                                               const float (&v)[32], bool mirror) {
-  uint16_t* base = q.out + l * q.out_mat;
-  if (nv == 32) {
+// Staging tile for one TMA store: 32 rows x 32 bf16 (64-byte rows) in the
+// 64-byte swizzle the tensor map declares: 16-byte chunk c of row r sits at
+// chunk c ^ ((r >> 1) & 3), which also keeps the row-per-lane writes free of
+// bank conflicts.
+__device__ __forceinline__ uint32_t stage_offset(int r, int chunk16) {
+  return static_cast<uint32_t>(r * 64 + ((chunk16 ^ ((r >> 1) & 3)) << 4));
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+// This lane's 32 values become row `lane` of the staging tile.
+__device__ __forceinline__ void stage_as_row(uint32_t buf, int lane, const uint16_t (&b)[32]) {
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      uint32_t w[PLANES][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint16_t a[PLANES], b[PLANES];
-        split_planes<PLANES>(v[8 * h + 2 * i], a);
-        split_planes<PLANES>(v[8 * h + 2 * i + 1], b);
-#pragma unroll
-        for (int p = 0; p < PLANES; ++p)
-          w[p][i] = static_cast<uint32_t>(a[p]) | (static_cast<uint32_t>(b[p]) << 16);
-      }
-#pragma unroll
-      for (int p = 0; p < PLANES; ++p) {
-        uint16_t* dst = base + p * q.out_plane + static_cast<long long>(row) * q.out_pitch + j0 + 8 * h;
-        *reinterpret_cast<uint4*>(dst) = make_uint4(w[p][0], w[p][1], w[p][2], w[p][3]);
-      }
-    }
-  } else {
-#pragma unroll
-    for (int t = 0; t < 32; ++t) {
-      if (t >= nv) continue;
-      uint16_t a[PLANES];
-      split_planes<PLANES>(v[t], a);
-#pragma unroll
-      for (int p = 0; p < PLANES; ++p)
-        base[p * q.out_plane + static_cast<long long>(row) * q.out_pitch + j0 + t] = a[p];
-    }
+  for (int h = 0; h < 4; ++h) {
+    const int o = 8 * h;
+    st_shared_v4(buf + stage_offset(lane, h),
+                 static_cast<uint32_t>(b[o + 0]) | (static_cast<uint32_t>(b[o + 1]) << 16),
+                 static_cast<uint32_t>(b[o + 2]) | (static_cast<uint32_t>(b[o + 3]) << 16),
+                 static_cast<uint32_t>(b[o + 4]) | (static_cast<uint32_t>(b[o + 5]) << 16),
+                 static_cast<uint32_t>(b[o + 6]) | (static_cast<uint32_t>(b[o + 7]) << 16));
   }
-  if (mirror) {
-    // (row, j) -> (j, row): lanes hold consecutive rows, so each store is coalesced.
+}
+
+// This lane's 32 values become column `lane` of the staging tile (the mirror).
+__device__ __forceinline__ void stage_as_col(uint32_t buf, int lane, const uint16_t (&b)[32]) {
 #pragma unroll
-    for (int t = 0; t < 32; ++t) {
-      if (t >= nv) continue;
-      uint16_t a[PLANES];
-      split_planes<PLANES>(v[t], a);
-#pragma unroll
-      for (int p = 0; p < PLANES; ++p)
-        base[p * q.out_plane + static_cast<long long>(j0 + t) * q.out_pitch + row] = a[p];
-    }
+  for (int t = 0; t < 32; ++t) st_shared_u16(buf + stage_offset(t, lane >> 3) + 2 * (lane & 7), b[t]);
+}
+
+// One 32 x 32 TMA store from the warp's next staging buffer.  Lane 0 first
+// makes sure the store that last read this buffer has finished reading it.
+template <bool AS_COL>
+__device__ __forceinline__ void store_chunk(const CUtensorMap* map, uint32_t stage_base, int& sb, int lane,
+                                            const uint16_t (&b)[32], int x, int y, int l, int p) {
+  const uint32_t buf = stage_base + static_cast<uint32_t>(sb) * 2048u;
+  if (lane == 0) bulk_wait_group_read<1>();
+  __syncwarp();
+  if (AS_COL) stage_as_col(buf, lane, b);
+  else stage_as_row(buf, lane, b);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_4d(map, buf, x, y, l, p);
+    bulk_commit_group();
   }
+  sb ^= 1;
 }
 
 // W (or Out) element of wide position (row, j).
@@ -255,34 +268,15 @@ __device__ __forceinline__ void write_caller(const GemmProblem& q, int l, int ro
   }
 }
 
-__device__ __forceinline__ void epilogue_chunk(const GemmProblem& q, const Tile& ti, int row,
-                                               int j0, const uint32_t (&r)[32], float sl,
-                                               bool skip) {
-  if (row >= q.M || j0 >= q.N) return;
-  const int nv = min(32, q.N - j0);
-  float v[32];
-#pragma unroll
-  for (int t = 0; t < 32; ++t) v[t] = q.alpha * __uint_as_float(r[t]);
-  if (q.cin != nullptr) add_cin(q, ti.l, row, j0, nv, v);
-#pragma unroll
-  for (int t = 0; t < 32; ++t) v[t] *= sl;
-  if (q.epi == EPI_STORE) {
-    const bool mirror = q.sym && (j0 >= ti.m0 + BM);
-    if (q.planes == 3) store_tile_row<3>(q, ti.l, row, j0, nv, v, mirror);
-    else store_tile_row<1>(q, ti.l, row, j0, nv, v, mirror);
-  } else if (!skip) {
-    write_caller(q, ti.l, row, j0, nv, v, q.epi == EPI_APPLY);
-  }
-}
-
 // ------------------------------------------------------------------ kernel
 __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_constant__ GemmParams P) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t bar0 = base + STAGES * STAGE_BYTES;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + STAGES * STAGE_BYTES + 8 * NUM_BARS);
+  const uint32_t stage_area = base + STAGES * STAGE_BYTES;
+  const uint32_t bar0 = stage_area + EPI_WARPS * STAGING_BYTES_PER_WARP;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + (bar0 - base) + 8 * NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -301,7 +295,7 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 128);
+      mbar_init(tempty_bar(a), 32 * EPI_WARPS);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -312,6 +306,7 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
     for (int i = 0; i < P.nprob; ++i) {
       tma_prefetch_map(&P.prob[i].tmA);
       tma_prefetch_map(&P.prob[i].tmB);
+      if (P.prob[i].epi == EPI_STORE) tma_prefetch_map(&P.prob[i].tmOut);
     }
   }
   if (warp == 1) {
@@ -410,8 +405,13 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
       }
     }
   } else {
-    // ------------------------------------------------ epilogue (warps 2..5)
-    const int quarter = warp & 3;  // TMEM lanes this warp may read
+    // ------------------------------------------------ epilogue (warps 2 .. 2+EPI_WARPS-1)
+    // Two warps share each TMEM lane quarter and split its 32-column chunks.
+    const int e = warp - 2;
+    const int quarter = warp & 3;
+    const int half = e >> 2;
+    const uint32_t my_stage = stage_area + static_cast<uint32_t>(e) * STAGING_BYTES_PER_WARP;
+    int sb = 0;
     int local = 0;
     for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++local) {
       const Tile ti = decode_tile(P, t);
@@ -420,20 +420,50 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
       const uint32_t aph = (local >> 1) & 1;
       if (!mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, P.status)) break;
       tc_fence_after();
-      const int row = ti.m0 + 32 * quarter + lane;
+      const int row0 = ti.m0 + 32 * quarter;
+      const int row = row0 + lane;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * ACC_COLS;
-      const float sl = q.mat_scale != nullptr ? q.mat_scale[ti.l] : 1.0f;
+      const float scale = q.alpha * (q.mat_scale != nullptr ? q.mat_scale[ti.l] : 1.0f);
       const bool skip = q.epi == EPI_APPLY && q.flags != nullptr && q.flags[q.flag_offset + ti.l] != 0;
-      for (int c = 0; c < ti.nw; c += 32) {
-        uint32_t r[32];
-        __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the guarded stores
-        tmem_load_32cols(tbase + c, r);
-        tmem_load_wait();
-        epilogue_chunk(q, ti, row, ti.n0 + c, r, sl, skip);
+      if (row0 < q.M) {
+        for (int c = 32 * half; c < ti.nw; c += 64) {
+          const int j0 = ti.n0 + c;
+          if (j0 >= q.N) break;
+          const int nv = min(32, q.N - j0);
+          uint32_t r[32];
+          __syncwarp();  // tcgen05.ld is warp-collective
+          tmem_load_32cols(tbase + c, r);
+          tmem_load_wait();
+          float v[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[k] = scale * __uint_as_float(r[k]);
+          if (q.cin != nullptr && row < q.M) add_cin(q, ti.l, row, j0, nv, v);
+          if (q.diag != 0.f) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (j0 + k == row) v[k] += q.diag;
+          }
+          if (q.epi == EPI_STORE) {
+            const bool mirror = q.sym && (j0 >= ti.m0 + BM);
+            for (int p = 0; p < q.planes; ++p) {
+              uint16_t b[32];
+#pragma unroll
+              for (int k = 0; k < 32; ++k) {
+                b[k] = float_to_bf16_bits(v[k]);
+                v[k] -= bf16_bits_to_float(b[k]);  // residual for the next plane
+              }
+              store_chunk<false>(&q.tmOut, my_stage, sb, lane, b, j0, row0, ti.l, p);
+              if (mirror) store_chunk<true>(&q.tmOut, my_stage, sb, lane, b, row0, j0, ti.l, p);
+            }
+          } else if (!skip && row < q.M) {
+            write_caller(q, ti.l, row, j0, nv, v, q.epi == EPI_APPLY);
+          }
+        }
       }
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
     }
+    if (lane == 0) bulk_wait_group_all();
   }
 
   __syncthreads();
@@ -445,7 +475,9 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
 
 }  // namespace
 
-size_t gemm_smem_bytes() { return STAGES * STAGE_BYTES + BAR_BYTES + 1024; }
+size_t gemm_smem_bytes() {
+  return STAGES * STAGE_BYTES + EPI_WARPS * STAGING_BYTES_PER_WARP + BAR_BYTES + 1024;
+}
 
 int gemm_tiles_per_matrix(int M, int N, int sym) {
   if (sym) {

@@ -40,10 +40,11 @@ cudaError_t launch_momentum(const MomentumParams& p, int batch, bool g_is_f32, b
 int momentum_blocks_per_matrix(int rows, int cols);
 
 // ------------------------------------------------------------------ GEMM
+// Every epilogue first forms  v = alpha * s_l * acc + beta * cin + (row == col ? diag : 0).
 enum EpilogueKind : int {
-  EPI_STORE = 0,  // out = s_l * (alpha*acc + beta*cin), written as planes (and mirrored if sym)
-  EPI_APPLY = 1,  // O = s_l*(alpha*acc + beta*cin); W <- decay*W - lrs*O (oriented)
-  EPI_OUT = 2,    // O as above written to a caller matrix (oriented)
+  EPI_STORE = 0,  // v written as planes through TMA tensor stores (mirrored too if sym)
+  EPI_APPLY = 1,  // W <- decay*W - lrs*v on the caller's matrix (oriented)
+  EPI_OUT = 2,    // v written to the caller's matrix (oriented)
 };
 
 constexpr int kMaxProblems = 2;
@@ -52,6 +53,7 @@ struct alignas(64) GemmProblem {
   CUtensorMap tmA;  // A operand [planes][L][M][K], K contiguous, box {64, 128}
   CUtensorMap tmB;  // B operand: K-major [planes][L][N][K] box {64,128}, or
                     //            MN-major [planes][L][K][N] box {64, 64}
+  CUtensorMap tmOut;  // EPI_STORE output [planes][L][M][N], box {32, 32}, 64-byte swizzle
   int M, N, K, L;
   int nseg;          // 1 (bf16) or 6 (three-plane split)
   int b_mn_major;    // 0: B stored N x K; 1: B stored K x N
@@ -61,7 +63,7 @@ struct alignas(64) GemmProblem {
   int tile_base;     // first global tile index of this problem
   int k_tiles;       // ceil(K / 64)
   int planes;        // planes of out / cin (1 or 3)
-  float alpha, beta;
+  float alpha, beta, diag;
   const float* mat_scale;  // per-matrix factor s_l, or null for 1
   uint16_t* out;           // [planes][L][M][out_pitch] (EPI_STORE)
   long long out_plane, out_mat;

@@ -55,9 +55,12 @@ EncodeTiledFn get_encoder() {
 }
 
 // bf16 buffer [planes][L][rows][pitch] viewed as 4-D {cols, rows, L, planes};
-// box {box_cols, box_rows}, 128-byte swizzle, out-of-range reads give zeros.
+// box {box_cols, box_rows}.  Operand maps use the 128-byte swizzle the UMMA
+// descriptors expect; store maps use the 64-byte swizzle of the epilogue's
+// 32 x 32 staging tiles.  Out-of-range reads give zeros, stores are clipped.
 bool encode_map(CUtensorMap* map, const void* base, int cols, int rows, int L, int planes,
-                int pitch, int box_cols, int box_rows) {
+                int pitch, int box_cols, int box_rows,
+                CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn enc = get_encoder();
   if (!enc) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
@@ -67,7 +70,7 @@ bool encode_map(CUtensorMap* map, const void* base, int cols, int rows, int L, i
   cuuint32_t box[4] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -277,6 +280,7 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, bool last, 
   std::memset(static_cast<void*>(&q), 0, sizeof(q));
   const float a = c->coeffs[3 * it], b = c->coeffs[3 * it + 1], cc = c->coeffs[3 * it + 2];
   const int src = it & 1, dst = (it + 1) & 1;
+  (void)dst;
   uint16_t* X = ws_at(c, p.off_x[src]);
   uint16_t* Xn = ws_at(c, p.off_x[dst]);
   uint16_t* A = ws_at(c, p.off_a);
@@ -287,38 +291,44 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, bool last, 
   q.planes = p.planes;
   q.flags = c->d_flags;
   q.flag_offset = p.mat_off;
+  const bool have_poly = cc != 0.f;
+  const CUtensorMapSwizzle sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
   switch (ph) {
     case PH_GRAM:
+      // A = s2 * X X^T; with c = 0 the polynomial is linear and the Gram
+      // epilogue writes B' = b A + a I directly.
       if (!encode_map(&q.tmA, X, n, m, p.batch, p.planes, p.pitch_n, 64, 128)) return false;
       q.tmB = q.tmA;
+      if (!encode_map(&q.tmOut, have_poly ? A : B, m, m, p.batch, p.planes, p.pitch_m, 32, 32, sw64))
+        return false;
       q.M = m; q.N = m; q.K = n;
       q.b_mn_major = 0; q.sym = 1; q.epi = EPI_STORE;
-      q.alpha = 1.f; q.beta = 0.f;
+      q.alpha = have_poly ? 1.f : b;
+      q.beta = 0.f;
+      q.diag = have_poly ? 0.f : a;
       q.mat_scale = it == 0 ? c->d_s2 + p.mat_off : nullptr;
-      q.out = A; q.out_plane = p.a_plane; q.out_mat = p.a_mat; q.out_pitch = p.pitch_m;
       break;
     case PH_POLY:
+      // B' = c A A + b A + a I
       if (!encode_map(&q.tmA, A, m, m, p.batch, p.planes, p.pitch_m, 64, 128)) return false;
       q.tmB = q.tmA;
+      if (!encode_map(&q.tmOut, B, m, m, p.batch, p.planes, p.pitch_m, 32, 32, sw64)) return false;
       q.M = m; q.N = m; q.K = m;
       q.b_mn_major = 0; q.sym = 1; q.epi = EPI_STORE;
-      q.alpha = cc; q.beta = b;
+      q.alpha = cc; q.beta = b; q.diag = a;
       q.cin = A; q.cin_plane = p.a_plane; q.cin_mat = p.a_mat; q.cin_pitch = p.pitch_m;
-      q.out = B; q.out_plane = p.a_plane; q.out_mat = p.a_mat; q.out_pitch = p.pitch_m;
       break;
     case PH_UPDATE: {
-      const bool have_poly = cc != 0.f;
-      if (!encode_map(&q.tmA, have_poly ? B : A, m, m, p.batch, p.planes, p.pitch_m, 64, 128)) return false;
+      // X' = s1 * B' X   (s1 = 1/(nu+eps) on the first iteration, X = U unnormalised)
+      if (!encode_map(&q.tmA, B, m, m, p.batch, p.planes, p.pitch_m, 64, 128)) return false;
       if (!encode_map(&q.tmB, X, n, m, p.batch, p.planes, p.pitch_n, 64, 64)) return false;
       q.M = m; q.N = n; q.K = m;
       q.b_mn_major = 1; q.sym = 0;
-      q.alpha = have_poly ? 1.f : b;
-      q.beta = a;
+      q.alpha = 1.f; q.beta = 0.f; q.diag = 0.f;
       q.mat_scale = it == 0 ? c->d_s1 + p.mat_off : nullptr;
-      q.cin = X; q.cin_plane = p.x_plane; q.cin_mat = p.x_mat; q.cin_pitch = p.pitch_n;
       if (!last) {
         q.epi = EPI_STORE;
-        q.out = Xn; q.out_plane = p.x_plane; q.out_mat = p.x_mat; q.out_pitch = p.pitch_n;
+        if (!encode_map(&q.tmOut, Xn, n, m, p.batch, p.planes, p.pitch_n, 32, 32, sw64)) return false;
       } else {
         q.epi = step ? EPI_APPLY : EPI_OUT;
         q.wrows = p.rows; q.wcols = p.cols; q.transposed = p.transposed; q.w_f32 = p.f32;
