@@ -289,7 +289,7 @@ __device__ __forceinline__ void write_w_f32(const GemmProblem& q, int l, int row
 }
 
 // ------------------------------------------------------------------ kernel
-__global__ void __maxnreg__(200) ns_gemm_kernel(const __grid_constant__ GemmParams P) {
+__global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_constant__ GemmParams P) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
