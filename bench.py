@@ -84,6 +84,11 @@ def momentum_bytes(groups):
     return 12 * elements(groups)
 
 
+def apply_bytes(groups):
+    """Algorithmic bytes of the apply pass: O 2 (read) + W 2 (read) + W 2 (write) per element (bf16)."""
+    return 6 * elements(groups)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -391,6 +396,8 @@ def main():
     burst, sustained = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
     traffic = recorded_traffic(args.workload)
     mom_launches, mom_ms = prof["momentum"]
+    app_launches, app_ms = prof["apply"]
+    app_gbs = apply_bytes(groups) * args.steps / (app_ms / 1e3) / 1e9 if app_ms > 0 else None
     mom_gbs = momentum_bytes(groups) * args.steps / (mom_ms / 1e3) / 1e9 if mom_ms > 0 else None
     h2d = sum(L * R * C * 2 for _, L, R, C in groups)
     d2h = n_mats * 8
@@ -413,6 +420,9 @@ def main():
         "momentum_kernel": {"bound": "hbm", "achieved_gbs": mom_gbs, "peak_gbs": peaks["hbm_gbs"],
                             "frac": (mom_gbs / peaks["hbm_gbs"]) if mom_gbs else None,
                             "bytes_per_element": 12, "launches": mom_launches},
+        "apply_kernel": {"bound": "hbm", "achieved_gbs": app_gbs, "peak_gbs": peaks["hbm_gbs"],
+                         "frac": (app_gbs / peaks["hbm_gbs"]) if app_gbs else None,
+                         "bytes_per_element": 6, "launches": app_launches},
         "kernel_ms_per_step": {k: v[1] / args.steps for k, v in prof.items()},
         "cpu_baseline": cpu,
         "clocks": clk,

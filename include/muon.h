@@ -178,8 +178,9 @@ typedef enum {
   MUON_KERNEL_MOMENTUM = 0, /* momentum + Nesterov + norm pass        */
   MUON_KERNEL_GRAM = 1,     /* A = X X^T                                */
   MUON_KERNEL_POLY = 2,     /* B = b A + c A A                          */
-  MUON_KERNEL_UPDATE = 3,   /* X <- a X + B X (last one applies to W)   */
-  MUON_KERNEL_KINDS = 4
+  MUON_KERNEL_UPDATE = 3,   /* X <- s B' X  with B' = aI + bA + cAA     */
+  MUON_KERNEL_APPLY = 4,    /* W <- (1 - lr wd) W - lr s O              */
+  MUON_KERNEL_KINDS = 5
 } muon_kernel_kind;
 
 typedef struct {

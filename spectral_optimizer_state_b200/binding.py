@@ -38,7 +38,7 @@ EXPORTS = (
     "muon_ns_orthogonalize", "muon_get_status", "muon_get_norms", "muon_workspace_bytes",
     "muon_profile_enable", "muon_profile_read",
 )
-KERNEL_KINDS = ("momentum", "gram", "poly", "update")
+KERNEL_KINDS = ("momentum", "gram", "poly", "update", "apply")
 
 
 class MuonError(RuntimeError):
@@ -56,7 +56,7 @@ class Hparams(ctypes.Structure):
 
 
 class Profile(ctypes.Structure):
-    _fields_ = [("launches", ctypes.c_int * 4), ("ms", ctypes.c_double * 4)]
+    _fields_ = [("launches", ctypes.c_int * 5), ("ms", ctypes.c_double * 5)]
 
 
 class Group(ctypes.Structure):

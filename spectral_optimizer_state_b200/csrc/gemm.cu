@@ -204,90 +204,6 @@ __device__ __forceinline__ void store_chunk(const CUtensorMap* map, uint32_t sta
   sb ^= 1;
 }
 
-// W (or Out) element of wide position (row, j).
-__device__ __forceinline__ long long w_index(const GemmProblem& q, int row, int j) {
-  return q.transposed ? static_cast<long long>(j) * q.wcols + row
-                      : static_cast<long long>(row) * q.wcols + j;
-}
-
-// bf16 W chunk (32 values of one wide row) packed two per register.  Loaded
-// ahead of use so the reads of the caller's matrix overlap the main loop.
-__device__ __forceinline__ void load_w_bf16(const GemmProblem& q, int l, int row, int j0, int nv,
-                                            uint32_t (&w)[16]) {
-  const uint16_t* W = static_cast<const uint16_t*>(q.wtab[l]);
-  if (q.w_vec && !q.transposed && nv == 32) {
-    const uint4* p4 = reinterpret_cast<const uint4*>(W + w_index(q, row, j0));
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const uint4 x = p4[h];
-      w[4 * h] = x.x; w[4 * h + 1] = x.y; w[4 * h + 2] = x.z; w[4 * h + 3] = x.w;
-    }
-  } else {
-    uint16_t e[32];
-#pragma unroll
-    for (int t = 0; t < 32; ++t) e[t] = t < nv ? W[w_index(q, row, j0 + t)] : static_cast<uint16_t>(0);
-#pragma unroll
-    for (int t = 0; t < 16; ++t) w[t] = static_cast<uint32_t>(e[2 * t]) | (static_cast<uint32_t>(e[2 * t + 1]) << 16);
-  }
-}
-
-// W <- decay*W - lrs*v (apply) or W <- v, bf16, from the prefetched chunk.
-__device__ __forceinline__ void store_w_bf16(const GemmProblem& q, int l, int row, int j0, int nv,
-                                             const float (&v)[32], const uint32_t (&w)[16], bool apply) {
-  uint32_t o[16];
-#pragma unroll
-  for (int t = 0; t < 16; ++t) {
-    float a = v[2 * t], b = v[2 * t + 1];
-    if (apply) {
-      a = fmaf(q.decay, __uint_as_float(w[t] << 16), -q.lrs * a);
-      b = fmaf(q.decay, __uint_as_float(w[t] & 0xFFFF0000u), -q.lrs * b);
-    }
-    o[t] = pack_bf16x2(a, b);
-  }
-  uint16_t* W = static_cast<uint16_t*>(q.wtab[l]);
-  if (q.w_vec && !q.transposed && nv == 32) {
-    uint4* p4 = reinterpret_cast<uint4*>(W + w_index(q, row, j0));
-#pragma unroll
-    for (int h = 0; h < 4; ++h) p4[h] = make_uint4(o[4 * h], o[4 * h + 1], o[4 * h + 2], o[4 * h + 3]);
-  } else {
-#pragma unroll
-    for (int t = 0; t < 32; ++t)
-      if (t < nv) W[w_index(q, row, j0 + t)] = static_cast<uint16_t>(o[t >> 1] >> (16 * (t & 1)));
-  }
-}
-
-// fp32 caller matrix: every read of the chunk is issued before any write.
-__device__ __forceinline__ void write_w_f32(const GemmProblem& q, int l, int row, int j0, int nv,
-                                            const float (&v)[32], bool apply) {
-  float* W = static_cast<float*>(q.wtab[l]);
-  float c[32];
-  if (q.w_vec && !q.transposed && nv == 32) {
-    float4* p4 = reinterpret_cast<float4*>(W + w_index(q, row, j0));
-    if (apply) {
-#pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        const float4 x = p4[h];
-        c[4 * h] = x.x; c[4 * h + 1] = x.y; c[4 * h + 2] = x.z; c[4 * h + 3] = x.w;
-      }
-    }
-#pragma unroll
-    for (int h = 0; h < 8; ++h) {
-      float o[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) o[i] = apply ? fmaf(q.decay, c[4 * h + i], -q.lrs * v[4 * h + i]) : v[4 * h + i];
-      p4[h] = make_float4(o[0], o[1], o[2], o[3]);
-    }
-  } else {
-    if (apply) {
-#pragma unroll
-      for (int t = 0; t < 32; ++t) c[t] = t < nv ? W[w_index(q, row, j0 + t)] : 0.f;
-    }
-#pragma unroll
-    for (int t = 0; t < 32; ++t)
-      if (t < nv) W[w_index(q, row, j0 + t)] = apply ? fmaf(q.decay, c[t], -q.lrs * v[t]) : v[t];
-  }
-}
-
 // ------------------------------------------------------------------ kernel
 __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_constant__ GemmParams P) {
   extern __shared__ uint8_t smem_raw[];
@@ -326,7 +242,7 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
     for (int i = 0; i < P.nprob; ++i) {
       tma_prefetch_map(&P.prob[i].tmA);
       tma_prefetch_map(&P.prob[i].tmB);
-      if (P.prob[i].epi == EPI_STORE) tma_prefetch_map(&P.prob[i].tmOut);
+      tma_prefetch_map(&P.prob[i].tmOut);
     }
   }
   if (warp == 1) {
@@ -438,32 +354,17 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
       const GemmProblem& q = P.prob[ti.pi];
       const int acc = local & 1;
       const uint32_t aph = (local >> 1) & 1;
-      const int row0 = ti.m0 + 32 * quarter;
-      const int row = row0 + lane;
-      const bool skip = q.epi == EPI_APPLY && q.flags != nullptr && q.flags[q.flag_offset + ti.l] != 0;
-      // bf16 caller matrix: fetch the first chunk of W before the accumulator is ready
-      const bool w_bf16 = q.epi != EPI_STORE && !q.w_f32 && !skip && row < q.M;
-      const bool w_read = w_bf16 && q.epi == EPI_APPLY;
-      uint32_t wa[16], wb[16];
-      if (w_read && 32 * half < ti.nw && ti.n0 + 32 * half < q.N)
-        load_w_bf16(q, ti.l, row, ti.n0 + 32 * half, min(32, q.N - ti.n0 - 32 * half), wa);
       if (!mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, P.status)) break;
       tc_fence_after();
+      const int row0 = ti.m0 + 32 * quarter;
+      const int row = row0 + lane;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * ACC_COLS;
       const float scale = q.alpha * (q.mat_scale != nullptr ? q.mat_scale[ti.l] : 1.0f);
       if (row0 < q.M) {
-        int k = 0;
-        for (int c = 32 * half; c < ti.nw; c += 64, ++k) {
+        for (int c = 32 * half; c < ti.nw; c += 64) {
           const int j0 = ti.n0 + c;
           if (j0 >= q.N) break;
           const int nv = min(32, q.N - j0);
-          // prefetch the next chunk of W into the other register set
-          const int jn = j0 + 64;
-          const bool next = w_read && c + 64 < ti.nw && jn < q.N;
-          if (next) {
-            if (k & 1) load_w_bf16(q, ti.l, row, jn, min(32, q.N - jn), wa);
-            else load_w_bf16(q, ti.l, row, jn, min(32, q.N - jn), wb);
-          }
           uint32_t r[32];
           __syncwarp();  // tcgen05.ld is warp-collective
           tmem_load_32cols(tbase + c, r);
@@ -477,23 +378,16 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
             for (int i = 0; i < 32; ++i)
               if (j0 + i == row) v[i] += q.diag;
           }
-          if (q.epi == EPI_STORE) {
-            const bool mirror = q.sym && (j0 >= ti.m0 + BM);
-            for (int p = 0; p < q.planes; ++p) {
-              uint16_t b[32];
+          const bool mirror = q.sym && (j0 >= ti.m0 + BM);
+          for (int p = 0; p < q.planes; ++p) {
+            uint16_t b[32];
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                b[i] = float_to_bf16_bits(v[i]);
-                v[i] -= bf16_bits_to_float(b[i]);  // residual for the next plane
-              }
-              store_chunk<false>(&q.tmOut, my_stage, sb, lane, b, j0, row0, ti.l, p);
-              if (mirror) store_chunk<true>(&q.tmOut, my_stage, sb, lane, b, row0, j0, ti.l, p);
+            for (int i = 0; i < 32; ++i) {
+              b[i] = float_to_bf16_bits(v[i]);
+              v[i] -= bf16_bits_to_float(b[i]);  // residual for the next plane
             }
-          } else if (w_bf16) {
-            if (k & 1) store_w_bf16(q, ti.l, row, j0, nv, v, wb, q.epi == EPI_APPLY);
-            else store_w_bf16(q, ti.l, row, j0, nv, v, wa, q.epi == EPI_APPLY);
-          } else if (!skip && row < q.M) {
-            write_w_f32(q, ti.l, row, j0, nv, v, q.epi == EPI_APPLY);
+            store_chunk<false>(&q.tmOut, my_stage, sb, lane, b, j0, row0, ti.l, p);
+            if (mirror) store_chunk<true>(&q.tmOut, my_stage, sb, lane, b, row0, j0, ti.l, p);
           }
         }
       }

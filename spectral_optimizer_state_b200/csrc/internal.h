@@ -39,13 +39,23 @@ cudaError_t launch_momentum(const MomentumParams& p, int batch, bool g_is_f32, b
 // Number of blocks per matrix K1 uses for a rows x cols matrix.
 int momentum_blocks_per_matrix(int rows, int cols);
 
-// ------------------------------------------------------------------ GEMM
-// Every epilogue first forms  v = alpha * s_l * acc + beta * cin + (row == col ? diag : 0).
-enum EpilogueKind : int {
-  EPI_STORE = 0,  // v written as planes through TMA tensor stores (mirrored too if sym)
-  EPI_APPLY = 1,  // W <- decay*W - lrs*v on the caller's matrix (oriented)
-  EPI_OUT = 2,    // v written to the caller's matrix (oriented)
+// ------------------------------------------------------------------ K5 apply
+struct ApplyParams {
+  void* w[MUON_MAX_BATCH];  // caller matrices rows x cols (W, or Out)
+  const uint16_t* o;        // final iterate [planes][batch][m][pitch] bf16 bits (wide)
+  long long o_plane, o_mat; // elements
+  int pitch, rows, cols, planes;
+  int apply;                // 1: W <- decay*W - lrs*O ; 0: W <- O
+  float decay, lrs;
+  const int* flags;         // matrices with a nonzero flag are left unchanged (null: none)
+  int nblk;                 // blocks per matrix
 };
+
+cudaError_t launch_apply(const ApplyParams& p, int batch, bool w_f32, cudaStream_t stream);
+
+// ------------------------------------------------------------------ GEMM
+// The epilogue forms  v = alpha * s_l * acc + beta * cin + (row == col ? diag : 0)
+// and writes it as planes through TMA tensor stores (mirrored too if sym).
 
 constexpr int kMaxProblems = 2;
 
@@ -53,33 +63,20 @@ struct alignas(64) GemmProblem {
   CUtensorMap tmA;  // A operand [planes][L][M][K], K contiguous, box {64, 128}
   CUtensorMap tmB;  // B operand: K-major [planes][L][N][K] box {64,128}, or
                     //            MN-major [planes][L][K][N] box {64, 64}
-  CUtensorMap tmOut;  // EPI_STORE output [planes][L][M][N], box {32, 32}, 64-byte swizzle
+  CUtensorMap tmOut;  // output [planes][L][M][N], box {32, 32}, 64-byte swizzle
   int M, N, K, L;
   int nseg;          // 1 (bf16) or 6 (three-plane split)
   int b_mn_major;    // 0: B stored N x K; 1: B stored K x N
   int sym;           // output symmetric: compute upper tiles only, mirror the rest
-  int epi;           // EpilogueKind
   int tiles_per_matrix;
   int tile_base;     // first global tile index of this problem
   int k_tiles;       // ceil(K / 64)
   int planes;        // planes of out / cin (1 or 3)
   float alpha, beta, diag;
   const float* mat_scale;  // per-matrix factor s_l, or null for 1
-  uint16_t* out;           // [planes][L][M][out_pitch] (EPI_STORE)
-  long long out_plane, out_mat;
-  int out_pitch;
   const uint16_t* cin;     // [planes][L][M][cin_pitch], null when beta == 0
   long long cin_plane, cin_mat;
   int cin_pitch;
-  // EPI_APPLY / EPI_OUT: caller matrices, rows x cols row-major (W dims)
-  int wrows, wcols;
-  int transposed;          // wide O(i,j) lands at W(j,i)
-  int w_f32;               // 1: fp32 W/Out, 0: bf16
-  int w_vec;               // rows of W are 16-byte aligned for vector access
-  float decay, lrs;        // W <- decay*W - lrs*O
-  const int* flags;        // skip matrices whose flag is set (EPI_APPLY)
-  int flag_offset;
-  void* wtab[MUON_MAX_BATCH];
 };
 
 struct GemmParams {

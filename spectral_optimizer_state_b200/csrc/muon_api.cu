@@ -275,8 +275,7 @@ uint16_t* ws_at(muon_ctx* c, size_t off) {
 enum Phase { PH_GRAM, PH_POLY, PH_UPDATE };
 
 // Fill one GEMM problem for group p, phase ph of iteration `it`.
-bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, bool last, bool step,
-                  const muon_hparams* hp, GemmProblem& q) {
+bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem& q) {
   std::memset(static_cast<void*>(&q), 0, sizeof(q));
   const float a = c->coeffs[3 * it], b = c->coeffs[3 * it + 1], cc = c->coeffs[3 * it + 2];
   const int src = it & 1, dst = (it + 1) & 1;
@@ -289,8 +288,6 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, bool last, 
   q.L = p.batch;
   q.nseg = p.planes == 3 ? 6 : 1;
   q.planes = p.planes;
-  q.flags = c->d_flags;
-  q.flag_offset = p.mat_off;
   const bool have_poly = cc != 0.f;
   const CUtensorMapSwizzle sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
   switch (ph) {
@@ -302,7 +299,7 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, bool last, 
       if (!encode_map(&q.tmOut, have_poly ? A : B, m, m, p.batch, p.planes, p.pitch_m, 32, 32, sw64))
         return false;
       q.M = m; q.N = m; q.K = n;
-      q.b_mn_major = 0; q.sym = 1; q.epi = EPI_STORE;
+      q.b_mn_major = 0; q.sym = 1;
       q.alpha = have_poly ? 1.f : b;
       q.beta = 0.f;
       q.diag = have_poly ? 0.f : a;
@@ -314,7 +311,7 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, bool last, 
       q.tmB = q.tmA;
       if (!encode_map(&q.tmOut, B, m, m, p.batch, p.planes, p.pitch_m, 32, 32, sw64)) return false;
       q.M = m; q.N = m; q.K = m;
-      q.b_mn_major = 0; q.sym = 1; q.epi = EPI_STORE;
+      q.b_mn_major = 0; q.sym = 1;
       q.alpha = cc; q.beta = b; q.diag = a;
       q.cin = A; q.cin_plane = p.a_plane; q.cin_mat = p.a_mat; q.cin_pitch = p.pitch_m;
       break;
@@ -326,23 +323,7 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, bool last, 
       q.b_mn_major = 1; q.sym = 0;
       q.alpha = 1.f; q.beta = 0.f; q.diag = 0.f;
       q.mat_scale = it == 0 ? c->d_s1 + p.mat_off : nullptr;
-      if (!last) {
-        q.epi = EPI_STORE;
-        if (!encode_map(&q.tmOut, Xn, n, m, p.batch, p.planes, p.pitch_n, 32, 32, sw64)) return false;
-      } else {
-        q.epi = step ? EPI_APPLY : EPI_OUT;
-        q.wrows = p.rows; q.wcols = p.cols; q.transposed = p.transposed; q.w_f32 = p.f32;
-        bool vec = (p.cols % (p.f32 ? 4 : 8)) == 0;
-        for (int l = 0; l < p.batch; ++l) {
-          q.wtab[l] = p.w[l];
-          if (reinterpret_cast<uintptr_t>(p.w[l]) % 16) vec = false;
-        }
-        q.w_vec = vec;
-        if (step) {
-          q.decay = 1.0f - hp->lr * hp->weight_decay;
-          q.lrs = hp->lr * shape_scale(p.rows, p.cols, hp->scale_mode);
-        }
-      }
+      if (!encode_map(&q.tmOut, Xn, n, m, p.batch, p.planes, p.pitch_n, 32, 32, sw64)) return false;
       break;
     }
   }
@@ -391,7 +372,6 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
   // k Newton-Schulz iterations; each phase covers up to two groups per launch.
   GemmParams gp;
   for (int it = 0; it < c->k; ++it) {
-    const bool last = it == c->k - 1;
     const bool have_poly = c->coeffs[3 * it + 2] != 0.f;
     for (int ph = PH_GRAM; ph <= PH_UPDATE; ++ph) {
       if (ph == PH_POLY && !have_poly) continue;
@@ -401,7 +381,7 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
         int tiles = 0;
         for (size_t g = g0; g < std::min(plans.size(), g0 + kMaxProblems); ++g) {
           GemmProblem& q = gp.prob[gp.nprob];
-          if (!fill_problem(c, plans[g], static_cast<Phase>(ph), it, last, step, hp, q))
+          if (!fill_problem(c, plans[g], static_cast<Phase>(ph), it, q))
             return cuda_fail(cudaErrorInvalidValue, "tensor map encoding");
           q.tile_base = tiles;
           tiles += q.tiles_per_matrix * q.L;
@@ -414,6 +394,29 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
         prof_end(c, slot, s);
       }
     }
+  }
+  // K5: scale + decoupled decay applied to W (or the plain copy to Out).
+  for (auto& p : plans) {
+    ApplyParams ap;
+    std::memset(static_cast<void*>(&ap), 0, sizeof(ap));
+    for (int l = 0; l < p.batch; ++l) ap.w[l] = p.w[l];
+    ap.o = ws_at(c, p.off_x[c->k & 1]);
+    ap.o_plane = p.x_plane;
+    ap.o_mat = p.x_mat;
+    ap.pitch = p.pitch_n;
+    ap.rows = p.rows;
+    ap.cols = p.cols;
+    ap.planes = p.planes;
+    ap.apply = step ? 1 : 0;
+    if (step) {
+      ap.decay = 1.0f - hp->lr * hp->weight_decay;
+      ap.lrs = hp->lr * shape_scale(p.rows, p.cols, hp->scale_mode);
+      ap.flags = c->d_flags + p.mat_off;
+    }
+    ap.nblk = momentum_blocks_per_matrix(p.rows, p.cols);
+    const int slot = prof_begin(c, MUON_KERNEL_APPLY, s);
+    MUON_CUDA(launch_apply(ap, p.batch, p.f32 != 0, s), "apply kernel");
+    prof_end(c, slot, s);
   }
   c->last_count = total;
   c->last_stream = s;
