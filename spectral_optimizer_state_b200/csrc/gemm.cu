@@ -58,6 +58,10 @@ struct Tile {
   int pi, l, m0, n0, nw;
 };
 
+// Tile t of the launch: problem, matrix, first row (multiple of TM), first
+// column and width (a multiple of NG, at most BN).  Symmetric outputs start
+// each TM-row block at its diagonal block.
+template <int TM, int NG>
 __device__ __forceinline__ Tile decode_tile(const GemmParams& P, int t) {
   Tile ti;
   ti.pi = (P.nprob > 1 && t >= P.prob[1].tile_base) ? 1 : 0;
@@ -68,20 +72,20 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& P, int t) {
   if (q.sym) {
     int mb = 0;
     for (;;) {
-      const int cnt = (q.M - BM * mb + BN - 1) / BN;
+      const int cnt = (q.M - TM * mb + BN - 1) / BN;
       if (r < cnt) break;
       r -= cnt;
       ++mb;
     }
-    ti.m0 = BM * mb;
-    ti.n0 = BM * mb + BN * r;
+    ti.m0 = TM * mb;
+    ti.n0 = TM * mb + BN * r;
   } else {
     const int tn = (q.N + BN - 1) / BN;
     const int mb = r / tn;
-    ti.m0 = BM * mb;
+    ti.m0 = TM * mb;
     ti.n0 = (r - mb * tn) * BN;
   }
-  const int nw = ((q.N - ti.n0 + 63) / 64) * 64;
+  const int nw = ((q.N - ti.n0 + NG - 1) / NG) * NG;
   ti.nw = nw < BN ? nw : BN;
   return ti;
 }
@@ -204,6 +208,47 @@ __device__ __forceinline__ void store_chunk(const CUtensorMap* map, uint32_t sta
   sb ^= 1;
 }
 
+// One warp's share of a finished accumulator tile: TMEM rows row0..row0+31
+// (this warp's lane quarter), 32-column chunks c_first, c_first + 64, ...
+// v = alpha s_l acc + beta cin + diag on the diagonal, split into planes and
+// stored through TMA; columns from `mirror_from` on are also stored transposed.
+__device__ __forceinline__ void epilogue_warp_tile(const GemmProblem& q, const Tile& ti, uint32_t tbase,
+                                                   int row0, int lane, int c_first, int mirror_from,
+                                                   uint32_t my_stage, int& sb) {
+  if (row0 >= q.M) return;
+  const int row = row0 + lane;
+  const float scale = q.alpha * (q.mat_scale != nullptr ? q.mat_scale[ti.l] : 1.0f);
+  for (int c = c_first; c < ti.nw; c += 64) {
+    const int j0 = ti.n0 + c;
+    if (j0 >= q.N) break;
+    const int nv = min(32, q.N - j0);
+    uint32_t r[32];
+    __syncwarp();  // tcgen05.ld is warp-collective
+    tmem_load_32cols(tbase + c, r);
+    tmem_load_wait();
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = scale * __uint_as_float(r[i]);
+    if (q.cin != nullptr && row < q.M) add_cin(q, ti.l, row, j0, nv, v);
+    if (q.diag != 0.f) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (j0 + i == row) v[i] += q.diag;
+    }
+    const bool mirror = q.sym && (j0 >= mirror_from);
+    for (int p = 0; p < q.planes; ++p) {
+      uint16_t b[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        b[i] = float_to_bf16_bits(v[i]);
+        v[i] -= bf16_bits_to_float(b[i]);  // residual for the next plane
+      }
+      store_chunk<false>(&q.tmOut, my_stage, sb, lane, b, j0, row0, ti.l, p);
+      if (mirror) store_chunk<true>(&q.tmOut, my_stage, sb, lane, b, row0, j0, ti.l, p);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ kernel
 __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_constant__ GemmParams P) {
   extern __shared__ uint8_t smem_raw[];
@@ -260,7 +305,7 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
       uint32_t it = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < P.total_tiles; t += gridDim.x) {
-        const Tile ti = decode_tile(P, t);
+        const Tile ti = decode_tile<BM, 64>(P, t);
         const GemmProblem& q = P.prob[ti.pi];
         const int nk = q.k_tiles * q.nseg;
         const uint32_t bbytes = q.b_mn_major ? static_cast<uint32_t>(ti.nw / 64) * MNMAJ_BOX_BYTES
@@ -302,7 +347,7 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
       int local = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < P.total_tiles; t += gridDim.x, ++local) {
-        const Tile ti = decode_tile(P, t);
+        const Tile ti = decode_tile<BM, 64>(P, t);
         const GemmProblem& q = P.prob[ti.pi];
         const int acc = local & 1;
         const uint32_t aph = (local >> 1) & 1;
@@ -350,47 +395,14 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
     int sb = 0;
     int local = 0;
     for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++local) {
-      const Tile ti = decode_tile(P, t);
+      const Tile ti = decode_tile<BM, 64>(P, t);
       const GemmProblem& q = P.prob[ti.pi];
       const int acc = local & 1;
       const uint32_t aph = (local >> 1) & 1;
       if (!mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, P.status)) break;
       tc_fence_after();
-      const int row0 = ti.m0 + 32 * quarter;
-      const int row = row0 + lane;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * ACC_COLS;
-      const float scale = q.alpha * (q.mat_scale != nullptr ? q.mat_scale[ti.l] : 1.0f);
-      if (row0 < q.M) {
-        for (int c = 32 * half; c < ti.nw; c += 64) {
-          const int j0 = ti.n0 + c;
-          if (j0 >= q.N) break;
-          const int nv = min(32, q.N - j0);
-          uint32_t r[32];
-          __syncwarp();  // tcgen05.ld is warp-collective
-          tmem_load_32cols(tbase + c, r);
-          tmem_load_wait();
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = scale * __uint_as_float(r[i]);
-          if (q.cin != nullptr && row < q.M) add_cin(q, ti.l, row, j0, nv, v);
-          if (q.diag != 0.f) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (j0 + i == row) v[i] += q.diag;
-          }
-          const bool mirror = q.sym && (j0 >= ti.m0 + BM);
-          for (int p = 0; p < q.planes; ++p) {
-            uint16_t b[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              b[i] = float_to_bf16_bits(v[i]);
-              v[i] -= bf16_bits_to_float(b[i]);  // residual for the next plane
-            }
-            store_chunk<false>(&q.tmOut, my_stage, sb, lane, b, j0, row0, ti.l, p);
-            if (mirror) store_chunk<true>(&q.tmOut, my_stage, sb, lane, b, row0, j0, ti.l, p);
-          }
-        }
-      }
+      epilogue_warp_tile(q, ti, tbase, ti.m0 + 32 * quarter, lane, 32 * half, ti.m0 + BM, my_stage, sb);
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
     }
@@ -404,33 +416,256 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
   }
 }
 
+
+// ------------------------------------------------------------------ CTA-pair kernel
+// cta_group::2: a cluster of two CTAs computes a 256 x 256 tile.  CTA r holds
+// rows [128 r, 128 r + 128) of the A tile and columns [r N/2, (r+1) N/2) of
+// the B tile in its own shared memory; the leader (rank 0) issues the MMAs,
+// which read both CTAs' halves and write each CTA's 128 accumulator rows to
+// its own TMEM.  Every CTA needs only 32 KB per 64-deep stage (six stages in
+// flight) instead of 48 KB, for the same MMA time per stage.
+//   full[s]   leader only: its producer posts the bytes of both CTAs; the
+//             follower's loads complete their bytes on the leader's barrier.
+//   empty[s]  both CTAs: the leader's commit arrives on both (multicast).
+//   tfull[a]  both CTAs: likewise, when a tile's MMAs are done.
+//   tempty[a] leader only: one arrival per epilogue warp of either CTA.
+constexpr int PBM = 256;                       // pair tile rows
+constexpr int PSTAGES = 6;
+constexpr uint32_t PA_BYTES = 128 * BK * 2;    // 16 KB: this CTA's A rows
+constexpr uint32_t PB_BYTES = 128 * BK * 2;    // 16 KB: this CTA's half of B
+constexpr uint32_t PSTAGE_BYTES = PA_BYTES + PB_BYTES;
+constexpr uint32_t PBOX_BYTES = 64 * BK * 2;   // any B box {64, 64}
+constexpr int PNUM_BARS = 2 * PSTAGES + 5;
+constexpr uint32_t PBAR_BYTES = 8 * PNUM_BARS + 16;
+
+__global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_constant__ GemmParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t stage_area = base + PSTAGES * PSTAGE_BYTES;
+  const uint32_t bar0 = stage_area + EPI_WARPS * STAGING_BYTES_PER_WARP;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + (bar0 - base) + 8 * PNUM_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (PSTAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * PSTAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * PSTAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * PSTAGES + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_cta_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PSTAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 2 * EPI_WARPS);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < P.nprob; ++i) {
+      tma_prefetch_map(&P.prob[i].tmA);
+      tma_prefetch_map(&P.prob[i].tmB);
+      tma_prefetch_map(&P.prob[i].tmOut);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_addr(tmem_holder), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised, TMEM address written
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < P.total_tiles; t += npairs) {
+        const Tile ti = decode_tile<PBM, 128>(P, t);
+        const GemmProblem& q = P.prob[ti.pi];
+        const int nk = q.k_tiles * q.nseg;
+        const int half_n = ti.nw >> 1;                 // this CTA's B columns (64 or 128)
+        const int nb = half_n / 64;                    // B boxes per stage
+        const int n_mine = ti.n0 + static_cast<int>(rank) * half_n;
+        const uint32_t pair_bytes = 2u * (PA_BYTES + static_cast<uint32_t>(nb) * PBOX_BYTES);
+        for (int kk = 0; kk < nk; ++kk, ++it) {
+          const int s = it % PSTAGES;
+          const uint32_t ph = (it / PSTAGES) & 1u;
+          if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, P.status)) {
+            ok = false;
+            break;
+          }
+          const int seg = kk / q.k_tiles;
+          const int kb = kk - seg * q.k_tiles;
+          int pa, pb;
+          segment_planes(q.nseg, seg, pa, pb);
+          const uint32_t sa = base + s * PSTAGE_BYTES;
+          const uint32_t sb = sa + PA_BYTES;
+          const uint32_t fb = map_shared_rank(full_bar(s), 0);  // the leader's full barrier
+          if (leader) mbar_arrive_expect_tx(full_bar(s), pair_bytes);
+          tma_load_4d_pair(sa, &q.tmA, fb, kb * BK, ti.m0 + 128 * static_cast<int>(rank), ti.l, pa);
+          for (int c = 0; c < nb; ++c) {
+            if (q.b_mn_major)
+              tma_load_4d_pair(sb + c * PBOX_BYTES, &q.tmB, fb, n_mine + 64 * c, kb * BK, ti.l, pb);
+            else
+              tma_load_4d_pair(sb + c * PBOX_BYTES, &q.tmB, fb, kb * BK, n_mine + 64 * c, ti.l, pb);
+          }
+        }
+      }
+      if (!ok) {
+        // The copies this thread started complete on the leader's barriers; give
+        // them a bounded time to land before the CTA may leave.
+        if (leader) {
+          const uint32_t n = it < PSTAGES ? it : PSTAGES;
+          for (uint32_t j = it - n; j < it; ++j) wait_drain(full_bar(j % PSTAGES), (j / PSTAGES) & 1u);
+        } else {
+          const uint64_t t0 = global_timer_ns();
+          while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ UMMA issuer (leader only)
+    if (lane == 0 && leader) {
+      uint32_t it = 0;
+      int local = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < P.total_tiles; t += npairs, ++local) {
+        const Tile ti = decode_tile<PBM, 128>(P, t);
+        const GemmProblem& q = P.prob[ti.pi];
+        const int acc = local & 1;
+        const uint32_t aph = (local >> 1) & 1;
+        if (!mbar_wait_bounded(tempty_bar(acc), aph ^ 1u, abort_flag, P.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        const uint32_t idesc = instr_desc_bf16(PBM, ti.nw, q.b_mn_major != 0);
+        const int nk = q.k_tiles * q.nseg;
+        for (int kk = 0; kk < nk; ++kk, ++it) {
+          const int s = it % PSTAGES;
+          const uint32_t ph = (it / PSTAGES) & 1u;
+          if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, P.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base + s * PSTAGE_BYTES;
+          const uint32_t sb = sa + PA_BYTES;
+#pragma unroll
+          for (int k4 = 0; k4 < BK / 16; ++k4) {
+            const uint64_t ad = smem_desc_sw128(sa + 32u * k4, 16u, 1024u);
+            const uint64_t bd = q.b_mn_major ? smem_desc_sw128(sb + 2048u * k4, PBOX_BYTES, 1024u)
+                                             : smem_desc_sw128(sb + 32u * k4, 16u, 1024u);
+            tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kk | k4) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair(empty_bar(s), 0x3);
+        }
+        if (ok) tc_commit_pair(tfull_bar(acc), 0x3);
+      }
+      if (!ok) {
+        tc_commit_pair(drain_bar, 0x1);
+        wait_drain(drain_bar, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (both CTAs)
+    const int e = warp - 2;
+    const int quarter = warp & 3;
+    const int half = e >> 2;
+    const uint32_t my_stage = stage_area + static_cast<uint32_t>(e) * STAGING_BYTES_PER_WARP;
+    int sb = 0;
+    int local = 0;
+    for (int t = pair; t < P.total_tiles; t += npairs, ++local) {
+      const Tile ti = decode_tile<PBM, 128>(P, t);
+      const GemmProblem& q = P.prob[ti.pi];
+      const int acc = local & 1;
+      const uint32_t aph = (local >> 1) & 1;
+      if (!mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, P.status)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * ACC_COLS;
+      epilogue_warp_tile(q, ti, tbase, ti.m0 + 128 * static_cast<int>(rank) + 32 * quarter, lane,
+                         32 * half, ti.m0 + PBM, my_stage, sb);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_shared_rank(tempty_bar(acc), 0));
+    }
+    if (lane == 0) bulk_wait_group_all();
+  }
+
+  __syncthreads();
+  cluster_sync_all();  // no MMA, load or arrival still targets the other CTA
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 }  // namespace
 
-size_t gemm_smem_bytes() {
+size_t gemm_smem_bytes(int kind) {
+  if (kind == GEMM_PAIR) return PSTAGES * PSTAGE_BYTES + EPI_WARPS * STAGING_BYTES_PER_WARP + PBAR_BYTES + 1024;
   return STAGES * STAGE_BYTES + EPI_WARPS * STAGING_BYTES_PER_WARP + BAR_BYTES + 1024;
 }
 
-int gemm_tiles_per_matrix(int M, int N, int sym) {
+int gemm_tiles_per_matrix(int kind, int M, int N, int sym) {
+  const int tm = kind == GEMM_PAIR ? PBM : BM;
   if (sym) {
     int n = 0;
-    for (int mb = 0; mb * BM < M; ++mb) n += (M - BM * mb + BN - 1) / BN;
+    for (int mb = 0; mb * tm < M; ++mb) n += (M - tm * mb + BN - 1) / BN;
     return n;
   }
-  return ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  return ((M + tm - 1) / tm) * ((N + BN - 1) / BN);
 }
 
-cudaError_t launch_gemm(const GemmParams& p, int grid, cudaStream_t stream) {
-  static int configured_device = -1;
+cudaError_t launch_gemm(const GemmParams& p, int kind, int units, cudaStream_t stream) {
+  static int configured_device[2] = {-1, -1};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (configured_device != dev) {
-    e = cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(gemm_smem_bytes()));
+  const void* fn = kind == GEMM_PAIR ? reinterpret_cast<const void*>(ns_gemm_pair_kernel)
+                                     : reinterpret_cast<const void*>(ns_gemm_kernel);
+  const int smem = static_cast<int>(gemm_smem_bytes(kind));
+  if (configured_device[kind] != dev) {
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    configured_device = dev;
+    configured_device[kind] = dev;
   }
-  ns_gemm_kernel<<<grid, THREADS, gemm_smem_bytes(), stream>>>(p);
+  if (kind == GEMM_PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * units, 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, ns_gemm_pair_kernel, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
+  ns_gemm_kernel<<<units, THREADS, smem, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -86,10 +86,17 @@ struct GemmParams {
   int* status;
 };
 
-size_t gemm_smem_bytes();
-cudaError_t launch_gemm(const GemmParams& p, int grid, cudaStream_t stream);
+// Two kernels share the problem description:
+//   single CTA: 128 x 256 tiles; B operand boxes {64, 128} (K-major) or {64, 64}.
+//   CTA pair (cta_group::2): 256 x 256 tiles, each CTA holds 128 rows of A and
+//   half of the tile's N columns of B; B operand boxes {64, 64}.
+enum GemmKind : int { GEMM_SINGLE = 0, GEMM_PAIR = 1 };
+
+size_t gemm_smem_bytes(int kind);
+// `units`: CTAs (single) or CTA pairs (pair) to launch.
+cudaError_t launch_gemm(const GemmParams& p, int kind, int units, cudaStream_t stream);
 
 // Tiles one matrix of this problem shape contributes.
-int gemm_tiles_per_matrix(int M, int N, int sym);
+int gemm_tiles_per_matrix(int kind, int M, int N, int sym);
 
 }  // namespace muon

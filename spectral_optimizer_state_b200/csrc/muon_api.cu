@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -111,6 +112,7 @@ struct muon_ctx {
   unsigned* d_counters = nullptr;
   float* d_partials = nullptr;
   int* d_status = nullptr;
+  int gemm_kind = GEMM_PAIR;  // MUON_GEMM=single selects the single-CTA kernel
   int last_count = 0;
   cudaStream_t last_stream = nullptr;
   bool pending = false;
@@ -290,12 +292,14 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
   q.planes = p.planes;
   const bool have_poly = cc != 0.f;
   const CUtensorMapSwizzle sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
+  // K-major B operand box height: 128 rows (single CTA) or 64 (each CTA of a pair)
+  const int kb_rows = c->gemm_kind == GEMM_PAIR ? 64 : 128;
   switch (ph) {
     case PH_GRAM:
       // A = s2 * X X^T; with c = 0 the polynomial is linear and the Gram
       // epilogue writes B' = b A + a I directly.
       if (!encode_map(&q.tmA, X, n, m, p.batch, p.planes, p.pitch_n, 64, 128)) return false;
-      q.tmB = q.tmA;
+      if (!encode_map(&q.tmB, X, n, m, p.batch, p.planes, p.pitch_n, 64, kb_rows)) return false;
       if (!encode_map(&q.tmOut, have_poly ? A : B, m, m, p.batch, p.planes, p.pitch_m, 32, 32, sw64))
         return false;
       q.M = m; q.N = m; q.K = n;
@@ -308,7 +312,7 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
     case PH_POLY:
       // B' = c A A + b A + a I
       if (!encode_map(&q.tmA, A, m, m, p.batch, p.planes, p.pitch_m, 64, 128)) return false;
-      q.tmB = q.tmA;
+      if (!encode_map(&q.tmB, A, m, m, p.batch, p.planes, p.pitch_m, 64, kb_rows)) return false;
       if (!encode_map(&q.tmOut, B, m, m, p.batch, p.planes, p.pitch_m, 32, 32, sw64)) return false;
       q.M = m; q.N = m; q.K = m;
       q.b_mn_major = 0; q.sym = 1;
@@ -327,7 +331,7 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
       break;
     }
   }
-  q.tiles_per_matrix = gemm_tiles_per_matrix(q.M, q.N, q.sym);
+  q.tiles_per_matrix = gemm_tiles_per_matrix(c->gemm_kind, q.M, q.N, q.sym);
   q.k_tiles = (q.K + 63) / 64;
   return true;
 }
@@ -388,9 +392,9 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
           ++gp.nprob;
         }
         gp.total_tiles = tiles;
-        const int grid = std::min(tiles, c->sm_count);
+        const int units = std::min(tiles, c->gemm_kind == GEMM_PAIR ? c->sm_count / 2 : c->sm_count);
         const int slot = prof_begin(c, MUON_KERNEL_GRAM + (ph - PH_GRAM), s);
-        MUON_CUDA(launch_gemm(gp, grid, s), "newton-schulz gemm");
+        MUON_CUDA(launch_gemm(gp, c->gemm_kind, units, s), "newton-schulz gemm");
         prof_end(c, slot, s);
       }
     }
@@ -479,6 +483,9 @@ muon_status muon_create(muon_ctx** out, int device) {
   c->sm_count = prop.multiProcessorCount;
   for (int i = 0; i < 5; ++i) std::memcpy(&c->coeffs[3 * i], kQuintic, sizeof(kQuintic));
   c->k = 5;
+  if (const char* g = std::getenv("MUON_GEMM")) {
+    if (std::strcmp(g, "single") == 0) c->gemm_kind = GEMM_SINGLE;
+  }
   if (cudaMalloc(&c->d_status, sizeof(int)) != cudaSuccess) {
     cudaGetLastError();
     delete c;

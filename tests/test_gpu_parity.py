@@ -328,3 +328,31 @@ def test_ill_conditioned_variant(ctx, dtype):
         else:
             assert dominant_subspace_error(to_numpy(o), ref, g) <= BF16_TOL
             assert full < 0.15  # reported; single-pass bf16 cannot resolve sigma ~1e-6 directions
+
+
+def test_single_cta_and_pair_kernels_agree():
+    """The single-CTA (128 x 256) and CTA-pair (256 x 256) kernels compute the same products."""
+    import os
+    import torch
+    from spectral_optimizer_state_b200 import Muon
+    outs = {}
+    shapes = [(200, 328), (768, 1536), (3352, 768)]
+    for kind in ("single", "pair"):
+        os.environ["MUON_GEMM"] = kind
+        try:
+            m = Muon(0)
+        finally:
+            del os.environ["MUON_GEMM"]
+        m.set_coeffs(QUINTIC5)
+        res = []
+        for i, shape in enumerate(shapes):
+            X = [to_device(g, "bf16") for g in _inputs(shape, 2, seed=300 + i, kind="spike")]
+            Out = [torch.empty_like(x) for x in X]
+            m.ns_orthogonalize(X, Out, eps=1e-7)
+            assert m.status()[0] == 0
+            res.append([to_numpy(o) for o in Out])
+        m.close()
+        outs[kind] = res
+    for a_list, b_list in zip(outs["single"], outs["pair"]):
+        for a, b in zip(a_list, b_list):
+            assert rel_f(a, b) <= 5e-3

@@ -9,16 +9,19 @@ its [rows][pitch] buffer.
 import numpy as np
 import pytest
 
-BM, BN = 128, 256
+BN = 256
+KINDS = {"single": (128, 64), "pair": (256, 128)}  # (tile rows, column granularity)
 
 
-def tiles_per_matrix(M, N, sym):
+def tiles_per_matrix(M, N, sym, kind="single"):
+    BM = KINDS[kind][0]
     if sym:
         return sum((M - BM * mb + BN - 1) // BN for mb in range((M + BM - 1) // BM))
     return ((M + BM - 1) // BM) * ((N + BN - 1) // BN)
 
 
-def decode(M, N, sym, r):
+def decode(M, N, sym, r, kind="single"):
+    BM, NG = KINDS[kind]
     if sym:
         mb = 0
         while True:
@@ -32,7 +35,7 @@ def decode(M, N, sym, r):
         tn = (N + BN - 1) // BN
         mb = r // tn
         m0, n0 = BM * mb, (r - mb * tn) * BN
-    nw = min(BN, (N - n0 + 63) // 64 * 64)
+    nw = min(BN, (N - n0 + NG - 1) // NG * NG)
     return m0, n0, nw
 
 
@@ -40,15 +43,17 @@ SHAPES = [(64, 96), (128, 128), (200, 328), (257, 700), (96, 1000), (37, 53), (7
           (2048, 4096), (2048, 8768), (8192, 8192), (1, 1), (130, 260)]
 
 
+@pytest.mark.parametrize("kind", sorted(KINDS))
 @pytest.mark.parametrize("m,n", SHAPES)
-def test_symmetric_cover_exactly_once(m, n):
+def test_symmetric_cover_exactly_once(m, n, kind):
     if m > 2048:
         pytest.skip("large")
+    BM, NG = KINDS[kind]
     pitch = (m + 7) // 8 * 8
     hits = np.zeros((m, pitch), np.int32)
-    for r in range(tiles_per_matrix(m, m, 1)):
-        m0, n0, nw = decode(m, m, 1, r)
-        assert n0 % 64 == 0 and nw % 64 == 0 and 64 <= nw <= 256 and n0 >= m0
+    for r in range(tiles_per_matrix(m, m, 1, kind)):
+        m0, n0, nw = decode(m, m, 1, r, kind)
+        assert n0 % 64 == 0 and nw % NG == 0 and NG <= nw <= 256 and n0 >= m0
         rows = np.arange(m0, min(m0 + BM, m))
         for c in range(0, nw, 32):
             j0 = n0 + c
@@ -62,26 +67,33 @@ def test_symmetric_cover_exactly_once(m, n):
     assert np.all(hits[:, m:] == 0)
 
 
+@pytest.mark.parametrize("kind", sorted(KINDS))
 @pytest.mark.parametrize("m,n", SHAPES)
-def test_update_cover_exactly_once(m, n):
+def test_update_cover_exactly_once(m, n, kind):
     if m * n > 2048 * 8768:
         pytest.skip("large")
+    BM, NG = KINDS[kind]
     hits = np.zeros((m, n), np.int32)
-    for r in range(tiles_per_matrix(m, n, 0)):
-        m0, n0, nw = decode(m, n, 0, r)
-        assert n0 % 64 == 0 and nw % 64 == 0 and nw <= 256
-        assert n0 + nw <= (n + 63) // 64 * 64
+    for r in range(tiles_per_matrix(m, n, 0, kind)):
+        m0, n0, nw = decode(m, n, 0, r, kind)
+        assert n0 % 64 == 0 and nw % NG == 0 and nw <= 256
+        assert n0 + nw <= (n + NG - 1) // NG * NG
         rows = slice(m0, min(m0 + BM, m))
         hits[rows, n0:min(n0 + nw, n)] += 1
     assert np.all(hits == 1)
 
 
+@pytest.mark.parametrize("kind", sorted(KINDS))
 @pytest.mark.parametrize("m,n", SHAPES)
-def test_tma_coordinates_aligned(m, n):
+def test_tma_coordinates_aligned(m, n, kind):
     for sym, N, K in ((1, m, n), (1, m, m), (0, n, m)):
-        for r in range(min(tiles_per_matrix(m, N, sym), 4000)):
-            m0, n0, nw = decode(m, N, sym, r)
+        for r in range(min(tiles_per_matrix(m, N, sym, kind), 4000)):
+            m0, n0, nw = decode(m, N, sym, r, kind)
             for kb in range((K + 63) // 64):
                 assert (kb * 64 * 2) % 16 == 0  # A / K-major B: x = k
-            for c in range(nw // 64):
-                assert ((n0 + 64 * c) * 2) % 16 == 0  # MN-major B: x = n
+            half = nw // 2 if kind == "pair" else nw
+            for rank in ((0, 1) if kind == "pair" else (0,)):
+                for c in range(half // 64):
+                    x = n0 + rank * half + 64 * c
+                    assert (x * 2) % 16 == 0  # MN-major B: x = n
+                    assert half % 64 == 0
