@@ -389,8 +389,9 @@ def main():
 
     n_mats = sum(L for _, L, _, _ in groups)
     steps_per_s = world * args.steps / (ms / 1e3)
-    gemm_launches = sum(prof[k][0] for k in ("gram", "poly", "update"))
-    gemm_ms = sum(prof[k][1] for k in ("gram", "poly", "update"))
+    gemm_kinds = ("gram", "poly", "update", "ns_fused")
+    gemm_launches = sum(prof[k][0] for k in gemm_kinds)
+    gemm_ms = sum(prof[k][1] for k in gemm_kinds)
     flops_timed = ns_flops(groups) * args.steps
     achieved_tf = flops_timed / (gemm_ms / 1e3) / 1e12
     burst, sustained = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]

@@ -180,7 +180,8 @@ typedef enum {
   MUON_KERNEL_POLY = 2,     /* B = b A + c A A                          */
   MUON_KERNEL_UPDATE = 3,   /* X <- s B' X  with B' = aI + bA + cAA     */
   MUON_KERNEL_APPLY = 4,    /* W <- (1 - lr wd) W - lr s O              */
-  MUON_KERNEL_KINDS = 5
+  MUON_KERNEL_NS_FUSED = 5, /* several phases (and iterations) in one persistent launch */
+  MUON_KERNEL_KINDS = 6
 } muon_kernel_kind;
 
 typedef struct {

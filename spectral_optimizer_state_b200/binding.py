@@ -38,7 +38,7 @@ EXPORTS = (
     "muon_ns_orthogonalize", "muon_get_status", "muon_get_norms", "muon_workspace_bytes",
     "muon_profile_enable", "muon_profile_read",
 )
-KERNEL_KINDS = ("momentum", "gram", "poly", "update", "apply")
+KERNEL_KINDS = ("momentum", "gram", "poly", "update", "apply", "ns_fused")
 
 
 class MuonError(RuntimeError):
@@ -56,7 +56,7 @@ class Hparams(ctypes.Structure):
 
 
 class Profile(ctypes.Structure):
-    _fields_ = [("launches", ctypes.c_int * 5), ("ms", ctypes.c_double * 5)]
+    _fields_ = [("launches", ctypes.c_int * 6), ("ms", ctypes.c_double * 6)]
 
 
 class Group(ctypes.Structure):

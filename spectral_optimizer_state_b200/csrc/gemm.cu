@@ -45,7 +45,7 @@ constexpr uint32_t B_BYTES = BN * BK * 2;     // 32 KB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t KMAJ_BOX_BYTES = 128 * BK * 2;  // box {64 K, 128 rows}
 constexpr uint32_t MNMAJ_BOX_BYTES = 64 * BK * 2;  // box {64 N, 64 K rows}
-constexpr int EPI_WARPS = 8;
+constexpr int EPI_WARPS = kEpilogueWarps;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint32_t STAGING_BYTES_PER_WARP = 2 * 2048;  // two 32 x 32 bf16 store tiles
 constexpr uint32_t TMEM_COLS = 512;
@@ -64,7 +64,13 @@ struct Tile {
 template <int TM, int NG>
 __device__ __forceinline__ Tile decode_tile(const GemmParams& P, int t) {
   Tile ti;
-  ti.pi = (P.nprob > 1 && t >= P.prob[1].tile_base) ? 1 : 0;
+  int lo = 0, hi = P.nprob - 1;  // last problem whose first tile is <= t
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (P.prob[mid].tile_base <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  ti.pi = lo;
   const GemmProblem& q = P.prob[ti.pi];
   const int local = t - q.tile_base;
   ti.l = local / q.tiles_per_matrix;
@@ -139,14 +145,14 @@ __device__ __forceinline__ void add_cin(const GemmProblem& q, int l, int row, in
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         float f[8];
-        unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(src) + h), f);
+        unpack_bf16x8(__ldcg(reinterpret_cast<const uint4*>(src) + h), f);
 #pragma unroll
         for (int t = 0; t < 8; ++t) c[8 * h + t] += f[t];
       }
     } else {
 #pragma unroll
       for (int t = 0; t < 32; ++t)
-        if (t < nv) c[t] += bf16_bits_to_float(src[t]);
+        if (t < nv) c[t] += bf16_bits_to_float(__ldcg(src + t));
     }
   }
 #pragma unroll
@@ -307,6 +313,14 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
       for (int t = blockIdx.x; ok && t < P.total_tiles; t += gridDim.x) {
         const Tile ti = decode_tile<BM, 64>(P, t);
         const GemmProblem& q = P.prob[ti.pi];
+        if (q.done_dep != nullptr) {
+          // the previous phase of this matrix must have landed before it is read
+          if (!wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status)) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_global();
+        }
         const int nk = q.k_tiles * q.nseg;
         const uint32_t bbytes = q.b_mn_major ? static_cast<uint32_t>(ti.nw / 64) * MNMAJ_BOX_BYTES
                                              : static_cast<uint32_t>((ti.nw + 127) / 128) * KMAJ_BOX_BYTES;
@@ -366,7 +380,6 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
             ok = false;
             break;
           }
-          tc_fence_after();
           const uint32_t sa = base + s * STAGE_BYTES;
           const uint32_t sb = sa + A_BYTES;
 #pragma unroll
@@ -402,7 +415,21 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
       if (!mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, P.status)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * ACC_COLS;
+      if (q.cin != nullptr && q.done_dep != nullptr) {
+        // cin was written earlier in this launch: acquire it for this warp's plain loads
+        if (!wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status)) break;
+      }
       epilogue_warp_tile(q, ti, tbase, ti.m0 + 32 * quarter, lane, 32 * half, ti.m0 + BM, my_stage, sb);
+      if (q.done_self != nullptr) {
+        // this warp's stores of the tile are complete and visible: count it done
+        if (lane == 0) {
+          bulk_wait_group_all();
+          fence_proxy_async_global();
+          __threadfence();
+          atomicAdd(q.done_self + ti.l, 1u);
+        }
+        __syncwarp();
+      }
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
     }
@@ -566,7 +593,6 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_c
             ok = false;
             break;
           }
-          tc_fence_after();
           const uint32_t sa = base + s * PSTAGE_BYTES;
           const uint32_t sb = sa + PA_BYTES;
 #pragma unroll

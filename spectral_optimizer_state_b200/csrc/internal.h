@@ -57,7 +57,11 @@ cudaError_t launch_apply(const ApplyParams& p, int batch, bool w_f32, cudaStream
 // The epilogue forms  v = alpha * s_l * acc + beta * cin + (row == col ? diag : 0)
 // and writes it as planes through TMA tensor stores (mirrored too if sym).
 
-constexpr int kMaxProblems = 2;
+// Epilogue warps per CTA (each signals a finished tile once).
+constexpr int kEpilogueWarps = 8;
+
+// Problems (one per group, iteration and phase) a single launch may carry.
+constexpr int kMaxProblems = 30;
 
 struct alignas(64) GemmProblem {
   CUtensorMap tmA;  // A operand [planes][L][M][K], K contiguous, box {64, 128}
@@ -77,6 +81,13 @@ struct alignas(64) GemmProblem {
   const uint16_t* cin;     // [planes][L][M][cin_pitch], null when beta == 0
   long long cin_plane, cin_mat;
   int cin_pitch;
+  // Cross-phase ordering inside one launch.  Every epilogue warp that finishes
+  // its share of a tile of matrix l adds 1 to done_self[l] once the tile's
+  // stores have landed; a tile of matrix l may load only after
+  // done_dep[l] >= dep_target (the previous phase of that matrix finished).
+  unsigned* done_self;       // [L], or null
+  const unsigned* done_dep;  // [L], or null when the inputs were written by an earlier launch
+  unsigned dep_target;
 };
 
 struct GemmParams {

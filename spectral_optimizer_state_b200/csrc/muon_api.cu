@@ -112,7 +112,8 @@ struct muon_ctx {
   unsigned* d_counters = nullptr;
   float* d_partials = nullptr;
   int* d_status = nullptr;
-  int gemm_kind = GEMM_PAIR;  // MUON_GEMM=single selects the single-CTA kernel
+  unsigned* d_done = nullptr;  // [kMaxProblems][MUON_MAX_BATCH] phase-completion counters
+  int gemm_kind = GEMM_SINGLE;  // MUON_GEMM=pair selects the CTA-pair kernel
   int last_count = 0;
   cudaStream_t last_stream = nullptr;
   bool pending = false;
@@ -373,32 +374,57 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
     prof_end(c, slot, s);
   }
 
-  // k Newton-Schulz iterations; each phase covers up to two groups per launch.
-  GemmParams gp;
+  // k Newton-Schulz iterations.  The single-CTA kernel runs every phase of
+  // every group in one persistent launch (as many as fit in one parameter
+  // block), ordered phase by phase; per-(phase, matrix) counters let a tile
+  // start as soon as the previous phase of its own matrix has landed.  The
+  // CTA-pair kernel runs one launch per phase.
+  std::vector<Phase> seq_ph;
+  std::vector<int> seq_it;
   for (int it = 0; it < c->k; ++it) {
-    const bool have_poly = c->coeffs[3 * it + 2] != 0.f;
     for (int ph = PH_GRAM; ph <= PH_UPDATE; ++ph) {
-      if (ph == PH_POLY && !have_poly) continue;
-      for (size_t g0 = 0; g0 < plans.size(); g0 += kMaxProblems) {
-        std::memset(static_cast<void*>(&gp), 0, sizeof(gp));
-        gp.status = c->d_status;
-        int tiles = 0;
-        for (size_t g = g0; g < std::min(plans.size(), g0 + kMaxProblems); ++g) {
-          GemmProblem& q = gp.prob[gp.nprob];
-          if (!fill_problem(c, plans[g], static_cast<Phase>(ph), it, q))
-            return cuda_fail(cudaErrorInvalidValue, "tensor map encoding");
-          q.tile_base = tiles;
-          tiles += q.tiles_per_matrix * q.L;
-          ++gp.nprob;
-        }
-        gp.total_tiles = tiles;
-        const int units = std::min(tiles, c->gemm_kind == GEMM_PAIR ? c->sm_count / 2 : c->sm_count);
-        const int slot = prof_begin(c, MUON_KERNEL_GRAM + (ph - PH_GRAM), s);
-        MUON_CUDA(launch_gemm(gp, c->gemm_kind, units, s), "newton-schulz gemm");
-        prof_end(c, slot, s);
-      }
+      if (ph == PH_POLY && c->coeffs[3 * it + 2] == 0.f) continue;
+      seq_ph.push_back(static_cast<Phase>(ph));
+      seq_it.push_back(it);
     }
   }
+  const bool persistent = c->gemm_kind == GEMM_SINGLE;
+  const int ng = static_cast<int>(plans.size());
+  const int phases_per_launch = persistent ? std::max(1, kMaxProblems / ng) : 1;
+  GemmParams gp;
+  for (size_t p0 = 0; p0 < seq_ph.size(); p0 += phases_per_launch) {
+    const size_t p1 = std::min(seq_ph.size(), p0 + phases_per_launch);
+    std::memset(static_cast<void*>(&gp), 0, sizeof(gp));
+    gp.status = c->d_status;
+    int tiles = 0;
+    for (size_t pi = p0; pi < p1; ++pi) {
+      for (int g = 0; g < ng; ++g) {
+        GemmProblem& q = gp.prob[gp.nprob];
+        if (!fill_problem(c, plans[g], seq_ph[pi], seq_it[pi], q))
+          return cuda_fail(cudaErrorInvalidValue, "tensor map encoding");
+        q.tile_base = tiles;
+        tiles += q.tiles_per_matrix * q.L;
+        if (persistent) {
+          q.done_self = c->d_done + static_cast<size_t>(gp.nprob) * MUON_MAX_BATCH;
+          if (pi > p0) {
+            const GemmProblem& prev = gp.prob[gp.nprob - ng];  // same group, previous phase
+            q.done_dep = prev.done_self;
+            q.dep_target = static_cast<unsigned>(kEpilogueWarps * prev.tiles_per_matrix);
+          }
+        }
+        ++gp.nprob;
+      }
+    }
+    gp.total_tiles = tiles;
+    if (persistent)
+      MUON_CUDA(cudaMemsetAsync(c->d_done, 0, sizeof(unsigned) * gp.nprob * MUON_MAX_BATCH, s), "clear counters");
+    const int units = std::min(tiles, persistent ? c->sm_count : c->sm_count / 2);
+    const int kind = p1 - p0 > 1 ? MUON_KERNEL_NS_FUSED : MUON_KERNEL_GRAM + (seq_ph[p0] - PH_GRAM);
+    const int slot = prof_begin(c, kind, s);
+    MUON_CUDA(launch_gemm(gp, c->gemm_kind, units, s), "newton-schulz gemm");
+    prof_end(c, slot, s);
+  }
+
   // K5: scale + decoupled decay applied to W (or the plain copy to Out).
   for (auto& p : plans) {
     ApplyParams ap;
@@ -484,7 +510,7 @@ muon_status muon_create(muon_ctx** out, int device) {
   for (int i = 0; i < 5; ++i) std::memcpy(&c->coeffs[3 * i], kQuintic, sizeof(kQuintic));
   c->k = 5;
   if (const char* g = std::getenv("MUON_GEMM")) {
-    if (std::strcmp(g, "single") == 0) c->gemm_kind = GEMM_SINGLE;
+    if (std::strcmp(g, "pair") == 0) c->gemm_kind = GEMM_PAIR;
   }
   if (cudaMalloc(&c->d_status, sizeof(int)) != cudaSuccess) {
     cudaGetLastError();
@@ -492,6 +518,12 @@ muon_status muon_create(muon_ctx** out, int device) {
     return MUON_ERR_ALLOC;
   }
   cudaMemset(c->d_status, 0, sizeof(int));
+  if (cudaMalloc(&c->d_done, sizeof(unsigned) * kMaxProblems * MUON_MAX_BATCH) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(c->d_status);
+    delete c;
+    return MUON_ERR_ALLOC;
+  }
   *out = c;
   return MUON_OK;
 }
@@ -508,6 +540,7 @@ muon_status muon_destroy(muon_ctx* c) {
   cudaFree(c->d_counters);
   cudaFree(c->d_partials);
   cudaFree(c->d_status);
+  cudaFree(c->d_done);
   cudaFree(c->d_stage);
   for (cudaEvent_t e : c->events) cudaEventDestroy(e);
   delete c;
