@@ -310,20 +310,34 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
+      // counter of the next tile's dependency, read early (relaxed) so its
+      // latency hides behind the current tile's loads
+      unsigned dep_seen = 0;
+      if (blockIdx.x < P.total_tiles) {
+        const Tile t0 = decode_tile<BM, 64>(P, blockIdx.x);
+        if (P.prob[t0.pi].done_dep != nullptr) dep_seen = ld_relaxed_gpu(P.prob[t0.pi].done_dep + t0.l);
+      }
       for (int t = blockIdx.x; ok && t < P.total_tiles; t += gridDim.x) {
         const Tile ti = decode_tile<BM, 64>(P, t);
         const GemmProblem& q = P.prob[ti.pi];
         if (q.done_dep != nullptr) {
           // the previous phase of this matrix must have landed before it is read
-          if (!wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status)) {
+          if (dep_seen >= q.dep_target) {
+            __threadfence();  // acquire: pairs with the writers' release increments
+          } else if (!wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status)) {
             ok = false;
             break;
           }
           fence_proxy_async_global();
         }
+        const int tn = t + gridDim.x;
+        if (tn < P.total_tiles) {
+          const Tile tin = decode_tile<BM, 64>(P, tn);
+          dep_seen = P.prob[tin.pi].done_dep != nullptr ? ld_relaxed_gpu(P.prob[tin.pi].done_dep + tin.l) : 0u;
+        }
         const int nk = q.k_tiles * q.nseg;
-        const uint32_t bbytes = q.b_mn_major ? static_cast<uint32_t>(ti.nw / 64) * MNMAJ_BOX_BYTES
-                                             : static_cast<uint32_t>((ti.nw + 127) / 128) * KMAJ_BOX_BYTES;
+        const bool narrow = !q.b_mn_major && ti.nw <= 128;
+        const uint32_t bbytes = q.b_mn_major ? 4u * MNMAJ_BOX_BYTES : (narrow ? KMAJ_BOX_BYTES : 2u * KMAJ_BOX_BYTES);
         for (int kk = 0; kk < nk; ++kk, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -339,13 +353,10 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
           const uint32_t sb = sa + A_BYTES;
           mbar_arrive_expect_tx(full_bar(s), A_BYTES + bbytes);
           tma_load_4d(sa, &q.tmA, full_bar(s), kb * BK, ti.m0, ti.l, pa);
-          if (q.b_mn_major) {
-            for (int c = 0; c < ti.nw / 64; ++c)
-              tma_load_4d(sb + c * MNMAJ_BOX_BYTES, &q.tmB, full_bar(s), ti.n0 + 64 * c, kb * BK, ti.l, pb);
-          } else {
-            for (int h = 0; h < (ti.nw + 127) / 128; ++h)
-              tma_load_4d(sb + h * KMAJ_BOX_BYTES, &q.tmB, full_bar(s), kb * BK, ti.n0 + 128 * h, ti.l, pb);
-          }
+          if (q.b_mn_major)
+            tma_load_5d(sb, &q.tmB, full_bar(s), 0, kb * BK, ti.n0 / 64, ti.l, pb);
+          else
+            tma_load_4d(sb, narrow ? &q.tmB2 : &q.tmB, full_bar(s), kb * BK, ti.n0, ti.l, pb);
         }
       }
       if (!ok) {
@@ -425,8 +436,7 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
         if (lane == 0) {
           bulk_wait_group_all();
           fence_proxy_async_global();
-          __threadfence();
-          atomicAdd(q.done_self + ti.l, 1u);
+          red_release_gpu_add(q.done_self + ti.l, 1u);
         }
         __syncwarp();
       }

@@ -64,9 +64,12 @@ constexpr int kEpilogueWarps = 8;
 constexpr int kMaxProblems = 30;
 
 struct alignas(64) GemmProblem {
-  CUtensorMap tmA;  // A operand [planes][L][M][K], K contiguous, box {64, 128}
-  CUtensorMap tmB;  // B operand: K-major [planes][L][N][K] box {64,128}, or
-                    //            MN-major [planes][L][K][N] box {64, 64}
+  CUtensorMap tmA;   // A operand [planes][L][M][K], K contiguous, box {64, 128}
+  CUtensorMap tmB;   // B operand.  Single-CTA kernel: K-major [planes][L][N][K] box
+                     // {64, 256}; MN-major as the 5-D chunked view {64 n, K, N/64,
+                     // L, planes} with box {64, 64, 4, 1, 1} (one load per stage).
+                     // CTA-pair kernel: 4-D box {64, 64} in either layout.
+  CUtensorMap tmB2;  // single-CTA kernel, K-major B: box {64, 128} for tiles <= 128 wide
   CUtensorMap tmOut;  // output [planes][L][M][N], box {32, 32}, 64-byte swizzle
   int M, N, K, L;
   int nseg;          // 1 (bf16) or 6 (three-plane split)

@@ -80,6 +80,25 @@ constexpr float kQuintic[3] = {3.4445f, -4.7750f, 2.0315f};
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int round8(int x) { return (x + 7) / 8 * 8; }
+int round64(int x) { return (x + 63) / 64 * 64; }
+
+// MN-major operand [planes][L][rows][pitch] as the 5-D view {64, rows, pitch/64, L, planes}:
+// one box {64, 64, 4, 1, 1} brings 64 rows of four 64-column chunks, chunk after chunk
+// (the layout the UMMA descriptor walks with an 8 KB leading-dimension offset).
+bool encode_chunked_map(CUtensorMap* map, const void* base, int rows, int L, int planes, int pitch) {
+  EncodeTiledFn enc = get_encoder();
+  if (!enc || pitch % 64) return false;
+  cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(pitch / 64),
+                        static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(planes)};
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(pitch) * 2;
+  cuuint64_t strides[4] = {row_bytes, 128, row_bytes * rows, row_bytes * rows * L};
+  cuuint32_t box[5] = {64, 64, 4, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 // One group as the kernels see it.
 struct GroupPlan {
@@ -261,7 +280,7 @@ GroupPlan plan_group(const muon_group& g) {
   p.transposed = g.rows > g.cols;
   p.m_rows = std::min(g.rows, g.cols);
   p.n_cols = std::max(g.rows, g.cols);
-  p.pitch_n = round8(p.n_cols);
+  p.pitch_n = round64(p.n_cols);  // the chunked MN-major view never leaves a row
   p.pitch_m = round8(p.m_rows);
   p.nblk = momentum_blocks_per_matrix(g.rows, g.cols);
   p.x_mat = static_cast<long long>(p.m_rows) * p.pitch_n;
@@ -293,14 +312,16 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
   q.planes = p.planes;
   const bool have_poly = cc != 0.f;
   const CUtensorMapSwizzle sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
-  // K-major B operand box height: 128 rows (single CTA) or 64 (each CTA of a pair)
-  const int kb_rows = c->gemm_kind == GEMM_PAIR ? 64 : 128;
+  // K-major B operand box height: 256 rows (single CTA; 128 for narrow tiles) or 64 (pair)
+  const bool pair = c->gemm_kind == GEMM_PAIR;
+  const int kb_rows = pair ? 64 : 256;
   switch (ph) {
     case PH_GRAM:
       // A = s2 * X X^T; with c = 0 the polynomial is linear and the Gram
       // epilogue writes B' = b A + a I directly.
       if (!encode_map(&q.tmA, X, n, m, p.batch, p.planes, p.pitch_n, 64, 128)) return false;
       if (!encode_map(&q.tmB, X, n, m, p.batch, p.planes, p.pitch_n, 64, kb_rows)) return false;
+      if (!pair && !encode_map(&q.tmB2, X, n, m, p.batch, p.planes, p.pitch_n, 64, 128)) return false;
       if (!encode_map(&q.tmOut, have_poly ? A : B, m, m, p.batch, p.planes, p.pitch_m, 32, 32, sw64))
         return false;
       q.M = m; q.N = m; q.K = n;
@@ -314,6 +335,7 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
       // B' = c A A + b A + a I
       if (!encode_map(&q.tmA, A, m, m, p.batch, p.planes, p.pitch_m, 64, 128)) return false;
       if (!encode_map(&q.tmB, A, m, m, p.batch, p.planes, p.pitch_m, 64, kb_rows)) return false;
+      if (!pair && !encode_map(&q.tmB2, A, m, m, p.batch, p.planes, p.pitch_m, 64, 128)) return false;
       if (!encode_map(&q.tmOut, B, m, m, p.batch, p.planes, p.pitch_m, 32, 32, sw64)) return false;
       q.M = m; q.N = m; q.K = m;
       q.b_mn_major = 0; q.sym = 1;
@@ -323,7 +345,11 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
     case PH_UPDATE: {
       // X' = s1 * B' X   (s1 = 1/(nu+eps) on the first iteration, X = U unnormalised)
       if (!encode_map(&q.tmA, B, m, m, p.batch, p.planes, p.pitch_m, 64, 128)) return false;
-      if (!encode_map(&q.tmB, X, n, m, p.batch, p.planes, p.pitch_n, 64, 64)) return false;
+      if (pair) {
+        if (!encode_map(&q.tmB, X, n, m, p.batch, p.planes, p.pitch_n, 64, 64)) return false;
+      } else if (!encode_chunked_map(&q.tmB, X, m, p.batch, p.planes, p.pitch_n)) {
+        return false;
+      }
       q.M = m; q.N = n; q.K = m;
       q.b_mn_major = 1; q.sym = 0;
       q.alpha = 1.f; q.beta = 0.f; q.diag = 0.f;
