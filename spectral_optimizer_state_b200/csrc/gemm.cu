@@ -73,8 +73,9 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& P, int t) {
   ti.pi = lo;
   const GemmProblem& q = P.prob[ti.pi];
   const int local = t - q.tile_base;
-  ti.l = local / q.tiles_per_matrix;
-  int r = local - ti.l * q.tiles_per_matrix;
+  const int lm = local / q.tiles_per_matrix;
+  int r = local - lm * q.tiles_per_matrix;
+  ti.l = q.reverse ? q.L - 1 - lm : lm;
   if (q.sym) {
     int mb = 0;
     for (;;) {

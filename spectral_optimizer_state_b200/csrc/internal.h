@@ -75,6 +75,7 @@ struct alignas(64) GemmProblem {
   int nseg;          // 1 (bf16) or 6 (three-plane split)
   int b_mn_major;    // 0: B stored N x K; 1: B stored K x N
   int sym;           // output symmetric: compute upper tiles only, mirror the rest
+  int reverse;       // walk the matrices last to first (L2 reuse of the previous phase)
   int tiles_per_matrix;
   int tile_base;     // first global tile index of this problem
   int k_tiles;       // ceil(K / 64)

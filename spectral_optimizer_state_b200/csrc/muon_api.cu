@@ -416,36 +416,66 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
   }
   const bool persistent = c->gemm_kind == GEMM_SINGLE;
   const int ng = static_cast<int>(plans.size());
-  const int phases_per_launch = persistent ? std::max(1, kMaxProblems / ng) : 1;
+  const int nph = static_cast<int>(seq_ph.size());
+  // Launch order of (group, phase) problems.  Persistent launches go group by
+  // group (one group's matrices stay in L2 across its phases; the next group
+  // starts while the last phases drain), and each update phase walks the
+  // matrices in reverse, so it starts on the X the Gram phase read last and
+  // the next Gram starts on the X' the update wrote last.  The CTA-pair kernel
+  // runs one launch per phase covering every group.
+  struct Item { int g, pi; };
+  std::vector<std::vector<Item>> launches;
+  if (persistent) {
+    std::vector<Item> cur;
+    for (int g = 0; g < ng; ++g) {
+      for (int pi = 0; pi < nph; ++pi) {
+        if (static_cast<int>(cur.size()) == kMaxProblems) {
+          launches.push_back(cur);
+          cur.clear();
+        }
+        cur.push_back({g, pi});
+      }
+    }
+    if (!cur.empty()) launches.push_back(cur);
+  } else {
+    for (int pi = 0; pi < nph; ++pi) {
+      std::vector<Item> cur;
+      for (int g = 0; g < ng; ++g) cur.push_back({g, pi});
+      launches.push_back(cur);
+    }
+  }
   GemmParams gp;
-  for (size_t p0 = 0; p0 < seq_ph.size(); p0 += phases_per_launch) {
-    const size_t p1 = std::min(seq_ph.size(), p0 + phases_per_launch);
+  for (const auto& items : launches) {
     std::memset(static_cast<void*>(&gp), 0, sizeof(gp));
     gp.status = c->d_status;
     int tiles = 0;
-    for (size_t pi = p0; pi < p1; ++pi) {
-      for (int g = 0; g < ng; ++g) {
-        GemmProblem& q = gp.prob[gp.nprob];
-        if (!fill_problem(c, plans[g], seq_ph[pi], seq_it[pi], q))
-          return cuda_fail(cudaErrorInvalidValue, "tensor map encoding");
-        q.tile_base = tiles;
-        tiles += q.tiles_per_matrix * q.L;
-        if (persistent) {
-          q.done_self = c->d_done + static_cast<size_t>(gp.nprob) * MUON_MAX_BATCH;
-          if (pi > p0) {
-            const GemmProblem& prev = gp.prob[gp.nprob - ng];  // same group, previous phase
-            q.done_dep = prev.done_self;
-            q.dep_target = static_cast<unsigned>(kEpilogueWarps * prev.tiles_per_matrix);
-          }
+    int last_of_group[MUON_MAX_GROUPS];
+    for (int g = 0; g < ng; ++g) last_of_group[g] = -1;
+    for (const Item& itm : items) {
+      GemmProblem& q = gp.prob[gp.nprob];
+      if (!fill_problem(c, plans[itm.g], seq_ph[itm.pi], seq_it[itm.pi], q))
+        return cuda_fail(cudaErrorInvalidValue, "tensor map encoding");
+      q.tile_base = tiles;
+      tiles += q.tiles_per_matrix * q.L;
+      q.reverse = persistent && seq_ph[itm.pi] == PH_UPDATE;
+      if (persistent) {
+        q.done_self = c->d_done + static_cast<size_t>(gp.nprob) * MUON_MAX_BATCH;
+        const int prev = last_of_group[itm.g];
+        if (prev >= 0) {  // the previous phase of this group is in the same launch
+          q.done_dep = gp.prob[prev].done_self;
+          q.dep_target = static_cast<unsigned>(kEpilogueWarps * gp.prob[prev].tiles_per_matrix);
         }
-        ++gp.nprob;
+        last_of_group[itm.g] = gp.nprob;
       }
+      ++gp.nprob;
     }
     gp.total_tiles = tiles;
     if (persistent)
       MUON_CUDA(cudaMemsetAsync(c->d_done, 0, sizeof(unsigned) * gp.nprob * MUON_MAX_BATCH, s), "clear counters");
     const int units = std::min(tiles, persistent ? c->sm_count : c->sm_count / 2);
-    const int kind = p1 - p0 > 1 ? MUON_KERNEL_NS_FUSED : MUON_KERNEL_GRAM + (seq_ph[p0] - PH_GRAM);
+    const int kind = items.size() > static_cast<size_t>(ng) || persistent
+                         ? MUON_KERNEL_NS_FUSED
+                         : MUON_KERNEL_GRAM + (seq_ph[items[0].pi] - PH_GRAM);
     const int slot = prof_begin(c, kind, s);
     MUON_CUDA(launch_gemm(gp, c->gemm_kind, units, s), "newton-schulz gemm");
     prof_end(c, slot, s);

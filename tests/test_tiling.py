@@ -83,6 +83,16 @@ def test_update_cover_exactly_once(m, n, kind):
     assert np.all(hits == 1)
 
 
+def test_reverse_walk_visits_every_matrix_once():
+    L, tpm = 5, 7
+    seen = []
+    for local in range(L * tpm):
+        lm, r = divmod(local, tpm)
+        seen.append((L - 1 - lm, r))
+    assert sorted(seen) == [(l, r) for l in range(L) for r in range(tpm)]
+    assert seen[0][0] == L - 1 and seen[-1][0] == 0
+
+
 @pytest.mark.parametrize("kind", sorted(KINDS))
 @pytest.mark.parametrize("m,n", SHAPES)
 def test_tma_coordinates_aligned(m, n, kind):
