@@ -418,11 +418,12 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
   const int ng = static_cast<int>(plans.size());
   const int nph = static_cast<int>(seq_ph.size());
   // Launch order of (group, phase) problems.  Persistent launches go group by
-  // group (one group's matrices stay in L2 across its phases; the next group
-  // starts while the last phases drain), and each update phase walks the
-  // matrices in reverse, so it starts on the X the Gram phase read last and
-  // the next Gram starts on the X' the update wrote last.  The CTA-pair kernel
-  // runs one launch per phase covering every group.
+  // group: one group's X stays (mostly) L2-resident across its phases, and the
+  // next group starts while the last phases of the previous one drain.  (Each
+  // phase keeps the matrix order of the previous one, so a matrix's next phase
+  // is dispatched a whole phase after its previous one; reversing the order for
+  // L2 reuse measured slower because of those dependency waits.)  The CTA-pair
+  // kernel runs one launch per phase covering every group.
   struct Item { int g, pi; };
   std::vector<std::vector<Item>> launches;
   if (persistent) {
@@ -457,7 +458,6 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
         return cuda_fail(cudaErrorInvalidValue, "tensor map encoding");
       q.tile_base = tiles;
       tiles += q.tiles_per_matrix * q.L;
-      q.reverse = persistent && seq_ph[itm.pi] == PH_UPDATE;
       if (persistent) {
         q.done_self = c->d_done + static_cast<size_t>(gp.nprob) * MUON_MAX_BATCH;
         const int prev = last_of_group[itm.g];
