@@ -192,6 +192,29 @@ typedef struct {
 muon_status muon_profile_enable(muon_ctx* ctx, int on);
 muon_status muon_profile_read(muon_ctx* ctx, muon_profile* out, int reset);
 
+/* Bytes of the library's static device scratch used by muon_momentum_norm_noalloc. */
+#define MUON_NOALLOC_SCRATCH_BYTES (256u * 1024u)
+
+/* Momentum, look-ahead and Frobenius norm for callers that cannot allocate
+ * device memory (a caller-owned memory pool, an allocator-free runtime, a
+ * hook running during CUDA graph capture).  No counterpart in the pages: it
+ * is the first pass of muon_step (M <- beta*M + G; U = G + beta*M, or U = M
+ * when nesterov == 0; nu_l = ||U_l||_F) without a context and without any
+ * allocation, and it does not materialise U.
+ * G: host array of `batch` device pointers, rows x cols of `dtype`, read only.
+ * M: host array of `batch` device pointers, rows x cols fp32, updated in place.
+ * nu: DEVICE array of `batch` floats, written.
+ * Scratch: a static device array of MUON_NOALLOC_SCRATCH_BYTES that every GPU
+ * loading the library holds until exit.  It must hold one float per 8192
+ * elements of each matrix: batch * ceil(rows*cols / 8192) <= 65280, else
+ * MUON_ERR_UNSUPPORTED_SHAPE.  The first call on a device looks the scratch
+ * address up (cudaGetSymbolAddress), so make it before any stream capture.
+ * Every call shares the scratch: calls that overlap on the GPU race on it.
+ * Asynchronous on `stream`; argument errors return before anything is queued. */
+muon_status muon_momentum_norm_noalloc(const void* const* G, float* const* M, float* nu, int batch,
+                                       int rows, int cols, int dtype, float beta, int nesterov,
+                                       void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -36,7 +36,7 @@ EXPORTS = (
     "muon_abi_version", "muon_status_string", "muon_last_cuda_error", "muon_create", "muon_destroy",
     "muon_set_coeffs", "muon_get_coeffs", "muon_step", "muon_step_groups", "muon_step_groups_host",
     "muon_ns_orthogonalize", "muon_get_status", "muon_get_norms", "muon_workspace_bytes",
-    "muon_profile_enable", "muon_profile_read",
+    "muon_profile_enable", "muon_profile_read", "muon_momentum_norm_noalloc",
 )
 KERNEL_KINDS = ("momentum", "gram", "poly", "update", "apply", "ns_fused")
 
@@ -97,6 +97,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "muon_workspace_bytes": (sz, [vp]),
         "muon_profile_enable": (i, [vp, i]),
         "muon_profile_read": (i, [vp, ctypes.POINTER(Profile), i]),
+        "muon_momentum_norm_noalloc": (i, [pvp, pvp, vp, i, i, i, i, f, i, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -287,6 +288,27 @@ class Muon:
         p = Profile()
         self._check(self.lib.muon_profile_read(self.handle, ctypes.byref(p), int(bool(reset))), "muon_profile_read")
         return {k: (p.launches[i], p.ms[i]) for i, k in enumerate(KERNEL_KINDS)}
+
+
+def momentum_norm_noalloc(G, M, nu, beta=0.95, nesterov=True, stream=None):
+    """M <- beta M + G in place and nu[l] = ||G + beta M||_F (or ||M||_F), without allocating.
+
+    For callers that cannot allocate device memory: no context is created and
+    the library's fixed static scratch is used (see include/muon.h).  `nu` is
+    a float32 CUDA tensor with one entry per matrix.
+    """
+    import torch
+    lib = load_library()
+    shape, dt = tuple(G[0].shape), G[0].dtype
+    _check_same(G, shape, dt, "cuda", "G")
+    _check_same(M, shape, torch.float32, "cuda", "M")
+    if len(G) != len(M) or nu.dtype != torch.float32 or not nu.is_cuda or nu.numel() < len(G):
+        raise ValueError("G, M and nu do not match")
+    st = lib.muon_momentum_norm_noalloc(_ptrs(G), _ptrs(M), ctypes.c_void_p(nu.data_ptr()), len(G), shape[0],
+                                        shape[1], _dtype_code(G[0]), float(beta), int(bool(nesterov)),
+                                        _stream_handle(stream))
+    if st != MUON_OK:
+        raise MuonError(st, "muon_momentum_norm_noalloc")
 
 
 def shape_scale(rows: int, cols: int, mode: int = SCALE_SQRT_RATIO) -> float:
