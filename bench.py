@@ -213,7 +213,7 @@ def blas_threads():
         return os.cpu_count()
 
 
-def oracle_sample(groups, budget_s=12.0, max_per_group=4):
+def oracle_sample(groups, budget_s=20.0, max_per_group=24):
     """Time the fp64 oracle on whole matrices of one step until ~budget_s; returns steps/s and a label."""
     import oracle
     from synthetic import group_inputs, group_weights
