@@ -281,6 +281,18 @@ def config_dict(args):
                 elements(WORKLOADS[args.workload]) * 8 / 1e9)}
 
 
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The slowest rank's value (one all-reduce on `device`); the value itself at N = 1."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -361,11 +373,7 @@ def main():
     prof = mu.profile_read(reset=True)
     st, flags = mu.status()
     assert st == 0, f"device status {st}"
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), world, device)
 
     # e2e through the host-gradient entry point (pinned host G in, norms + flags out)
     e2e_steps = max(3, min(args.e2e_steps, args.steps))
@@ -381,11 +389,7 @@ def main():
         mu.step_groups_host([(Ws[g], Ghost[g], Ms[g]) for g in range(len(groups))], stream=stream, **HP)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
 
     n_mats = sum(L for _, L, _, _ in groups)
     steps_per_s = world * args.steps / (ms / 1e3)
