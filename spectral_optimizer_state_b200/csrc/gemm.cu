@@ -534,14 +534,34 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_c
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
+      unsigned dep_seen = 0;  // next tile's dependency counter, read a tile ahead
+      if (pair < P.total_tiles) {
+        const Tile t0 = decode_tile<PBM, 128>(P, pair);
+        if (P.prob[t0.pi].done_dep != nullptr) dep_seen = ld_relaxed_gpu(P.prob[t0.pi].done_dep + t0.l);
+      }
       for (int t = pair; ok && t < P.total_tiles; t += npairs) {
         const Tile ti = decode_tile<PBM, 128>(P, t);
         const GemmProblem& q = P.prob[ti.pi];
+        if (q.done_dep != nullptr) {
+          // both CTAs load, so both acquire the previous phase of this matrix
+          if (dep_seen >= q.dep_target) {
+            __threadfence();
+          } else if (!wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status)) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_global();
+        }
+        const int tn = t + npairs;
+        if (tn < P.total_tiles) {
+          const Tile tin = decode_tile<PBM, 128>(P, tn);
+          dep_seen = P.prob[tin.pi].done_dep != nullptr ? ld_relaxed_gpu(P.prob[tin.pi].done_dep + tin.l) : 0u;
+        }
         const int nk = q.k_tiles * q.nseg;
         const int half_n = ti.nw >> 1;                 // this CTA's B columns (64 or 128)
-        const int nb = half_n / 64;                    // B boxes per stage
+        const bool narrow = half_n <= 64;
         const int n_mine = ti.n0 + static_cast<int>(rank) * half_n;
-        const uint32_t pair_bytes = 2u * (PA_BYTES + static_cast<uint32_t>(nb) * PBOX_BYTES);
+        const uint32_t pair_bytes = 2u * (PA_BYTES + (narrow ? PBOX_BYTES : 2u * PBOX_BYTES));
         for (int kk = 0; kk < nk; ++kk, ++it) {
           const int s = it % PSTAGES;
           const uint32_t ph = (it / PSTAGES) & 1u;
@@ -558,12 +578,11 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_c
           const uint32_t fb = map_shared_rank(full_bar(s), 0);  // the leader's full barrier
           if (leader) mbar_arrive_expect_tx(full_bar(s), pair_bytes);
           tma_load_4d_pair(sa, &q.tmA, fb, kb * BK, ti.m0 + 128 * static_cast<int>(rank), ti.l, pa);
-          for (int c = 0; c < nb; ++c) {
-            if (q.b_mn_major)
-              tma_load_4d_pair(sb + c * PBOX_BYTES, &q.tmB, fb, n_mine + 64 * c, kb * BK, ti.l, pb);
-            else
-              tma_load_4d_pair(sb + c * PBOX_BYTES, &q.tmB, fb, kb * BK, n_mine + 64 * c, ti.l, pb);
-          }
+          const CUtensorMap* mb = narrow ? &q.tmB2 : &q.tmB;
+          if (q.b_mn_major)
+            tma_load_5d_pair(sb, mb, fb, 0, kb * BK, n_mine / 64, ti.l, pb);
+          else
+            tma_load_4d_pair(sb, mb, fb, kb * BK, n_mine, ti.l, pb);
         }
       }
       if (!ok) {
@@ -638,8 +657,19 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_c
       if (!mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, P.status)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * ACC_COLS;
+      if (q.cin != nullptr && q.done_dep != nullptr) {
+        if (!wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status)) break;
+      }
       epilogue_warp_tile(q, ti, tbase, ti.m0 + 128 * static_cast<int>(rank) + 32 * quarter, lane,
                          32 * half, ti.m0 + PBM, my_stage, sb);
+      if (q.done_self != nullptr) {
+        if (lane == 0) {
+          bulk_wait_group_all();
+          fence_proxy_async_global();
+          red_release_gpu_add(q.done_self + ti.l, 1u);
+        }
+        __syncwarp();
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_shared_rank(tempty_bar(acc), 0));

@@ -85,14 +85,15 @@ int round64(int x) { return (x + 63) / 64 * 64; }
 // MN-major operand [planes][L][rows][pitch] as the 5-D view {64, rows, pitch/64, L, planes}:
 // one box {64, 64, 4, 1, 1} brings 64 rows of four 64-column chunks, chunk after chunk
 // (the layout the UMMA descriptor walks with an 8 KB leading-dimension offset).
-bool encode_chunked_map(CUtensorMap* map, const void* base, int rows, int L, int planes, int pitch) {
+bool encode_chunked_map(CUtensorMap* map, const void* base, int rows, int L, int planes, int pitch,
+                        int chunks = 4) {
   EncodeTiledFn enc = get_encoder();
   if (!enc || pitch % 64) return false;
   cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(pitch / 64),
                         static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(planes)};
   const cuuint64_t row_bytes = static_cast<cuuint64_t>(pitch) * 2;
   cuuint64_t strides[4] = {row_bytes, 128, row_bytes * rows, row_bytes * rows * L};
-  cuuint32_t box[5] = {64, 64, 4, 1, 1};
+  cuuint32_t box[5] = {64, 64, static_cast<cuuint32_t>(chunks), 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -133,6 +134,7 @@ struct muon_ctx {
   int* d_status = nullptr;
   unsigned* d_done = nullptr;  // [kMaxProblems][MUON_MAX_BATCH] phase-completion counters
   int gemm_kind = GEMM_SINGLE;  // MUON_GEMM=pair selects the CTA-pair kernel
+  bool per_phase = false;       // MUON_LAUNCH=phase: one launch per phase (same work; per-phase timing)
   int last_count = 0;
   cudaStream_t last_stream = nullptr;
   bool pending = false;
@@ -312,16 +314,17 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
   q.planes = p.planes;
   const bool have_poly = cc != 0.f;
   const CUtensorMapSwizzle sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
-  // K-major B operand box height: 256 rows (single CTA; 128 for narrow tiles) or 64 (pair)
+  // K-major B operand box height: the tile's N (256, or 128 for narrow tiles) on a
+  // single CTA; half of it (128, or 64) on each CTA of a pair.
   const bool pair = c->gemm_kind == GEMM_PAIR;
-  const int kb_rows = pair ? 64 : 256;
+  const int kb_rows = pair ? 128 : 256;
   switch (ph) {
     case PH_GRAM:
       // A = s2 * X X^T; with c = 0 the polynomial is linear and the Gram
       // epilogue writes B' = b A + a I directly.
       if (!encode_map(&q.tmA, X, n, m, p.batch, p.planes, p.pitch_n, 64, 128)) return false;
       if (!encode_map(&q.tmB, X, n, m, p.batch, p.planes, p.pitch_n, 64, kb_rows)) return false;
-      if (!pair && !encode_map(&q.tmB2, X, n, m, p.batch, p.planes, p.pitch_n, 64, 128)) return false;
+      if (!encode_map(&q.tmB2, X, n, m, p.batch, p.planes, p.pitch_n, 64, kb_rows / 2)) return false;
       if (!encode_map(&q.tmOut, have_poly ? A : B, m, m, p.batch, p.planes, p.pitch_m, 32, 32, sw64))
         return false;
       q.M = m; q.N = m; q.K = n;
@@ -335,7 +338,7 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
       // B' = c A A + b A + a I
       if (!encode_map(&q.tmA, A, m, m, p.batch, p.planes, p.pitch_m, 64, 128)) return false;
       if (!encode_map(&q.tmB, A, m, m, p.batch, p.planes, p.pitch_m, 64, kb_rows)) return false;
-      if (!pair && !encode_map(&q.tmB2, A, m, m, p.batch, p.planes, p.pitch_m, 64, 128)) return false;
+      if (!encode_map(&q.tmB2, A, m, m, p.batch, p.planes, p.pitch_m, 64, kb_rows / 2)) return false;
       if (!encode_map(&q.tmOut, B, m, m, p.batch, p.planes, p.pitch_m, 32, 32, sw64)) return false;
       q.M = m; q.N = m; q.K = m;
       q.b_mn_major = 0; q.sym = 1;
@@ -345,11 +348,10 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
     case PH_UPDATE: {
       // X' = s1 * B' X   (s1 = 1/(nu+eps) on the first iteration, X = U unnormalised)
       if (!encode_map(&q.tmA, B, m, m, p.batch, p.planes, p.pitch_m, 64, 128)) return false;
-      if (pair) {
-        if (!encode_map(&q.tmB, X, n, m, p.batch, p.planes, p.pitch_n, 64, 64)) return false;
-      } else if (!encode_chunked_map(&q.tmB, X, m, p.batch, p.planes, p.pitch_n)) {
-        return false;
-      }
+      // chunked MN-major view: 4 chunks per load (single CTA) or 2 (each CTA of a pair);
+      // the narrow variant (pair, half-width tiles) loads one chunk
+      if (!encode_chunked_map(&q.tmB, X, m, p.batch, p.planes, p.pitch_n, pair ? 2 : 4)) return false;
+      if (pair && !encode_chunked_map(&q.tmB2, X, m, p.batch, p.planes, p.pitch_n, 1)) return false;
       q.M = m; q.N = n; q.K = m;
       q.b_mn_major = 1; q.sym = 0;
       q.alpha = 1.f; q.beta = 0.f; q.diag = 0.f;
@@ -414,7 +416,9 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
       seq_it.push_back(it);
     }
   }
-  const bool persistent = c->gemm_kind == GEMM_SINGLE;
+  const bool persistent = !c->per_phase;
+  const bool pair = c->gemm_kind == GEMM_PAIR;
+  const int signals_per_tile = kEpilogueWarps * (pair ? 2 : 1);
   const int ng = static_cast<int>(plans.size());
   const int nph = static_cast<int>(seq_ph.size());
   // Launch order of (group, phase) problems.  Persistent launches go group by
@@ -463,7 +467,7 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
         const int prev = last_of_group[itm.g];
         if (prev >= 0) {  // the previous phase of this group is in the same launch
           q.done_dep = gp.prob[prev].done_self;
-          q.dep_target = static_cast<unsigned>(kEpilogueWarps * gp.prob[prev].tiles_per_matrix);
+          q.dep_target = static_cast<unsigned>(signals_per_tile * gp.prob[prev].tiles_per_matrix);
         }
         last_of_group[itm.g] = gp.nprob;
       }
@@ -472,7 +476,7 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
     gp.total_tiles = tiles;
     if (persistent)
       MUON_CUDA(cudaMemsetAsync(c->d_done, 0, sizeof(unsigned) * gp.nprob * MUON_MAX_BATCH, s), "clear counters");
-    const int units = std::min(tiles, persistent ? c->sm_count : c->sm_count / 2);
+    const int units = std::min(tiles, pair ? c->sm_count / 2 : c->sm_count);
     const int kind = items.size() > static_cast<size_t>(ng) || persistent
                          ? MUON_KERNEL_NS_FUSED
                          : MUON_KERNEL_GRAM + (seq_ph[items[0].pi] - PH_GRAM);
@@ -567,6 +571,9 @@ muon_status muon_create(muon_ctx** out, int device) {
   c->k = 5;
   if (const char* g = std::getenv("MUON_GEMM")) {
     if (std::strcmp(g, "pair") == 0) c->gemm_kind = GEMM_PAIR;
+  }
+  if (const char* l = std::getenv("MUON_LAUNCH")) {
+    if (std::strcmp(l, "phase") == 0) c->per_phase = true;
   }
   if (cudaMalloc(&c->d_status, sizeof(int)) != cudaSuccess) {
     cudaGetLastError();
