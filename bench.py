@@ -391,6 +391,35 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
 
+    # AdamW over the parameters Muon does not take (the rest of Mamba-2 130M)
+    adamw = None
+    if args.workload == "mamba2-130m":
+        from spectral_optimizer_state_b200 import adamw_step
+        from synthetic import mamba2_130m_other_params
+        others = mamba2_130m_other_params()
+        aw = [torch.randn(int(np.prod(sh)), device=device).to(torch.bfloat16) * 0.02 for _, sh in others]
+        ag = [torch.randn(w.numel(), device=device).to(torch.bfloat16) for w in aw]
+        am = [torch.zeros(w.numel(), device=device) for w in aw]
+        av = [torch.zeros(w.numel(), device=device) for w in aw]
+        for i in range(3):
+            adamw_step(aw, ag, am, av, i + 1)
+        torch.cuda.synchronize()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        reps = 20
+        a0.record(stream)
+        for i in range(reps):
+            adamw_step(aw, ag, am, av, i + 4)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        a_ms = a0.elapsed_time(a1) / reps
+        numel = sum(w.numel() for w in aw)
+        gbs = 22 * numel / (a_ms / 1e3) / 1e9
+        adamw = {"bound": "hbm", "params": numel, "ms_per_step": a_ms, "achieved_gbs": gbs,
+                 "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"], "bytes_per_element": 22,
+                 "tensors": len(aw), "note": "AdamW over the non-Muon parameters of Mamba-2 130M, bf16"}
+        del aw, ag, am, av
+
     n_mats = sum(L for _, L, _, _ in groups)
     steps_per_s = world * args.steps / (ms / 1e3)
     gemm_kinds = ("gram", "poly", "update", "ns_fused")
@@ -429,6 +458,7 @@ def main():
                          "frac": (app_gbs / peaks["hbm_gbs"]) if app_gbs else None,
                          "bytes_per_element": 6, "launches": app_launches},
         "kernel_ms_per_step": {k: v[1] / args.steps for k, v in prof.items()},
+        "adamw_kernel": adamw,
         "cpu_baseline": cpu,
         "clocks": clk,
         "e2e": {"value": world * e2e_steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,

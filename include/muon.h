@@ -192,6 +192,24 @@ typedef struct {
 muon_status muon_profile_enable(muon_ctx* ctx, int on);
 muon_status muon_profile_read(muon_ctx* ctx, muon_profile* out, int reset);
 
+/* AdamW for the parameters Muon does not take (Muon Meets Mamba: Spectral
+ * Optimization for State Space Models, abstract: every weight group not
+ * trained with Muon is trained with AdamW).  For each of `count` tensors t:
+ *   m <- b1 m + (1 - b1) g ;  v <- b2 v + (1 - b2) g^2
+ *   W <- W (1 - lr wd) - lr (m / (1 - b1^step)) / (sqrt(v / (1 - b2^step)) + eps)
+ * W: host array of device pointers, numel[t] elements of `dtype`, updated in place.
+ * G: same, read only.  m, v: fp32, numel[t] elements, updated in place (start at 0).
+ * numel: HOST array of element counts.  Tensors may have any shape (flattened).
+ * No context and no allocation; asynchronous on `stream`. */
+typedef struct {
+  float lr, beta1, beta2, eps, weight_decay;
+  int step; /* 1-based step count used for bias correction */
+} muon_adamw_hparams;
+
+muon_status muon_adamw_step(void* const* W, const void* const* G, float* const* m, float* const* v,
+                            const long long* numel, int count, int dtype,
+                            const muon_adamw_hparams* hp, void* stream);
+
 /* Bytes of the library's static device scratch used by muon_momentum_norm_noalloc. */
 #define MUON_NOALLOC_SCRATCH_BYTES (256u * 1024u)
 

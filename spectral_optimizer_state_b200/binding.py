@@ -36,7 +36,7 @@ EXPORTS = (
     "muon_abi_version", "muon_status_string", "muon_last_cuda_error", "muon_create", "muon_destroy",
     "muon_set_coeffs", "muon_get_coeffs", "muon_step", "muon_step_groups", "muon_step_groups_host",
     "muon_ns_orthogonalize", "muon_get_status", "muon_get_norms", "muon_workspace_bytes",
-    "muon_profile_enable", "muon_profile_read", "muon_momentum_norm_noalloc",
+    "muon_profile_enable", "muon_profile_read", "muon_momentum_norm_noalloc", "muon_adamw_step",
 )
 KERNEL_KINDS = ("momentum", "gram", "poly", "update", "apply", "ns_fused")
 
@@ -57,6 +57,11 @@ class Hparams(ctypes.Structure):
 
 class Profile(ctypes.Structure):
     _fields_ = [("launches", ctypes.c_int * 6), ("ms", ctypes.c_double * 6)]
+
+
+class AdamWHparams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("step", ctypes.c_int)]
 
 
 class Group(ctypes.Structure):
@@ -98,6 +103,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "muon_profile_enable": (i, [vp, i]),
         "muon_profile_read": (i, [vp, ctypes.POINTER(Profile), i]),
         "muon_momentum_norm_noalloc": (i, [pvp, pvp, vp, i, i, i, i, f, i, vp]),
+        "muon_adamw_step": (i, [pvp, pvp, pvp, pvp, ctypes.POINTER(ctypes.c_longlong), i, i,
+                                ctypes.POINTER(AdamWHparams), vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -309,6 +316,33 @@ def momentum_norm_noalloc(G, M, nu, beta=0.95, nesterov=True, stream=None):
                                         _stream_handle(stream))
     if st != MUON_OK:
         raise MuonError(st, "muon_momentum_norm_noalloc")
+
+
+def adamw_step(W, G, m, v, step, lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, stream=None):
+    """AdamW on tensors of any shapes (one dtype, bf16 or fp32; fp32 moments), one launch per 256 tensors."""
+    import torch
+    lib = load_library()
+    if not (len(W) == len(G) == len(m) == len(v)) or len(W) == 0:
+        raise ValueError("W, G, m and v must be non-empty lists of equal length")
+    dt = W[0].dtype
+    for w, g, a, b in zip(W, G, m, v):
+        if w.dtype != dt or g.dtype != dt or a.dtype != torch.float32 or b.dtype != torch.float32:
+            raise ValueError("W and G share one dtype; m and v are float32")
+        if not (w.is_cuda and g.is_cuda and a.is_cuda and b.is_cuda):
+            raise ValueError("all tensors must be on the GPU")
+        if not (w.is_contiguous() and g.is_contiguous() and a.is_contiguous() and b.is_contiguous()):
+            raise ValueError("tensors must be contiguous")
+        if not (w.numel() == g.numel() == a.numel() == b.numel()):
+            raise ValueError("W, G, m and v must match in size")
+    hp = AdamWHparams(float(lr), float(beta1), float(beta2), float(eps), float(weight_decay), int(step))
+    for c0 in range(0, len(W), MAX_BATCH):
+        sl = slice(c0, c0 + MAX_BATCH)
+        ws, gs, ms, vs = W[sl], G[sl], m[sl], v[sl]
+        numel = (ctypes.c_longlong * len(ws))(*[t.numel() for t in ws])
+        st = lib.muon_adamw_step(_ptrs(ws), _ptrs(gs), _ptrs(ms), _ptrs(vs), numel, len(ws), _dtype_code(ws[0]),
+                                 ctypes.byref(hp), _stream_handle(stream))
+        if st != MUON_OK:
+            raise MuonError(st, "muon_adamw_step")
 
 
 def shape_scale(rows: int, cols: int, mode: int = SCALE_SQRT_RATIO) -> float:

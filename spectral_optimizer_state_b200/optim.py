@@ -1,0 +1,78 @@
+"""Muon for the selected projection weights, AdamW for everything else.
+
+The protocol of "Muon Meets Mamba: Spectral Optimization for State Space
+Models" (abstract) trains Mamba-2 130M with Muon on the output projections
+only, the input projections only, or both, and AdamW for the rest; the
+practitioner notes on the same paper (section 3.3) split the parameters by
+name.  This class is the host-side bookkeeping of that split: parameters are
+grouped by shape and dtype and handed to libmuon's muon_step_groups (Muon)
+and muon_adamw_step (AdamW); every update runs in the library's kernels.
+"""
+from __future__ import annotations
+
+from collections import OrderedDict
+
+from .binding import MAX_BATCH, MAX_GROUPS, Muon, adamw_step
+
+
+def takes_muon(name: str, shape, mode: str = "both") -> bool:
+    """2-D weights whose name marks them as the selected projection group(s)."""
+    if len(shape) != 2:
+        return False
+    if mode == "both":
+        return "in_proj" in name or "out_proj" in name
+    if mode in ("in_proj", "out_proj"):
+        return mode in name
+    if mode == "none":
+        return False
+    raise ValueError(f"unknown Muon selection {mode!r}")
+
+
+class MuonAdamW:
+    """named_params: iterable of (name, tensor) on one CUDA device."""
+
+    def __init__(self, named_params, mode="both", device=0, coeffs=None,
+                 muon_hp=None, adamw_hp=None):
+        import torch
+        self.mode = mode
+        self.muon_hp = dict(lr=0.02, beta=0.95, weight_decay=0.1, eps=1e-7, nesterov=True)
+        self.muon_hp.update(muon_hp or {})
+        self.adamw_hp = dict(lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1)
+        self.adamw_hp.update(adamw_hp or {})
+        self.ctx = Muon(device, coeffs)
+        self.muon = OrderedDict()   # (shape, dtype) -> [(name, W, M)]
+        self.adam = OrderedDict()   # dtype -> [(name, W, m, v)]
+        for name, p in named_params:
+            if takes_muon(name, tuple(p.shape), mode):
+                key = (tuple(p.shape), p.dtype)
+                self.muon.setdefault(key, []).append((name, p, torch.zeros(p.shape, dtype=torch.float32, device=p.device)))
+            else:
+                z = lambda: torch.zeros(p.numel(), dtype=torch.float32, device=p.device)  # noqa: E731
+                self.adam.setdefault(p.dtype, []).append((name, p, z(), z()))
+        self.t = 0
+
+    def muon_names(self):
+        return [n for entries in self.muon.values() for (n, _, _) in entries]
+
+    def adamw_names(self):
+        return [n for entries in self.adam.values() for (n, _, _, _) in entries]
+
+    def step(self, grads, stream=None):
+        """grads: mapping name -> gradient tensor (same shape and dtype as the parameter)."""
+        self.t += 1
+        groups = []
+        for entries in self.muon.values():
+            for c0 in range(0, len(entries), MAX_BATCH):
+                chunk = entries[c0:c0 + MAX_BATCH]
+                groups.append(([w for _, w, _ in chunk], [grads[n].contiguous() for n, _, _ in chunk],
+                               [mbuf for _, _, mbuf in chunk]))
+        for g0 in range(0, len(groups), MAX_GROUPS):
+            self.ctx.step_groups(groups[g0:g0 + MAX_GROUPS], stream=stream, **self.muon_hp)
+        for entries in self.adam.values():
+            W = [w.view(-1) for _, w, _, _ in entries]
+            G = [grads[n].contiguous().view(-1) for n, _, _, _ in entries]
+            adamw_step(W, G, [m for _, _, m, _ in entries], [v for _, _, _, v in entries], self.t,
+                       stream=stream, **self.adamw_hp)
+
+    def close(self):
+        self.ctx.close()

@@ -22,6 +22,21 @@ import numpy as np
 MAMBA2_130M_OUT_PROJ = (768, 1536)
 MAMBA2_130M_IN_PROJ = (3352, 768)
 MAMBA2_130M_LAYERS = 24
+# The other parameters of Mamba-2 130M (vocab 50280, conv width 4, 24 heads):
+# the embedding (tied with the output head), per layer the depthwise conv
+# weight and bias over d_inner + 2 d_state channels, A_log, D, dt_bias, the
+# gated norm over d_inner and the block norm; the final norm.
+def mamba2_130m_other_params():
+    shapes = [("embeddings.weight", (50280, 768))]
+    for layer in range(MAMBA2_130M_LAYERS):
+        pre = f"layers.{layer}."
+        shapes += [(pre + "mixer.conv1d.weight", (1792, 1, 4)), (pre + "mixer.conv1d.bias", (1792,)),
+                   (pre + "mixer.A_log", (24,)), (pre + "mixer.D", (24,)), (pre + "mixer.dt_bias", (24,)),
+                   (pre + "mixer.norm.weight", (1536,)), (pre + "norm.weight", (768,))]
+    shapes.append(("norm_f.weight", (768,)))
+    return shapes
+
+
 # Scaled Mamba-2-style model: d_model 2048, d_inner 4096, 48 layers.
 SCALED_2K_IN_PROJ = (8192 + 512 + 64, 2048)
 SCALED_2K_OUT_PROJ = (2048, 4096)
