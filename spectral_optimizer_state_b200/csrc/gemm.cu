@@ -234,35 +234,6 @@ __device__ __forceinline__ void store_chunk(const CUtensorMap* map, uint32_t sta
   sb ^= 1;
 }
 
-// Direct stores from registers: this lane's 32 values as four 16-byte stores
-// into its row, and (mirror) as 32 two-byte stores down column `row` (lanes
-// hold consecutive rows, so each of those is one 64-byte coalesced store).
-__device__ __forceinline__ void store_direct(const GemmProblem& q, int l, int p, int row, int j0, int nv,
-                                             const uint16_t (&b)[32], bool mirror) {
-  if (row >= q.M) return;
-  uint16_t* base = q.out + p * q.out_plane + l * q.out_mat;
-  if (nv == 32) {
-    uint4* dst = reinterpret_cast<uint4*>(base + static_cast<long long>(row) * q.out_pitch + j0);
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const int o = 8 * h;
-      dst[h] = make_uint4(static_cast<uint32_t>(b[o]) | (static_cast<uint32_t>(b[o + 1]) << 16),
-                          static_cast<uint32_t>(b[o + 2]) | (static_cast<uint32_t>(b[o + 3]) << 16),
-                          static_cast<uint32_t>(b[o + 4]) | (static_cast<uint32_t>(b[o + 5]) << 16),
-                          static_cast<uint32_t>(b[o + 6]) | (static_cast<uint32_t>(b[o + 7]) << 16));
-    }
-  } else {
-#pragma unroll
-    for (int t = 0; t < 32; ++t)
-      if (t < nv) base[static_cast<long long>(row) * q.out_pitch + j0 + t] = b[t];
-  }
-  if (mirror) {
-#pragma unroll
-    for (int t = 0; t < 32; ++t)
-      if (t < nv) base[static_cast<long long>(j0 + t) * q.out_pitch + row] = b[t];
-  }
-}
-
 // One warp's share of a finished accumulator tile: TMEM rows row0..row0+31
 // (this warp's lane quarter), 32-column chunks c_first, c_first + 64, ...
 // v = alpha s_l acc + beta cin + diag on the diagonal, split into planes and
@@ -318,12 +289,8 @@ __device__ __forceinline__ void epilogue_warp_tile(const GemmProblem& q, const T
         b[i] = float_to_bf16_bits(v[i]);
         v[i] -= bf16_bits_to_float(b[i]);  // residual for the next plane
       }
-      if (q.direct_store) {
-        store_direct(q, ti.l, p, row, j0, nv, b, mirror);
-      } else {
-        store_chunk<false>(&q.tmOut, my_stage, sb, lane, b, j0, row0, ti.l, p);
-        if (mirror) store_chunk<true>(&q.tmOut, my_stage, sb, lane, b, row0, j0, ti.l, p);
-      }
+      store_chunk<false>(&q.tmOut, my_stage, sb, lane, b, j0, row0, ti.l, p);
+      if (mirror) store_chunk<true>(&q.tmOut, my_stage, sb, lane, b, row0, j0, ti.l, p);
     }
   }
 }

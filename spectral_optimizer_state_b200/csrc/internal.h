@@ -82,10 +82,6 @@ struct alignas(64) GemmProblem {
   int planes;        // planes of out / cin (1 or 3)
   float alpha, beta, diag;
   const float* mat_scale;  // per-matrix factor s_l, or null for 1
-  uint16_t* out;           // output [planes][L][M][out_pitch] for direct stores
-  long long out_plane, out_mat;
-  int out_pitch;
-  int direct_store;        // 1: st.global from registers; 0: TMA stores through shared memory
   const uint16_t* cin;     // [planes][L][M][cin_pitch], null when beta == 0
   long long cin_plane, cin_mat;
   int cin_pitch;

@@ -135,7 +135,6 @@ struct muon_ctx {
   unsigned* d_done = nullptr;  // [kMaxProblems][MUON_MAX_BATCH] phase-completion counters
   int gemm_kind = GEMM_SINGLE;  // MUON_GEMM=pair selects the CTA-pair kernel
   bool per_phase = false;       // MUON_LAUNCH=phase: one launch per phase (same work; per-phase timing)
-  bool direct_store = false;    // MUON_EPI=direct: epilogue stores from registers instead of TMA
   int last_count = 0;
   cudaStream_t last_stream = nullptr;
   bool pending = false;
@@ -334,7 +333,6 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
       q.beta = 0.f;
       q.diag = have_poly ? 0.f : a;
       q.mat_scale = it == 0 ? c->d_s2 + p.mat_off : nullptr;
-      q.out = have_poly ? A : B; q.out_plane = p.a_plane; q.out_mat = p.a_mat; q.out_pitch = p.pitch_m;
       break;
     case PH_POLY:
       // B' = c A A + b A + a I
@@ -346,7 +344,6 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
       q.b_mn_major = 0; q.sym = 1;
       q.alpha = cc; q.beta = b; q.diag = a;
       q.cin = A; q.cin_plane = p.a_plane; q.cin_mat = p.a_mat; q.cin_pitch = p.pitch_m;
-      q.out = B; q.out_plane = p.a_plane; q.out_mat = p.a_mat; q.out_pitch = p.pitch_m;
       break;
     case PH_UPDATE: {
       // X' = s1 * B' X   (s1 = 1/(nu+eps) on the first iteration, X = U unnormalised)
@@ -360,11 +357,9 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
       q.alpha = 1.f; q.beta = 0.f; q.diag = 0.f;
       q.mat_scale = it == 0 ? c->d_s1 + p.mat_off : nullptr;
       if (!encode_map(&q.tmOut, Xn, n, m, p.batch, p.planes, p.pitch_n, 32, 32, sw64)) return false;
-      q.out = Xn; q.out_plane = p.x_plane; q.out_mat = p.x_mat; q.out_pitch = p.pitch_n;
       break;
     }
   }
-  q.direct_store = c->direct_store ? 1 : 0;
   q.tiles_per_matrix = gemm_tiles_per_matrix(c->gemm_kind, q.M, q.N, q.sym);
   q.k_tiles = (q.K + 63) / 64;
   return true;
@@ -576,9 +571,6 @@ muon_status muon_create(muon_ctx** out, int device) {
   c->k = 5;
   if (const char* g = std::getenv("MUON_GEMM")) {
     if (std::strcmp(g, "pair") == 0) c->gemm_kind = GEMM_PAIR;
-  }
-  if (const char* e = std::getenv("MUON_EPI")) {
-    if (std::strcmp(e, "direct") == 0) c->direct_store = true;
   }
   if (const char* l = std::getenv("MUON_LAUNCH")) {
     if (std::strcmp(l, "phase") == 0) c->per_phase = true;
