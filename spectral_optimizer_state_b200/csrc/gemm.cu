@@ -160,25 +160,6 @@ __device__ __forceinline__ void add_cin(const GemmProblem& q, int l, int row, in
   for (int t = 0; t < 32; ++t) v[t] = fmaf(q.beta, c[t], v[t]);
 }
 
-// The bf16 (single-plane) cin chunk of one row: 32 values in four 16-byte loads
-// from L2 (cin is rewritten within a launch, so no L1-cached loads).  Issued a
-// chunk ahead of its use so the L2 latency overlaps the TMEM load and math.
-__device__ __forceinline__ void load_cin_chunk(const GemmProblem& q, int l, int row, int j0, uint4 (&c)[4]) {
-  const uint16_t* src = q.cin + l * q.cin_mat + static_cast<long long>(row) * q.cin_pitch + j0;
-  if (j0 + 32 <= q.N) {
-#pragma unroll
-    for (int h = 0; h < 4; ++h) c[h] = __ldcg(reinterpret_cast<const uint4*>(src) + h);
-  } else {
-    uint16_t e[32];
-#pragma unroll
-    for (int t = 0; t < 32; ++t) e[t] = j0 + t < q.N ? __ldcg(src + t) : static_cast<uint16_t>(0);
-#pragma unroll
-    for (int h = 0; h < 4; ++h)
-      c[h] = make_uint4(e[8 * h] | (e[8 * h + 1] << 16), e[8 * h + 2] | (e[8 * h + 3] << 16),
-                        e[8 * h + 4] | (e[8 * h + 5] << 16), e[8 * h + 6] | (e[8 * h + 7] << 16));
-  }
-}
-
 // Staging tile for one TMA store: 32 rows x 32 bf16 (64-byte rows) in the
 // 64-byte swizzle the tensor map declares: 16-byte chunk c of row r sits at
 // chunk c ^ ((r >> 1) & 3), which also keeps the row-per-lane writes free of
@@ -240,22 +221,14 @@ __device__ __forceinline__ void store_chunk(const CUtensorMap* map, uint32_t sta
 // stored through TMA; columns from `mirror_from` on are also stored transposed.
 __device__ __forceinline__ void epilogue_warp_tile(const GemmProblem& q, const Tile& ti, uint32_t tbase,
                                                    int row0, int lane, int c_first, int mirror_from,
-                                                   uint32_t my_stage, int& sb, uint4 (&cpre)[4], bool have_pre) {
+                                                   uint32_t my_stage, int& sb) {
   if (row0 >= q.M) return;
   const int row = row0 + lane;
   const float scale = q.alpha * (q.mat_scale != nullptr ? q.mat_scale[ti.l] : 1.0f);
-  // single-plane cin comes through the prefetched chunk; three-plane cin is read in place
-  const bool pre = have_pre && q.cin != nullptr && q.planes == 1;
   for (int c = c_first; c < ti.nw; c += 64) {
     const int j0 = ti.n0 + c;
     if (j0 >= q.N) break;
     const int nv = min(32, q.N - j0);
-    uint4 cur[4];
-    if (pre) {
-#pragma unroll
-      for (int h = 0; h < 4; ++h) cur[h] = cpre[h];
-      if (c + 64 < ti.nw && j0 + 64 < q.N && row < q.M) load_cin_chunk(q, ti.l, row, j0 + 64, cpre);
-    }
     uint32_t r[32];
     __syncwarp();  // tcgen05.ld is warp-collective
     tmem_load_32cols(tbase + c, r);
@@ -263,19 +236,7 @@ __device__ __forceinline__ void epilogue_warp_tile(const GemmProblem& q, const T
     float v[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = scale * __uint_as_float(r[i]);
-    if (q.cin != nullptr && row < q.M) {
-      if (pre) {
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          float f[8];
-          unpack_bf16x8(cur[h], f);
-#pragma unroll
-          for (int t = 0; t < 8; ++t) v[8 * h + t] = fmaf(q.beta, f[t], v[8 * h + t]);
-        }
-      } else {
-        add_cin(q, ti.l, row, j0, nv, v);
-      }
-    }
+    if (q.cin != nullptr && row < q.M) add_cin(q, ti.l, row, j0, nv, v);
     if (q.diag != 0.f) {
 #pragma unroll
       for (int i = 0; i < 32; ++i)
@@ -463,26 +424,14 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
       const GemmProblem& q = P.prob[ti.pi];
       const int acc = local & 1;
       const uint32_t aph = (local >> 1) & 1;
-      const int row0 = ti.m0 + 32 * quarter;
-      uint4 cpre[4];
-      bool have_pre = false;
-      if (q.cin != nullptr && q.planes == 1 && row0 < q.M) {
-        // cin was written earlier in this launch: acquire it for this warp's loads,
-        // then fetch the first chunk while the tile's MMAs still run
-        if (q.done_dep != nullptr && !wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status))
-          break;
-        const int j0 = ti.n0 + 32 * half;
-        if (32 * half < ti.nw && j0 < q.N && row0 + lane < q.M) {
-          load_cin_chunk(q, ti.l, row0 + lane, j0, cpre);
-        }
-        have_pre = true;
-      } else if (q.cin != nullptr && q.done_dep != nullptr) {
-        if (!wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status)) break;
-      }
       if (!mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, P.status)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * ACC_COLS;
-      epilogue_warp_tile(q, ti, tbase, row0, lane, 32 * half, ti.m0 + BM, my_stage, sb, cpre, have_pre);
+      if (q.cin != nullptr && q.done_dep != nullptr) {
+        // cin was written earlier in this launch: acquire it for this warp's plain loads
+        if (!wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status)) break;
+      }
+      epilogue_warp_tile(q, ti, tbase, ti.m0 + 32 * quarter, lane, 32 * half, ti.m0 + BM, my_stage, sb);
       if (q.done_self != nullptr) {
         // this warp's stores of the tile are complete and visible: count it done
         if (lane == 0) {
@@ -705,21 +654,14 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_c
       const GemmProblem& q = P.prob[ti.pi];
       const int acc = local & 1;
       const uint32_t aph = (local >> 1) & 1;
-      const int row0 = ti.m0 + 128 * static_cast<int>(rank) + 32 * quarter;
-      uint4 cpre[4];
-      bool have_pre = false;
-      if (q.cin != nullptr && q.done_dep != nullptr) {
-        if (!wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status)) break;
-      }
-      if (q.cin != nullptr && q.planes == 1 && row0 < q.M) {
-        const int j0 = ti.n0 + 32 * half;
-        if (32 * half < ti.nw && j0 < q.N && row0 + lane < q.M) load_cin_chunk(q, ti.l, row0 + lane, j0, cpre);
-        have_pre = true;
-      }
       if (!mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, P.status)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * ACC_COLS;
-      epilogue_warp_tile(q, ti, tbase, row0, lane, 32 * half, ti.m0 + PBM, my_stage, sb, cpre, have_pre);
+      if (q.cin != nullptr && q.done_dep != nullptr) {
+        if (!wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status)) break;
+      }
+      epilogue_warp_tile(q, ti, tbase, ti.m0 + 128 * static_cast<int>(rank) + 32 * quarter, lane,
+                         32 * half, ti.m0 + PBM, my_stage, sb);
       if (q.done_self != nullptr) {
         if (lane == 0) {
           bulk_wait_group_all();
