@@ -356,3 +356,44 @@ def test_single_cta_and_pair_kernels_agree():
     for a_list, b_list in zip(outs["single"], outs["pair"]):
         for a, b in zip(a_list, b_list):
             assert rel_f(a, b) <= 5e-3
+
+
+def test_scaled_2k_model_full_size_sampled():
+    """Scaled Mamba-2-style model (d_model 2048): 48 x 8768 x 2048 + 48 x 2048 x 4096 bf16 in one
+    call, the same launches bench.py times; one matrix per group checked against the oracle.
+    Only the checked matrices come from the host generator; the rest are seeded on the device."""
+    import torch
+    from synthetic import SCALED_2K_IN_PROJ, SCALED_2K_OUT_PROJ
+    shapes = [SCALED_2K_OUT_PROJ, SCALED_2K_IN_PROJ]
+    check = {0: 7, 1: 40}
+    gen = torch.Generator(device="cuda").manual_seed(2024)
+    W, G, M, host = [], [], [], {}
+    for g, shape in enumerate(shapes):
+        Wg, Gg = [], []
+        for l in range(48):
+            if l == check[g]:
+                gh = round_bf16(draw("spike", rng_for(4000 + g, l), *shape).astype(np.float32))
+                wh = round_bf16((rng_for(4100 + g, l).standard_normal(shape) * 0.02).astype(np.float32))
+                host[g] = (wh, gh)
+                Wg.append(to_device(wh, "bf16"))
+                Gg.append(to_device(gh, "bf16"))
+            else:
+                Wg.append((torch.randn(shape, device="cuda", generator=gen) * 0.02).to(torch.bfloat16))
+                Gg.append((torch.randn(shape, device="cuda", generator=gen) * 1e-3).to(torch.bfloat16))
+        W.append(Wg)
+        G.append(Gg)
+        M.append([torch.zeros(shape, device="cuda") for _ in range(48)])
+    from spectral_optimizer_state_b200 import Muon
+    mu = Muon(0)
+    mu.set_coeffs(QUINTIC5)
+    mu.step_groups([(W[g], G[g], M[g]) for g in range(2)], **HP)
+    st, flags = mu.status()
+    assert st == 0 and not any(flags)
+    for g in range(2):
+        wh, gh = host[g]
+        r = oracle.muon_step(wh, gh.astype(np.float64), np.zeros(wh.shape), QUINTIC5, **HP)
+        l = check[g]
+        assert rel_f(to_numpy(M[g][l]), r["M"]) <= 1e-6
+        bound = BF16_TOL * np.linalg.norm(r["W"] - wh) + np.linalg.norm(half_ulp_bf16(r["W"]))
+        assert np.linalg.norm(to_numpy(W[g][l]) - r["W"]) <= bound
+    mu.close()
