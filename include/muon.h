@@ -192,6 +192,32 @@ typedef struct {
 muon_status muon_profile_enable(muon_ctx* ctx, int on);
 muon_status muon_profile_read(muon_ctx* ctx, muon_profile* out, int reset);
 
+/* Top singular triplet of each matrix by power iteration (Muon Meets Mamba:
+ * Spectral Optimization for State Space Models, abstract: Muon lowers the
+ * condition number of the projection it trains; the top singular value is the
+ * quantity to watch).  Starting from v_l (any nonzero vector; the previous
+ * step's v warm-starts it), `iters` times:
+ *   u = W v / |W v| ;  v = W^T u / |W^T u| ;  sigma = |W^T u|.
+ * W: host array of device pointers, rows x cols of `dtype`, read only.
+ * u: device pointers, `rows` floats each, written; v: `cols` floats each, in/out.
+ * sigma: DEVICE array of `batch` floats, written.  Uses context scratch. */
+muon_status muon_power_iteration(muon_ctx* ctx, const void* const* W, float* const* u, float* const* v,
+                                 float* sigma, int batch, int rows, int cols, int dtype, int iters,
+                                 void* stream);
+
+/* muon_step with the spectral cap (An Isotropy-Preserving Spectral Cap for
+ * Muon: each update loses the direction that contributes most to the growth
+ * of the top eigenvalue).  With (u_l, v_l) the top singular pair of the
+ * PRE-step W_l (e.g. from muon_power_iteration before this call), the
+ * orthogonalised update O_l is replaced by O_l - alpha_l u_l v_l^T,
+ * alpha_l = u_l^T O_l v_l, before the scale and decay are applied, so the
+ * update does not grow sigma_max(W_l) to first order.  u: `rows` floats,
+ * v: `cols` floats per matrix (device); alpha: DEVICE array of `batch`
+ * floats, written.  Other arguments as muon_step. */
+muon_status muon_step_capped(muon_ctx* ctx, void* const* W, const void* const* G, float* const* M,
+                             const float* const* u, const float* const* v, int batch, int rows, int cols,
+                             int dtype, const muon_hparams* hp, float* alpha, void* stream);
+
 /* AdamW for the parameters Muon does not take (Muon Meets Mamba: Spectral
  * Optimization for State Space Models, abstract: every weight group not
  * trained with Muon is trained with AdamW).  For each of `count` tensors t:

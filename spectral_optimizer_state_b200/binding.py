@@ -37,6 +37,7 @@ EXPORTS = (
     "muon_set_coeffs", "muon_get_coeffs", "muon_step", "muon_step_groups", "muon_step_groups_host",
     "muon_ns_orthogonalize", "muon_get_status", "muon_get_norms", "muon_workspace_bytes",
     "muon_profile_enable", "muon_profile_read", "muon_momentum_norm_noalloc", "muon_adamw_step",
+    "muon_power_iteration", "muon_step_capped",
 )
 KERNEL_KINDS = ("momentum", "gram", "poly", "update", "apply", "ns_fused")
 
@@ -105,6 +106,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "muon_momentum_norm_noalloc": (i, [pvp, pvp, vp, i, i, i, i, f, i, vp]),
         "muon_adamw_step": (i, [pvp, pvp, pvp, pvp, ctypes.POINTER(ctypes.c_longlong), i, i,
                                 ctypes.POINTER(AdamWHparams), vp]),
+        "muon_power_iteration": (i, [vp, pvp, pvp, pvp, vp, i, i, i, i, i, vp]),
+        "muon_step_capped": (i, [vp, pvp, pvp, pvp, pvp, pvp, i, i, i, i, ctypes.POINTER(Hparams), vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -265,6 +268,41 @@ class Muon:
         st = self.lib.muon_ns_orthogonalize(self.handle, px, po, len(X), shape[0], shape[1],
                                             _dtype_code(X[0]), float(eps), _stream_handle(stream))
         self._check(st, "muon_ns_orthogonalize")
+
+    # -------------------------------------------------------------- spectral
+    def power_iteration(self, W, u, v, sigma, iters=8, stream=None):
+        """Top singular triplet of each W[l] by `iters` power iterations.
+
+        v[l] (fp32, cols) holds the start vector and receives the right vector;
+        u[l] (fp32, rows) receives the left vector; sigma (fp32 CUDA, len(W))
+        the top singular value.
+        """
+        import torch
+        shape, dt = tuple(W[0].shape), W[0].dtype
+        _check_same(W, shape, dt, "cuda", "W")
+        _check_same(u, (shape[0],), torch.float32, "cuda", "u")
+        _check_same(v, (shape[1],), torch.float32, "cuda", "v")
+        if not (len(W) == len(u) == len(v)) or sigma.numel() < len(W) or sigma.dtype != torch.float32:
+            raise ValueError("W, u, v need one entry per matrix and sigma len(W) fp32 slots")
+        pw, pu, pv = _ptrs(W), _ptrs(u), _ptrs(v)
+        st = self.lib.muon_power_iteration(self.handle, pw, pu, pv, ctypes.c_void_p(sigma.data_ptr()), len(W),
+                                           shape[0], shape[1], _dtype_code(W[0]), int(iters),
+                                           _stream_handle(stream))
+        self._check(st, "muon_power_iteration")
+
+    def step_capped(self, W, G, M, u, v, alpha, stream=None, **hp):
+        """step() with the update's component along u[l] v[l]^T removed; alpha[l] receives u^T O v."""
+        import torch
+        g, (pw, pg, pm) = self._group(W, G, M)
+        _check_same(u, (g.rows,), torch.float32, "cuda", "u")
+        _check_same(v, (g.cols,), torch.float32, "cuda", "v")
+        if not (len(u) == len(v) == len(W)) or alpha.numel() < len(W) or alpha.dtype != torch.float32:
+            raise ValueError("u, v need one entry per matrix and alpha len(W) fp32 slots")
+        pu, pv = _ptrs(u), _ptrs(v)
+        h = self.hparams(**hp)
+        st = self.lib.muon_step_capped(self.handle, pw, pg, pm, pu, pv, g.batch, g.rows, g.cols, g.dtype,
+                                       ctypes.byref(h), ctypes.c_void_p(alpha.data_ptr()), _stream_handle(stream))
+        self._check(st, "muon_step_capped")
 
     # -------------------------------------------------------------- status
     def status(self):

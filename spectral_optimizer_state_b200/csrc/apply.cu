@@ -114,6 +114,11 @@ __global__ void __launch_bounds__(kThreads) apply_wide_kernel(const __grid_const
       const int j = static_cast<int>(v - i * per_row) * 8;
       float ov[8];
       load8_planes(o + i * p.pitch + j, p.o_plane, p.planes, ov);
+      if (p.alpha != nullptr) {
+        const float au = p.alpha[l] * p.cu[l][i];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) ov[t] = fmaf(-au, p.cv[l][j + t], ov[t]);
+      }
       char* dst = static_cast<char*>(w) + (i * C + j) * (F32 ? 4 : 2);
       rmw8<F32>(dst, ov, p.apply, p.decay, p.lrs);
     }
@@ -125,7 +130,9 @@ __global__ void __launch_bounds__(kThreads) apply_wide_kernel(const __grid_const
     for (long long e = beg + threadIdx.x; e < end; e += kThreads) {
       const long long i = e / C;
       const int j = static_cast<int>(e - i * C);
-      rmw1<F32>(w, e, load1_planes(o + i * p.pitch + j, p.o_plane, p.planes), p.apply, p.decay, p.lrs);
+      float ov = load1_planes(o + i * p.pitch + j, p.o_plane, p.planes);
+      if (p.alpha != nullptr) ov = fmaf(-p.alpha[l] * p.cu[l][i], p.cv[l][j], ov);
+      rmw1<F32>(w, e, ov, p.apply, p.decay, p.lrs);
     }
   }
 }
@@ -171,6 +178,12 @@ __global__ void __launch_bounds__(kThreads) apply_tall_kernel(const __grid_const
         float ov[8];
 #pragma unroll
         for (int t = 0; t < 8; ++t) ov[t] = tile[rl][cc + t];
+        if (p.alpha != nullptr) {
+          const float au = p.alpha[l] * p.cu[l][r];
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            if (c + t < C) ov[t] = fmaf(-au, p.cv[l][c + t], ov[t]);
+        }
         if (VEC) {
           if (c < C) {
             char* dst = static_cast<char*>(w) + (static_cast<long long>(r) * C + c) * (F32 ? 4 : 2);

@@ -49,9 +49,38 @@ struct ApplyParams {
   float decay, lrs;
   const int* flags;         // matrices with a nonzero flag are left unchanged (null: none)
   int nblk;                 // blocks per matrix
+  // spectral cap (null alpha: none): O is replaced by O - alpha_l u_l v_l^T,
+  // u_l of length rows and v_l of length cols of W
+  const float* cu[MUON_MAX_BATCH];
+  const float* cv[MUON_MAX_BATCH];
+  const float* alpha;
 };
 
 cudaError_t launch_apply(const ApplyParams& p, int batch, bool w_f32, cudaStream_t stream);
+
+// ------------------------------------------------------------------ spectral
+struct GemvParams {
+  const void* w[MUON_MAX_BATCH];   // rows x cols, bf16 or fp32
+  const float* x[MUON_MAX_BATCH];  // input: length cols (rows GEMV) or rows (cols GEMV)
+  float* y[MUON_MAX_BATCH];        // output: length rows (rows GEMV) or cols (cols GEMV)
+  int rows, cols;
+  float* partial;                  // cols GEMV: [batch][row_chunks][cols]
+  int row_chunks, rows_per_chunk;
+};
+
+struct CapParams {
+  const float* a[MUON_MAX_BATCH];  // length m (wide rows)
+  const float* b[MUON_MAX_BATCH];  // length n (wide columns)
+  const uint16_t* o;               // final iterate, wide, [planes][batch][m][pitch]
+  long long o_plane, o_mat;
+  int pitch, m, n, planes, rows_per_block;
+  double* partial;                 // [batch][blocks]
+};
+
+cudaError_t launch_gemv_rows(const GemvParams& p, int batch, bool f32, cudaStream_t s);
+cudaError_t launch_gemv_cols(const GemvParams& p, int batch, bool f32, cudaStream_t s);
+cudaError_t launch_normalize(float* const* vecs_dev, int batch, int n, float* norm, cudaStream_t s);
+cudaError_t launch_cap_alpha(const CapParams& p, int batch, float* alpha, cudaStream_t s);
 
 // ------------------------------------------------------------------ GEMM
 // The epilogue forms  v = alpha * s_l * acc + beta * cin + (row == col ? diag : 0)

@@ -141,6 +141,9 @@ struct muon_ctx {
   // device staging for gradients that arrive from host memory
   void* d_stage = nullptr;
   size_t stage_bytes = 0;
+  // scratch of the spectral passes (GEMV partials, norms, cap partials)
+  void* d_aux = nullptr;
+  size_t aux_bytes = 0;
   // per-launch timing
   bool profiling = false;
   std::vector<cudaEvent_t> events;  // pool, two per recorded launch
@@ -365,8 +368,30 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
   return true;
 }
 
+// Spectral cap of one group: per-matrix top singular vectors of the pre-step W
+// (u: length rows, v: length cols) and where the coefficients go.
+struct CapSpec {
+  const float* const* u;
+  const float* const* v;
+  float* alpha;  // device [batch]
+};
+
+muon_status ensure_aux(muon_ctx* c, size_t bytes) {
+  if (bytes <= c->aux_bytes) return MUON_OK;
+  MUON_CUDA(cudaDeviceSynchronize(), "sync before scratch growth");
+  cudaFree(c->d_aux);
+  c->d_aux = nullptr;
+  c->aux_bytes = 0;
+  if (cudaMalloc(&c->d_aux, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return MUON_ERR_ALLOC;
+  }
+  c->aux_bytes = bytes;
+  return MUON_OK;
+}
+
 muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* hp, bool step,
-                float eps, cudaStream_t s) {
+                float eps, cudaStream_t s, const CapSpec* cap = nullptr) {
   muon_status st = reserve(c, plans, s);
   if (st != MUON_OK) return st;
   int total = 0;
@@ -485,6 +510,30 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
     prof_end(c, slot, s);
   }
 
+  // Spectral cap: alpha_l = u_l^T O_l v_l from the final iterate (one group).
+  if (cap != nullptr) {
+    const GroupPlan& p = plans[0];
+    CapParams cp;
+    std::memset(static_cast<void*>(&cp), 0, sizeof(cp));
+    for (int l = 0; l < p.batch; ++l) {
+      cp.a[l] = p.transposed ? cap->v[l] : cap->u[l];  // wide rows are W's columns when tall
+      cp.b[l] = p.transposed ? cap->u[l] : cap->v[l];
+    }
+    cp.o = ws_at(c, p.off_x[c->k & 1]);
+    cp.o_plane = p.x_plane;
+    cp.o_mat = p.x_mat;
+    cp.pitch = p.pitch_n;
+    cp.m = p.m_rows;
+    cp.n = p.n_cols;
+    cp.planes = p.planes;
+    cp.rows_per_block = 8;
+    const size_t need = sizeof(double) * p.batch * ((p.m_rows + 7) / 8);
+    st = ensure_aux(c, need);
+    if (st != MUON_OK) return st;
+    cp.partial = static_cast<double*>(c->d_aux);
+    MUON_CUDA(launch_cap_alpha(cp, p.batch, cap->alpha, s), "cap coefficient");
+  }
+
   // K5: scale + decoupled decay applied to W (or the plain copy to Out).
   for (auto& p : plans) {
     ApplyParams ap;
@@ -504,6 +553,13 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
       ap.flags = c->d_flags + p.mat_off;
     }
     ap.nblk = momentum_blocks_per_matrix(p.rows, p.cols);
+    if (cap != nullptr) {
+      for (int l = 0; l < p.batch; ++l) {
+        ap.cu[l] = cap->u[l];
+        ap.cv[l] = cap->v[l];
+      }
+      ap.alpha = cap->alpha;
+    }
     const int slot = prof_begin(c, MUON_KERNEL_APPLY, s);
     MUON_CUDA(launch_apply(ap, p.batch, p.f32 != 0, s), "apply kernel");
     prof_end(c, slot, s);
@@ -605,6 +661,7 @@ muon_status muon_destroy(muon_ctx* c) {
   cudaFree(c->d_status);
   cudaFree(c->d_done);
   cudaFree(c->d_stage);
+  cudaFree(c->d_aux);
   for (cudaEvent_t e : c->events) cudaEventDestroy(e);
   delete c;
   return MUON_OK;
@@ -759,9 +816,76 @@ muon_status muon_step_groups_host(muon_ctx* c, const muon_group* groups, int ngr
   return muon_get_status(c, nullptr, 0, nullptr);
 }
 
+muon_status muon_power_iteration(muon_ctx* c, const void* const* W, float* const* u, float* const* v,
+                                 float* sigma, int batch, int rows, int cols, int dtype, int iters,
+                                 void* stream) {
+  if (!c || !W || !u || !v || !sigma || batch < 1 || batch > MUON_MAX_BATCH || iters < 1 || iters > 10000)
+    return MUON_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 1) return MUON_ERR_INVALID_ARG;
+  if (rows > 32768 || cols > 32768) return MUON_ERR_UNSUPPORTED_SHAPE;
+  if (dtype != MUON_BF16 && dtype != MUON_F32) return MUON_ERR_DTYPE;
+  for (int l = 0; l < batch; ++l)
+    if (!W[l] || !u[l] || !v[l]) return MUON_ERR_INVALID_ARG;
+  DeviceGuard guard(c->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  GemvParams gp;
+  std::memset(static_cast<void*>(&gp), 0, sizeof(gp));
+  gp.rows = rows;
+  gp.cols = cols;
+  gp.rows_per_chunk = 64;
+  gp.row_chunks = (rows + 63) / 64;
+  const size_t part_bytes = align_up(sizeof(float) * batch * gp.row_chunks * cols, 256);
+  muon_status st = ensure_aux(c, part_bytes + sizeof(float) * MUON_MAX_BATCH);
+  if (st != MUON_OK) return st;
+  gp.partial = static_cast<float*>(c->d_aux);
+  float* norms = reinterpret_cast<float*>(static_cast<char*>(c->d_aux) + part_bytes);
+  const bool f32 = dtype == MUON_F32;
+  for (int l = 0; l < batch; ++l) gp.w[l] = W[l];
+  MUON_CUDA(launch_normalize(v, batch, cols, norms, s), "normalise start vector");
+  for (int i = 0; i < iters; ++i) {
+    for (int l = 0; l < batch; ++l) {
+      gp.x[l] = v[l];
+      gp.y[l] = u[l];
+    }
+    MUON_CUDA(launch_gemv_rows(gp, batch, f32, s), "W v");
+    MUON_CUDA(launch_normalize(u, batch, rows, norms, s), "normalise u");
+    for (int l = 0; l < batch; ++l) {
+      gp.x[l] = u[l];
+      gp.y[l] = v[l];
+    }
+    MUON_CUDA(launch_gemv_cols(gp, batch, f32, s), "W^T u");
+    MUON_CUDA(launch_normalize(v, batch, cols, sigma, s), "normalise v");
+  }
+  return MUON_OK;
+}
+
+muon_status muon_step_capped(muon_ctx* c, void* const* W, const void* const* G, float* const* M,
+                             const float* const* u, const float* const* v, int batch, int rows, int cols,
+                             int dtype, const muon_hparams* hp, float* alpha, void* stream) {
+  if (!u || !v || !alpha) return MUON_ERR_INVALID_ARG;
+  muon_group g;
+  g.W = W;
+  g.G = G;
+  g.M = M;
+  g.batch = batch;
+  g.rows = rows;
+  g.cols = cols;
+  g.dtype = dtype;
+  std::vector<GroupPlan> plans;
+  muon_status st = validate_and_plan(c, &g, 1, true, plans);
+  if (st != MUON_OK) return st;
+  st = check_hparams(hp);
+  if (st != MUON_OK) return st;
+  for (int l = 0; l < batch; ++l)
+    if (!u[l] || !v[l]) return MUON_ERR_INVALID_ARG;
+  DeviceGuard guard(c->device);
+  CapSpec cap{u, v, alpha};
+  return run(c, plans, hp, true, hp->eps, static_cast<cudaStream_t>(stream), &cap);
+}
+
 size_t muon_workspace_bytes(const muon_ctx* c) {
   if (!c) return 0;
-  return c->ws_bytes + c->stage_bytes;
+  return c->ws_bytes + c->stage_bytes + c->aux_bytes;
 }
 
 muon_status muon_profile_enable(muon_ctx* c, int on) {

@@ -1,0 +1,151 @@
+"""Power iteration and the spectral-capped step vs the fp64 oracle (needs a B200)."""
+import numpy as np
+import pytest
+
+import oracle
+from synthetic import MAMBA2_130M_IN_PROJ, gaussian_spike, rng_for, round_bf16, weights
+from tests.gpu_common import BF16_TOL, F32_TOL, rel_f, to_device, to_numpy
+
+pytestmark = pytest.mark.gpu
+
+# wide, tall, ragged (scalar paths: cols % 8 != 0), and one past the 48 KB shared-memory default
+SHAPES = [(96, 200, 3), (200, 96, 2), (77, 45, 2), (45, 77, 1), (64, 13000, 1)]
+
+
+def _spiked(rows, cols, batch, seed, dtype):
+    Ws = []
+    for l in range(batch):
+        W = gaussian_spike(rng_for(seed, l), rows, cols, rank=1)
+        Ws.append(round_bf16(W) if dtype == "bf16" else W.astype(np.float32))
+    return Ws
+
+
+def _power(muon, Ws, v0s, iters, dtype):
+    import torch
+    W = [to_device(w, dtype) for w in Ws]
+    u = [torch.zeros(w.shape[0], dtype=torch.float32, device="cuda") for w in Ws]
+    v = [torch.from_numpy(v0.astype(np.float32)).cuda() for v0 in v0s]
+    sigma = torch.zeros(len(Ws), dtype=torch.float32, device="cuda")
+    muon.power_iteration(W, u, v, sigma, iters=iters)
+    torch.cuda.synchronize()
+    return [to_numpy(x) for x in u], [to_numpy(x) for x in v], to_numpy(sigma)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("rows,cols,batch", SHAPES)
+def test_power_iteration_matches_oracle(rows, cols, batch, dtype):
+    from spectral_optimizer_state_b200 import Muon
+    Ws = _spiked(rows, cols, batch, 71, dtype)
+    v0s = [rng_for(72, l).standard_normal(cols).astype(np.float32) for l in range(batch)]
+    with Muon() as muon:
+        u, v, sigma = _power(muon, Ws, v0s, 6, dtype)
+    for l in range(batch):
+        ru, rv, rs = oracle.power_iteration(Ws[l].astype(np.float64), v0s[l].astype(np.float64), 6)
+        # fp32 accumulation over at most 13000 terms of one sign-mixed dot product
+        assert abs(sigma[l] - rs) <= 1e-5 * rs
+        assert rel_f(u[l], ru) <= 1e-4
+        assert rel_f(v[l], rv) <= 1e-4
+
+
+def test_power_iteration_reaches_the_svd_on_full_size_in_proj():
+    """in_proj shape of the 130M model: 24 matrices with a planted top direction, 30 iterations."""
+    from spectral_optimizer_state_b200 import Muon
+    rows, cols = MAMBA2_130M_IN_PROJ
+    Ws = _spiked(rows, cols, 24, 73, "bf16")
+    v0s = [np.ones(cols, np.float32) for _ in range(24)]
+    with Muon() as muon:
+        _, v, sigma = _power(muon, Ws, v0s, 30, "bf16")
+    for l in (0, 11, 23):
+        _, s, Vt = np.linalg.svd(Ws[l].astype(np.float64), full_matrices=False)
+        assert abs(sigma[l] - s[0]) <= 1e-4 * s[0]
+        assert abs(abs(v[l] @ Vt[0]) - 1.0) <= 1e-4
+
+
+def test_power_iteration_zero_matrix_gives_zero_triplet():
+    from spectral_optimizer_state_b200 import Muon
+    Ws = [np.zeros((40, 72), np.float32)]
+    with Muon() as muon:
+        u, v, sigma = _power(muon, Ws, [np.ones(72, np.float32)], 3, "f32")
+    ru, rv, rs = oracle.power_iteration(Ws[0], np.ones(72), 3)
+    assert sigma[0] == rs == 0.0
+    assert not u[0].any() and not v[0].any() and not ru.any() and not rv.any()
+
+
+def _capped_case(rows, cols, batch, dtype, seed):
+    W0 = [weights(rng_for(seed, l), rows, cols) for l in range(batch)]
+    G = [gaussian_spike(rng_for(seed + 1, l), rows, cols, rank=4) for l in range(batch)]
+    if dtype == "bf16":
+        W0 = [round_bf16(w) for w in W0]
+        G = [round_bf16(g) for g in G]
+    else:
+        W0 = [w.astype(np.float32) for w in W0]
+        G = [g.astype(np.float32) for g in G]
+    uv = [oracle.power_iteration(w.astype(np.float64), np.ones(cols), 20)[:2] for w in W0]
+    return W0, G, uv
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("rows,cols,batch", [(192, 320, 2), (320, 192, 3), (77, 45, 1), (256, 256, 1)])
+def test_step_capped_matches_oracle(rows, cols, batch, dtype):
+    import torch
+    from spectral_optimizer_state_b200 import Muon
+    W0, G, uv = _capped_case(rows, cols, batch, dtype, 81)
+    hp = dict(lr=0.02, beta=0.95, weight_decay=0.1, eps=1e-7, nesterov=True, scale_mode=0)
+    W = [to_device(w, dtype) for w in W0]
+    Gd = [to_device(g, dtype) for g in G]
+    M = [torch.zeros((rows, cols), dtype=torch.float32, device="cuda") for _ in range(batch)]
+    u = [torch.from_numpy(x.astype(np.float32)).cuda() for x, _ in uv]
+    v = [torch.from_numpy(y.astype(np.float32)).cuda() for _, y in uv]
+    alpha = torch.zeros(batch, dtype=torch.float32, device="cuda")
+    with Muon() as muon:
+        coeffs = muon.get_coeffs()
+        muon.step_capped(W, Gd, M, u, v, alpha, **hp)
+        torch.cuda.synchronize()
+    tol = BF16_TOL if dtype == "bf16" else F32_TOL
+    a = to_numpy(alpha)
+    for l in range(batch):
+        # u, v as the kernel saw them (fp32)
+        ul, vl = uv[l][0].astype(np.float32).astype(np.float64), uv[l][1].astype(np.float32).astype(np.float64)
+        r = oracle.muon_step_capped(W0[l].astype(np.float64), G[l].astype(np.float64), np.zeros((rows, cols)),
+                                    coeffs, ul, vl, **hp)
+        dW_ref = r["W"] - W0[l]
+        dW = to_numpy(W[l]) - W0[l]
+        if dtype == "f32":
+            assert rel_f(dW, dW_ref) <= tol
+        else:
+            # the bf16 store of W rounds each element by at most half a bf16 ulp of the new value
+            assert rel_f(dW, dW_ref) <= tol + np.linalg.norm(np.abs(r["W"]) * 2.0 ** -8) / np.linalg.norm(dW_ref)
+        # |d alpha| = |u^T dO v| <= ||dO||_2 <= ||dO||_F
+        O_norm = np.linalg.norm(r["O"] + r["alpha"] * np.outer(ul, vl))
+        assert abs(a[l] - r["alpha"]) <= tol * O_norm
+        assert rel_f(to_numpy(M[l]), r["M"]) <= 1e-6
+
+
+def test_capped_update_has_no_component_along_the_top_pair():
+    """fp32 W: u^T (W_new - decay W_old) v is zero up to the orthogonalisation error."""
+    import torch
+    from spectral_optimizer_state_b200 import Muon
+    rows, cols = 320, 192
+    W0, G, uv = _capped_case(rows, cols, 1, "f32", 91)
+    W = [to_device(W0[0], "f32")]
+    M = [torch.zeros((rows, cols), dtype=torch.float32, device="cuda")]
+    u = [torch.from_numpy(uv[0][0].astype(np.float32)).cuda()]
+    v = [torch.from_numpy(uv[0][1].astype(np.float32)).cuda()]
+    alpha = torch.zeros(1, dtype=torch.float32, device="cuda")
+    lr, wd = 0.02, 0.1
+    with Muon() as muon:
+        muon.step_capped(W, [to_device(G[0], "f32")], M, u, v, alpha, lr=lr, weight_decay=wd)
+        torch.cuda.synchronize()
+    dW = to_numpy(W[0]) - (1 - lr * wd) * W0[0].astype(np.float64)
+    ul, vl = to_numpy(u[0]), to_numpy(v[0])
+    assert abs(ul @ dW @ vl) <= 1e-5 * np.linalg.norm(dW)
+    assert abs(to_numpy(alpha)[0]) > 1e-3  # the cap removed something
+
+
+def test_step_capped_rejects_missing_vectors():
+    import torch
+    from spectral_optimizer_state_b200 import Muon, MuonError
+    W = [torch.zeros((64, 64), dtype=torch.float32, device="cuda")]
+    with Muon() as muon:
+        with pytest.raises((MuonError, ValueError)):
+            muon.step_capped(W, W, [w.clone() for w in W], [], [], torch.zeros(1, device="cuda"))
