@@ -23,7 +23,8 @@ triple and the shape-scale convention.  Parity holds for whichever values are
 passed.
 """
 from .adamw_oracle import adamw_step, select_muon  # noqa: F401
-from .spectral_oracle import muon_step_capped, power_iteration, spectral_cap, stable_rank  # noqa: F401
+from .spectral_oracle import (min_singular_shifted, muon_step_capped, power_iteration, spectral_cap,  # noqa: F401
+                              stable_rank)
 from .muon_oracle import (  # noqa: F401
     CUBIC, QUINTIC, SCALE_SQRT_RATIO, SCALE_NONE, SCALE_RMS_MATCH,
     momentum_update, nesterov_lookahead, frobenius_norm, normalize,

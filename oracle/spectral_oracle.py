@@ -16,7 +16,8 @@ from __future__ import annotations
 
 import numpy as np
 
-from .muon_oracle import apply_update, momentum_update, nesterov_lookahead, orthogonalize, shape_scale, frobenius_norm
+from .muon_oracle import (apply_update, frobenius_norm, momentum_update, nesterov_lookahead, orthogonalize,
+                          shape_scale, wide_view)
 
 
 def power_iteration(W, v0, iters: int):
@@ -41,6 +42,30 @@ def power_iteration(W, v0, iters: int):
             return u, np.zeros(W.shape[1]), 0.0
         v = v / sigma
     return u, v, sigma
+
+
+def min_singular_shifted(W, y0, sigma_max: float, iters: int):
+    """Smallest singular value of W's wide view X (m = min(rows, cols) rows) by shifted power iteration.
+
+    With s = sigma_max^2, the largest eigenvalue of s I - X X^T is s - sigma_min^2,
+    so `iters` steps of y <- (s y - X (X^T y)) / |.| turn y toward the bottom left
+    singular vector of X; the estimate is the Rayleigh value |X^T y|, which is
+    >= sigma_min for every unit y.  Returns (y, sigma_min); kappa = sigma_max /
+    sigma_min.  READING: the pages report the condition number falling under
+    Muon without saying how it is computed; this is the plainest iteration that
+    needs only products with W.
+    """
+    X, _ = wide_view(np.asarray(W, np.float64))
+    s = float(sigma_max) ** 2
+    y = np.asarray(y0, np.float64)
+    y = y / np.linalg.norm(y)
+    for _ in range(iters):
+        y = s * y - X @ (X.T @ y)
+        n = np.linalg.norm(y)
+        if n == 0.0:
+            break
+        y = y / n
+    return y, float(np.linalg.norm(X.T @ y))
 
 
 def stable_rank(W, sigma_max: float) -> float:

@@ -67,3 +67,34 @@ def test_capped_step_matches_plain_step_when_direction_is_orthogonal():
     v = np.zeros(30)
     capped = oracle.muon_step_capped(W, G, np.zeros_like(G), q5, u, v)
     assert np.allclose(capped["W"], plain["W"], rtol=0, atol=1e-15) and capped["alpha"] == 0.0
+
+
+def test_min_singular_reaches_lapack_with_a_bottom_gap():
+    s = np.concatenate([np.linspace(3.0, 1.0, 29), [0.1]])  # full rank: 30 singular values
+    for m, n in ((30, 50), (50, 30)):  # wide and tall: the iteration runs on the short side
+        W, U, V = _with_spectrum(m, n, s, 3)
+        y0 = rng_for(4, 0).standard_normal(min(m, n))
+        y, smin = oracle.min_singular_shifted(W, y0, 3.0, 300)
+        # rate (9 - 1) / (9 - 0.01) per step on y; the Rayleigh value converges at its square
+        assert abs(smin - 0.1) < 1e-9
+        bottom = U[:, -1] if m <= n else V[:, -1]
+        assert abs(abs(y @ bottom) - 1) < 1e-9
+
+
+def test_min_singular_is_exact_on_semi_orthogonal_and_an_upper_bound_otherwise():
+    Q, _ = np.linalg.qr(rng_for(5, 0).standard_normal((90, 40)))
+    _, smin = oracle.min_singular_shifted(Q.T, np.ones(40), 1.0, 3)
+    assert abs(smin - 1.0) < 1e-13
+    G = gaussian(rng_for(6, 0), 40, 70)
+    true_min = np.linalg.svd(G, compute_uv=False)[-1]
+    for k in (0, 1, 5, 40):
+        _, est = oracle.min_singular_shifted(G, np.ones(40), np.linalg.norm(G, 2), k)
+        assert est >= true_min * (1 - 1e-12)
+
+
+def test_min_singular_brute_force_two_by_three():
+    # W W^T = diag(4, 1): sigma = (2, 1); one shifted step from (1, 1) with s = 4 gives y = (0, 3) / 3
+    W = np.array([[2.0, 0.0, 0.0], [0.0, 0.6, 0.8]])
+    y, smin = oracle.min_singular_shifted(W, np.array([1.0, 1.0]), 2.0, 1)
+    assert np.allclose(y, [0.0, 1.0], rtol=0, atol=1e-15)
+    assert abs(smin - 1.0) < 1e-15
