@@ -230,7 +230,7 @@ def blas_threads():
         return os.cpu_count()
 
 
-def oracle_sample(groups, budget_s=20.0, max_per_group=24):
+def oracle_sample(groups, budget_s=12.0, max_per_group=96):
     """Time the fp64 oracle on whole matrices of one step until ~budget_s; returns steps/s and a label."""
     import oracle
     from synthetic import group_inputs, group_weights
@@ -251,8 +251,75 @@ def oracle_sample(groups, budget_s=20.0, max_per_group=24):
             frac += 1.0 / total_mats
         if t_total >= budget_s:
             break
-    sample = " + ".join(f"{n} {lbl}" for lbl, n in done.items()) + " matrices of one step (oracle.muon_step, fp64 NumPy)"
+    sample = (" + ".join(f"{n} {lbl}" for lbl, n in done.items())
+              + " matrices, alternating groups, until about 12 s of fp64 NumPy (oracle.muon_step)")
     return frac / t_total, sample, t_total
+
+
+def measure_spectral(mu, Ws, Gs, Ms, groups, stream, peaks, pi_iters=8, min_iters=16, reps=5):
+    """Spectral diagnostics and the capped step on every group of the workload (device-timed)."""
+    import torch
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    w_bytes = sum(L * R * C * 2 for _, L, R, C in groups)
+    dev = Ws[0][0].device
+    vecs = []
+    for g, (_, L, R, C) in enumerate(groups):
+        u = [torch.zeros(R, device=dev) for _ in range(L)]
+        v = [torch.ones(C, device=dev) for _ in range(L)]
+        y = [torch.ones(min(R, C), device=dev) for _ in range(L)]
+        vecs.append((u, v, y, torch.zeros(L, device=dev), torch.zeros(L, device=dev), torch.zeros(L, device=dev)))
+
+    def power():
+        for g in range(len(groups)):
+            u, v, _, smax, _, _ = vecs[g]
+            mu.power_iteration(Ws[g], u, v, smax, iters=pi_iters, stream=stream)
+
+    def min_sv():
+        for g in range(len(groups)):
+            _, _, y, smax, smin, _ = vecs[g]
+            mu.min_singular(Ws[g], y, smax, smin, iters=min_iters, stream=stream)
+
+    def plain():
+        for g in range(len(groups)):
+            mu.step(Ws[g], Gs[g], Ms[g], stream=stream, **HP)
+
+    def capped():
+        for g in range(len(groups)):
+            u, v, _, _, _, alpha = vecs[g]
+            mu.step_capped(Ws[g], Gs[g], Ms[g], u, v, alpha, stream=stream, **HP)
+
+    pi_ms = timed(power)
+    min_ms = timed(min_sv)
+    plain_ms = timed(plain)
+    cap_ms = timed(capped)
+    st, _ = mu.status()
+    assert st == 0, f"device status {st}"
+    kappa = [float((vecs[g][3] / vecs[g][4]).max()) for g in range(len(groups))]
+    pi_gbs = 2 * pi_iters * w_bytes / (pi_ms / 1e3) / 1e9
+    min_gbs = (2 * min_iters + 1) * w_bytes / (min_ms / 1e3) / 1e9
+    hbm = peaks["hbm_gbs"]
+    return {
+        "bound": "hbm",
+        "note": ("GEMV passes over W; algorithmic bytes count every pass over W (2 per power iteration, "
+                 "2 per shifted iteration + 1), and one group's W (<= 124 MB at 130M) can stay in the "
+                 "126 MB L2 between passes"),
+        "power_iteration": {"iters": pi_iters, "ms": pi_ms, "achieved_gbs": pi_gbs, "frac": pi_gbs / hbm},
+        "min_singular": {"iters": min_iters, "ms": min_ms, "achieved_gbs": min_gbs, "frac": min_gbs / hbm,
+                         "max_kappa_estimate": kappa},
+        "capped_step_ms": cap_ms, "plain_step_ms": plain_ms, "cap_overhead_ms": cap_ms - plain_ms,
+        "step_entry": "muon_step / muon_step_capped per group (not the fused two-group call)",
+    }
 
 
 def run_reference(args, groups, rank):
@@ -320,6 +387,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="mamba2-130m")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-spectral", dest="spectral", action="store_false",
+                    help="skip the power-iteration / min-singular / capped-step measurements")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     groups = WORKLOADS[args.workload]
@@ -437,6 +506,8 @@ def main():
                  "tensors": len(aw), "note": "AdamW over the non-Muon parameters of Mamba-2 130M, bf16"}
         del aw, ag, am, av
 
+    spectral = measure_spectral(mu, Ws, Gsets[0], Ms, groups, stream, peaks) if args.spectral else None
+
     n_mats = sum(L for _, L, _, _ in groups)
     steps_per_s = world * args.steps / (ms / 1e3)
     gemm_kinds = ("gram", "poly", "update", "ns_fused")
@@ -481,6 +552,7 @@ def main():
                          "bytes_per_element": 6, "launches": app_launches},
         "kernel_ms_per_step": {k: v[1] / args.steps for k, v in prof.items()},
         "adamw_kernel": adamw,
+        "spectral": spectral,
         "cpu_baseline": cpu,
         "clocks": clk,
         "e2e": {"value": world * e2e_steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,

@@ -205,6 +205,21 @@ muon_status muon_power_iteration(muon_ctx* ctx, const void* const* W, float* con
                                  float* sigma, int batch, int rows, int cols, int dtype, int iters,
                                  void* stream);
 
+/* Smallest singular value of each matrix by shifted power iteration, so that
+ * the condition number sigma_max / sigma_min can be tracked (Muon Meets Mamba:
+ * Spectral Optimization for State Space Models, abstract: the condition number
+ * falls under Muon).  On the wide view X (W, or W^T when rows > cols; m =
+ * min(rows, cols)), with s = sigma_max[l]^2, `iters` times
+ *   y <- (s y - X X^T y) / |s y - X X^T y|,
+ * then sigma_min[l] = |X^T y|, an upper bound on the true value for every y
+ * that tightens as y turns toward the bottom singular vector.
+ * W: host array of device pointers (rows x cols, `dtype`), read only.
+ * y: device pointers, m floats each: start vector in, iterate out.
+ * sigma_max: DEVICE array of `batch` floats (e.g. from muon_power_iteration);
+ * sigma_min: DEVICE array of `batch` floats, written.  iters may be 0. */
+muon_status muon_min_singular(muon_ctx* ctx, const void* const* W, float* const* y, const float* sigma_max,
+                              float* sigma_min, int batch, int rows, int cols, int dtype, int iters, void* stream);
+
 /* muon_step with the spectral cap (An Isotropy-Preserving Spectral Cap for
  * Muon: each update loses the direction that contributes most to the growth
  * of the top eigenvalue).  With (u_l, v_l) the top singular pair of the

@@ -37,7 +37,7 @@ EXPORTS = (
     "muon_set_coeffs", "muon_get_coeffs", "muon_step", "muon_step_groups", "muon_step_groups_host",
     "muon_ns_orthogonalize", "muon_get_status", "muon_get_norms", "muon_workspace_bytes",
     "muon_profile_enable", "muon_profile_read", "muon_momentum_norm_noalloc", "muon_adamw_step",
-    "muon_power_iteration", "muon_step_capped",
+    "muon_power_iteration", "muon_min_singular", "muon_step_capped",
 )
 KERNEL_KINDS = ("momentum", "gram", "poly", "update", "apply", "ns_fused")
 
@@ -107,6 +107,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "muon_adamw_step": (i, [pvp, pvp, pvp, pvp, ctypes.POINTER(ctypes.c_longlong), i, i,
                                 ctypes.POINTER(AdamWHparams), vp]),
         "muon_power_iteration": (i, [vp, pvp, pvp, pvp, vp, i, i, i, i, i, vp]),
+        "muon_min_singular": (i, [vp, pvp, pvp, vp, vp, i, i, i, i, i, vp]),
         "muon_step_capped": (i, [vp, pvp, pvp, pvp, pvp, pvp, i, i, i, i, ctypes.POINTER(Hparams), vp, vp]),
     }
     for name, (res, args) in sig.items():
@@ -289,6 +290,28 @@ class Muon:
                                            shape[0], shape[1], _dtype_code(W[0]), int(iters),
                                            _stream_handle(stream))
         self._check(st, "muon_power_iteration")
+
+    def min_singular(self, W, y, sigma_max, sigma_min, iters=32, stream=None):
+        """Smallest singular value of each W[l] by `iters` shifted power iterations.
+
+        y[l] (fp32 CUDA, min(rows, cols)) is the start vector and receives the
+        iterate; sigma_max (fp32 CUDA, len(W)) the top singular values, e.g.
+        from power_iteration; sigma_min (fp32 CUDA, len(W)) receives the estimate.
+        """
+        import torch
+        shape, dt = tuple(W[0].shape), W[0].dtype
+        _check_same(W, shape, dt, "cuda", "W")
+        _check_same(y, (min(shape),), torch.float32, "cuda", "y")
+        for t, what in ((sigma_max, "sigma_max"), (sigma_min, "sigma_min")):
+            if t.dtype != torch.float32 or t.numel() < len(W) or t.device.type != "cuda":
+                raise ValueError(f"{what}: needs len(W) fp32 CUDA slots")
+        if len(y) != len(W):
+            raise ValueError("y needs one entry per matrix")
+        pw, py = _ptrs(W), _ptrs(y)
+        st = self.lib.muon_min_singular(self.handle, pw, py, ctypes.c_void_p(sigma_max.data_ptr()),
+                                        ctypes.c_void_p(sigma_min.data_ptr()), len(W), shape[0], shape[1],
+                                        _dtype_code(W[0]), int(iters), _stream_handle(stream))
+        self._check(st, "muon_min_singular")
 
     def step_capped(self, W, G, M, u, v, alpha, stream=None, **hp):
         """step() with the update's component along u[l] v[l]^T removed; alpha[l] receives u^T O v."""

@@ -81,6 +81,8 @@ cudaError_t launch_gemv_rows(const GemvParams& p, int batch, bool f32, cudaStrea
 cudaError_t launch_gemv_cols(const GemvParams& p, int batch, bool f32, cudaStream_t s);
 cudaError_t launch_normalize(float* const* vecs_dev, int batch, int n, float* norm, cudaStream_t s);
 cudaError_t launch_cap_alpha(const CapParams& p, int batch, float* alpha, cudaStream_t s);
+cudaError_t launch_shift_normalize(float* const* y, const float* const* z, int batch, int n, const float* sigma_max,
+                                   cudaStream_t s);
 
 // ------------------------------------------------------------------ GEMM
 // The epilogue forms  v = alpha * s_l * acc + beta * cin + (row == col ? diag : 0)

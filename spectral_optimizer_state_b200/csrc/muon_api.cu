@@ -859,6 +859,66 @@ muon_status muon_power_iteration(muon_ctx* c, const void* const* W, float* const
   return MUON_OK;
 }
 
+muon_status muon_min_singular(muon_ctx* c, const void* const* W, float* const* y, const float* sigma_max,
+                              float* sigma_min, int batch, int rows, int cols, int dtype, int iters, void* stream) {
+  if (!c || !W || !y || !sigma_max || !sigma_min || batch < 1 || batch > MUON_MAX_BATCH || iters < 0 ||
+      iters > 100000)
+    return MUON_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 1) return MUON_ERR_INVALID_ARG;
+  if (rows > 32768 || cols > 32768) return MUON_ERR_UNSUPPORTED_SHAPE;
+  if (dtype != MUON_BF16 && dtype != MUON_F32) return MUON_ERR_DTYPE;
+  for (int l = 0; l < batch; ++l)
+    if (!W[l] || !y[l]) return MUON_ERR_INVALID_ARG;
+  DeviceGuard guard(c->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool tall = rows > cols;
+  const int m = tall ? cols : rows, n = tall ? rows : cols;  // wide view X is m x n
+  GemvParams gp;
+  std::memset(static_cast<void*>(&gp), 0, sizeof(gp));
+  gp.rows = rows;
+  gp.cols = cols;
+  gp.rows_per_chunk = 64;
+  gp.row_chunks = (rows + 63) / 64;
+  const size_t part_bytes = align_up(sizeof(float) * batch * gp.row_chunks * cols, 256);
+  const size_t w_bytes = align_up(sizeof(float) * n, 256), z_bytes = align_up(sizeof(float) * m, 256);
+  muon_status st = ensure_aux(c, part_bytes + batch * (w_bytes + z_bytes));
+  if (st != MUON_OK) return st;
+  char* base = static_cast<char*>(c->d_aux);
+  gp.partial = reinterpret_cast<float*>(base);
+  float* wv[MUON_MAX_BATCH];
+  float* zv[MUON_MAX_BATCH];
+  for (int l = 0; l < batch; ++l) {
+    gp.w[l] = W[l];
+    wv[l] = reinterpret_cast<float*>(base + part_bytes + l * w_bytes);
+    zv[l] = reinterpret_cast<float*>(base + part_bytes + batch * w_bytes + l * z_bytes);
+  }
+  const bool f32 = dtype == MUON_F32;
+  // out <- X^T in (length n) and out <- X in (length m), X the wide view of W
+  auto apply_xt = [&](float* const* in, float* const* out) {
+    for (int l = 0; l < batch; ++l) {
+      gp.x[l] = in[l];
+      gp.y[l] = out[l];
+    }
+    return tall ? launch_gemv_rows(gp, batch, f32, s) : launch_gemv_cols(gp, batch, f32, s);
+  };
+  auto apply_x = [&](float* const* in, float* const* out) {
+    for (int l = 0; l < batch; ++l) {
+      gp.x[l] = in[l];
+      gp.y[l] = out[l];
+    }
+    return tall ? launch_gemv_cols(gp, batch, f32, s) : launch_gemv_rows(gp, batch, f32, s);
+  };
+  MUON_CUDA(launch_normalize(y, batch, m, nullptr, s), "normalise start vector");
+  for (int i = 0; i < iters; ++i) {
+    MUON_CUDA(apply_xt(y, wv), "X^T y");
+    MUON_CUDA(apply_x(wv, zv), "X X^T y");
+    MUON_CUDA(launch_shift_normalize(y, zv, batch, m, sigma_max, s), "shifted step");
+  }
+  MUON_CUDA(apply_xt(y, wv), "X^T y");
+  MUON_CUDA(launch_normalize(wv, batch, n, sigma_min, s), "Rayleigh estimate");
+  return MUON_OK;
+}
+
 muon_status muon_step_capped(muon_ctx* c, void* const* W, const void* const* G, float* const* M,
                              const float* const* u, const float* const* v, int batch, int rows, int cols,
                              int dtype, const muon_hparams* hp, float* alpha, void* stream) {

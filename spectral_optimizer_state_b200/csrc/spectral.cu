@@ -161,6 +161,37 @@ __global__ void __launch_bounds__(kThreads) normalize_kernel(const __grid_consta
   for (int i = threadIdx.x; i < n; i += kThreads) v[i] *= inv;
 }
 
+struct ShiftParams {
+  float* y[MUON_MAX_BATCH];
+  const float* z[MUON_MAX_BATCH];
+  const float* sigma_max;  // [batch]: the shift is sigma_max^2
+  int n;
+};
+
+// y <- (s y - z) / |s y - z| per matrix (left as is when that is zero).
+__global__ void __launch_bounds__(kThreads) shift_normalize_kernel(const __grid_constant__ ShiftParams p) {
+  __shared__ double scratch[kThreads / 32];
+  __shared__ float inv;
+  const int l = blockIdx.x;
+  float* y = p.y[l];
+  const float* z = p.z[l];
+  const float sm = p.sigma_max[l];
+  const float s = sm * sm;
+  double ss = 0.0;
+  for (int i = threadIdx.x; i < p.n; i += kThreads) {
+    const float t = fmaf(s, y[i], -z[i]);
+    y[i] = t;
+    ss += static_cast<double>(t) * t;
+  }
+  const double tot = block_sum<double>(ss, scratch);
+  if (threadIdx.x == 0) {
+    const float nrm = static_cast<float>(sqrt(tot));
+    inv = nrm > 0.f ? 1.0f / nrm : 0.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < p.n; i += kThreads) y[i] *= inv;
+}
+
 // alpha partials: wide O (m x n, planes summed) against a (length m) and b (length n).
 __global__ void __launch_bounds__(kThreads) cap_alpha_partial_kernel(const __grid_constant__ CapParams p) {
   __shared__ double scratch[kThreads / 32];
@@ -243,6 +274,19 @@ cudaError_t launch_normalize(float* const* vecs, int batch, int n, float* norm, 
   p.n = n;
   p.norm = norm;
   normalize_kernel<<<batch, kThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_shift_normalize(float* const* y, const float* const* z, int batch, int n, const float* sigma_max,
+                                   cudaStream_t s) {
+  ShiftParams p;
+  for (int l = 0; l < batch; ++l) {
+    p.y[l] = y[l];
+    p.z[l] = z[l];
+  }
+  p.sigma_max = sigma_max;
+  p.n = n;
+  shift_normalize_kernel<<<batch, kThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 

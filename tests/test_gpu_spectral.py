@@ -149,3 +149,45 @@ def test_step_capped_rejects_missing_vectors():
     with Muon() as muon:
         with pytest.raises((MuonError, ValueError)):
             muon.step_capped(W, W, [w.clone() for w in W], [], [], torch.zeros(1, device="cuda"))
+
+
+def _min_singular(muon, Ws, y0s, smax, iters, dtype):
+    import torch
+    W = [to_device(w, dtype) for w in Ws]
+    y = [torch.from_numpy(y0.astype(np.float32)).cuda() for y0 in y0s]
+    sm = torch.from_numpy(np.asarray(smax, np.float32)).cuda()
+    out = torch.zeros(len(Ws), dtype=torch.float32, device="cuda")
+    muon.min_singular(W, y, sm, out, iters=iters)
+    torch.cuda.synchronize()
+    return [to_numpy(t) for t in y], to_numpy(out)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("rows,cols,batch", SHAPES)
+@pytest.mark.parametrize("iters", [0, 20])
+def test_min_singular_matches_oracle(rows, cols, batch, dtype, iters):
+    from spectral_optimizer_state_b200 import Muon
+    Ws = [weights(rng_for(75, l), rows, cols) for l in range(batch)]
+    Ws = [round_bf16(w) if dtype == "bf16" else w.astype(np.float32) for w in Ws]
+    m = min(rows, cols)
+    y0s = [rng_for(76, l).standard_normal(m).astype(np.float32) for l in range(batch)]
+    smax = [np.linalg.svd(w.astype(np.float64), compute_uv=False)[0] for w in Ws]
+    smax = [float(np.float32(s)) for s in smax]  # the fp32 value the kernel receives
+    with Muon() as muon:
+        y, smin = _min_singular(muon, Ws, y0s, smax, iters, dtype)
+    for l in range(batch):
+        ry, rs = oracle.min_singular_shifted(Ws[l].astype(np.float64), y0s[l].astype(np.float64), smax[l], iters)
+        # fp32 products against fp64: a float32 replay of the same iteration stays within 1e-6
+        assert abs(smin[l] - rs) <= 1e-4 * rs
+        assert rel_f(y[l], ry) <= 1e-4
+        assert smin[l] >= np.linalg.svd(Ws[l].astype(np.float64), compute_uv=False)[-1] * (1 - 1e-4)
+
+
+def test_min_singular_of_semi_orthogonal_is_one():
+    from spectral_optimizer_state_b200 import Muon
+    Q, _ = np.linalg.qr(rng_for(77, 0).standard_normal((300, 128)))
+    Ws = [Q.astype(np.float32), np.ascontiguousarray(Q.T).astype(np.float32)]
+    with Muon() as muon:
+        _, smin_tall = _min_singular(muon, Ws[:1], [np.ones(128, np.float32)], [1.0], 5, "f32")
+        _, smin_wide = _min_singular(muon, Ws[1:], [np.ones(128, np.float32)], [1.0], 5, "f32")
+    assert abs(smin_tall[0] - 1.0) <= 1e-5 and abs(smin_wide[0] - 1.0) <= 1e-5
