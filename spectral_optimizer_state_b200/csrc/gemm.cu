@@ -128,11 +128,6 @@ __device__ __forceinline__ void unpack_bf16x8(uint4 q, float* v) {
   }
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-  return static_cast<uint32_t>(float_to_bf16_bits(a)) |
-         (static_cast<uint32_t>(float_to_bf16_bits(b)) << 16);
-}
-
 // v[t] += beta * sum_p cin_p(row, j0 + t) for t < nv (caller guarantees row < M, j0 < N)
 __device__ __forceinline__ void add_cin(const GemmProblem& q, int l, int row, int j0, int nv,
                                         float (&v)[32]) {
@@ -672,7 +667,7 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_c
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(map_shared_rank(tempty_bar(acc), 0));
+      if (lane == 0) mbar_arrive_remote(map_shared_rank(tempty_bar(acc), 0));
     }
     if (lane == 0) bulk_wait_group_all();
   }

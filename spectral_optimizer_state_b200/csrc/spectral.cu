@@ -15,6 +15,8 @@
 // deterministic.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "device_utils.cuh"
 #include "internal.h"
 
@@ -46,9 +48,10 @@ __device__ __forceinline__ float load1(const void* base, long long e) {
   return F32 ? static_cast<const float*>(base)[e] : bf16_bits_to_float(static_cast<const uint16_t*>(base)[e]);
 }
 
-// y[r] = sum_c W[r][c] x[c]; one warp per row, x staged in shared memory.
+// y[r] = sum_c W[r][c] x[c]; each warp takes rows_per_warp consecutive rows, x staged in shared memory
+// once per block.
 template <bool F32, bool VEC>
-__global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_constant__ GemvParams p) {
+__global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_constant__ GemvParams p, int rows_per_warp) {
   extern __shared__ float xs[];
   const int l = blockIdx.y;
   const float* x = p.x[l];
@@ -56,23 +59,26 @@ __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_consta
   __syncthreads();
   const void* W = p.w[l];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * (kThreads / 32) + warp;
-  if (r >= p.rows) return;
-  const long long row = static_cast<long long>(r) * p.cols;
-  float acc = 0.f;
-  if (VEC) {
-    for (int c = lane * 8; c < p.cols; c += 32 * 8) {
-      float w[8];
-      load8<F32>(W, row + c, w);
+  const int r0 = (blockIdx.x * (kThreads / 32) + warp) * rows_per_warp;
+  const int r1 = min(p.rows, r0 + rows_per_warp);
+  for (int r = r0; r < r1; ++r) {
+    const long long row = static_cast<long long>(r) * p.cols;
+    float acc = 0.f;
+    if (VEC) {
+#pragma unroll 2
+      for (int c = lane * 8; c < p.cols; c += 32 * 8) {
+        float w[8];
+        load8<F32>(W, row + c, w);
 #pragma unroll
-      for (int t = 0; t < 8; ++t) acc = fmaf(w[t], xs[c + t], acc);
+        for (int t = 0; t < 8; ++t) acc = fmaf(w[t], xs[c + t], acc);
+      }
+    } else {
+      for (int c = lane; c < p.cols; c += 32) acc = fmaf(load1<F32>(W, row + c), xs[c], acc);
     }
-  } else {
-    for (int c = lane; c < p.cols; c += 32) acc = fmaf(load1<F32>(W, row + c), xs[c], acc);
-  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (lane == 0) p.y[l][r] = acc;
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) p.y[l][r] = acc;
+  }
 }
 
 // partial[l][chunk][c] = sum over the chunk's rows of W[r][c] y[r]; thread owns 8 columns (VEC) or 1.
@@ -82,11 +88,12 @@ __global__ void __launch_bounds__(kThreads) gemv_cols_partial_kernel(const __gri
   const void* W = p.w[l];
   const float* y = p.x[l];
   const int per = VEC ? 8 : 1;
-  const int c0 = (blockIdx.x * kThreads + threadIdx.x) * per;
+  const int c0 = (blockIdx.x * blockDim.x + threadIdx.x) * per;
   if (c0 >= p.cols) return;
   const int r0 = blockIdx.y * p.rows_per_chunk;
   const int r1 = min(p.rows, r0 + p.rows_per_chunk);
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll 4
   for (int r = r0; r < r1; ++r) {
     const float yr = y[r];
     const long long e = static_cast<long long>(r) * p.cols + c0;
@@ -193,26 +200,47 @@ __global__ void __launch_bounds__(kThreads) shift_normalize_kernel(const __grid_
 }
 
 // alpha partials: wide O (m x n, planes summed) against a (length m) and b (length n).
+// One warp per row of O (rows_per_block == warps per block); each lane reads
+// 16-byte vectors of every plane (the wide pitch is a multiple of 64 elements,
+// so row starts are 128-byte aligned) and the ragged tail element by element.
 __global__ void __launch_bounds__(kThreads) cap_alpha_partial_kernel(const __grid_constant__ CapParams p) {
   __shared__ double scratch[kThreads / 32];
   const int l = blockIdx.y;
   const float* a = p.a[l];
   const float* b = p.b[l];
   const uint16_t* o = p.o + static_cast<long long>(l) * p.o_mat;
-  const int i0 = blockIdx.x * p.rows_per_block;
-  const int i1 = min(p.m, i0 + p.rows_per_block);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * (kThreads / 32) + warp;
   double acc = 0.0;
-  for (int i = i0; i < i1; ++i) {
+  if (i < p.m) {
+    const uint16_t* row = o + static_cast<long long>(i) * p.pitch;
+    const int nv = p.n & ~7;
     float s = 0.f;
-    for (int j = threadIdx.x; j < p.n; j += kThreads) {
+    for (int j = lane * 8; j < nv; j += 32 * 8) {
+      float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int q = 0; q < p.planes; ++q) {
+        const uint4 w = __ldcs(reinterpret_cast<const uint4*>(row + q * p.o_plane + j));
+        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          v[2 * t] += __uint_as_float(u[t] << 16);
+          v[2 * t + 1] += __uint_as_float(u[t] & 0xFFFF0000u);
+        }
+      }
+      // b is the caller's vector with no alignment promise: scalar reads (it stays in L1)
+#pragma unroll
+      for (int t = 0; t < 8; ++t) s = fmaf(v[t], __ldg(b + j + t), s);
+    }
+    for (int j = nv + lane; j < p.n; j += 32) {
       float v = 0.f;
-      for (int q = 0; q < p.planes; ++q)
-        v += bf16_bits_to_float(o[q * p.o_plane + static_cast<long long>(i) * p.pitch + j]);
+      for (int q = 0; q < p.planes; ++q) v += bf16_bits_to_float(row[q * p.o_plane + j]);
       s = fmaf(v, b[j], s);
     }
-    acc += static_cast<double>(s) * a[i];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    acc = static_cast<double>(s) * a[i];
   }
-  const double tot = block_sum<double>(acc, scratch);
+  const double tot = block_sum<double>(lane == 0 ? acc : 0.0, scratch);
   if (threadIdx.x == 0) p.partial[static_cast<long long>(l) * gridDim.x + blockIdx.x] = tot;
 }
 
@@ -226,7 +254,11 @@ __global__ void cap_alpha_reduce_kernel(const double* partial, int nblk, float* 
 }  // namespace
 
 cudaError_t launch_gemv_rows(const GemvParams& p, int batch, bool f32, cudaStream_t s) {
-  const dim3 grid((p.rows + kThreads / 32 - 1) / (kThreads / 32), batch);
+  constexpr int kWarps = kThreads / 32;
+  // rows per warp: up to 4 (fewer shared-memory fills of x) while keeping >= 4 blocks per SM
+  const long long total_rows = static_cast<long long>(p.rows) * batch;
+  const int rpw = static_cast<int>(std::max(1LL, std::min(4LL, total_rows / (kWarps * 148LL * 4))));
+  const dim3 grid((p.rows + kWarps * rpw - 1) / (kWarps * rpw), batch);
   const size_t smem = sizeof(float) * p.cols;  // up to 128 KB (cols <= 32768)
   // the attribute is per device: set it on every launch that needs more than the default 48 KB
   if (smem > 48 * 1024) {
@@ -240,11 +272,11 @@ cudaError_t launch_gemv_rows(const GemvParams& p, int batch, bool f32, cudaStrea
   for (int l = 0; l < batch && vec; ++l)
     if (reinterpret_cast<uintptr_t>(p.w[l]) % 16) vec = false;
   if (f32) {
-    if (vec) gemv_rows_kernel<true, true><<<grid, kThreads, smem, s>>>(p);
-    else gemv_rows_kernel<true, false><<<grid, kThreads, smem, s>>>(p);
+    if (vec) gemv_rows_kernel<true, true><<<grid, kThreads, smem, s>>>(p, rpw);
+    else gemv_rows_kernel<true, false><<<grid, kThreads, smem, s>>>(p, rpw);
   } else {
-    if (vec) gemv_rows_kernel<false, true><<<grid, kThreads, smem, s>>>(p);
-    else gemv_rows_kernel<false, false><<<grid, kThreads, smem, s>>>(p);
+    if (vec) gemv_rows_kernel<false, true><<<grid, kThreads, smem, s>>>(p, rpw);
+    else gemv_rows_kernel<false, false><<<grid, kThreads, smem, s>>>(p, rpw);
   }
   return cudaGetLastError();
 }
@@ -254,13 +286,17 @@ cudaError_t launch_gemv_cols(const GemvParams& p, int batch, bool f32, cudaStrea
   for (int l = 0; l < batch && vec; ++l)
     if (reinterpret_cast<uintptr_t>(p.w[l]) % 16) vec = false;
   const int per = vec ? 8 : 1;
-  const dim3 grid((p.cols + kThreads * per - 1) / (kThreads * per), p.row_chunks, batch);
+  // a block spans the columns (up to kThreads threads of `per` columns each): narrow matrices do
+  // not leave most of a 256-thread block idle
+  const int need = (p.cols + per - 1) / per;
+  const int threads = std::min(kThreads, std::max(32, (need + 31) / 32 * 32));
+  const dim3 grid((need + threads - 1) / threads, p.row_chunks, batch);
   if (f32) {
-    if (vec) gemv_cols_partial_kernel<true, true><<<grid, kThreads, 0, s>>>(p);
-    else gemv_cols_partial_kernel<true, false><<<grid, kThreads, 0, s>>>(p);
+    if (vec) gemv_cols_partial_kernel<true, true><<<grid, threads, 0, s>>>(p);
+    else gemv_cols_partial_kernel<true, false><<<grid, threads, 0, s>>>(p);
   } else {
-    if (vec) gemv_cols_partial_kernel<false, true><<<grid, kThreads, 0, s>>>(p);
-    else gemv_cols_partial_kernel<false, false><<<grid, kThreads, 0, s>>>(p);
+    if (vec) gemv_cols_partial_kernel<false, true><<<grid, threads, 0, s>>>(p);
+    else gemv_cols_partial_kernel<false, false><<<grid, threads, 0, s>>>(p);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -291,6 +327,8 @@ cudaError_t launch_shift_normalize(float* const* y, const float* const* z, int b
 }
 
 cudaError_t launch_cap_alpha(const CapParams& p, int batch, float* alpha, cudaStream_t s) {
+  // one warp per row: p.rows_per_block must equal the warps of a block
+  if (p.rows_per_block != kThreads / 32) return cudaErrorInvalidValue;
   const int nblk = (p.m + p.rows_per_block - 1) / p.rows_per_block;
   cap_alpha_partial_kernel<<<dim3(nblk, batch), kThreads, 0, s>>>(p);
   cudaError_t e = cudaGetLastError();
