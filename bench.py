@@ -480,22 +480,23 @@ def main():
     # AdamW over the parameters Muon does not take (the rest of Mamba-2 130M)
     adamw = None
     if args.workload == "mamba2-130m":
-        from spectral_optimizer_state_b200 import adamw_step
+        from spectral_optimizer_state_b200 import AdamWGroup
         from synthetic import mamba2_130m_other_params
         others = mamba2_130m_other_params()
         aw = [torch.randn(int(np.prod(sh)), device=device).to(torch.bfloat16) * 0.02 for _, sh in others]
         ag = [torch.randn(w.numel(), device=device).to(torch.bfloat16) for w in aw]
         am = [torch.zeros(w.numel(), device=device) for w in aw]
         av = [torch.zeros(w.numel(), device=device) for w in aw]
+        adam = AdamWGroup(aw, ag, am, av)  # checked and marshalled once, like an optimizer holding its state
         for i in range(3):
-            adamw_step(aw, ag, am, av, i + 1)
+            adam.step(i + 1, stream=stream)
         torch.cuda.synchronize()
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
         reps = 20
         a0.record(stream)
         for i in range(reps):
-            adamw_step(aw, ag, am, av, i + 4)
+            adam.step(i + 4, stream=stream)
         a1.record(stream)
         torch.cuda.synchronize()
         a_ms = a0.elapsed_time(a1) / reps
@@ -503,7 +504,8 @@ def main():
         gbs = 22 * numel / (a_ms / 1e3) / 1e9
         adamw = {"bound": "hbm", "params": numel, "ms_per_step": a_ms, "achieved_gbs": gbs,
                  "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"], "bytes_per_element": 22,
-                 "tensors": len(aw), "note": "AdamW over the non-Muon parameters of Mamba-2 130M, bf16"}
+                 "tensors": len(aw), "launches_per_step": len(adam._calls),
+                 "note": "AdamW over the non-Muon parameters of Mamba-2 130M, bf16 (AdamWGroup)"}
         del aw, ag, am, av
 
     spectral = measure_spectral(mu, Ws, Gsets[0], Ms, groups, stream, peaks) if args.spectral else None

@@ -379,10 +379,8 @@ def momentum_norm_noalloc(G, M, nu, beta=0.95, nesterov=True, stream=None):
         raise MuonError(st, "muon_momentum_norm_noalloc")
 
 
-def adamw_step(W, G, m, v, step, lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, stream=None):
-    """AdamW on tensors of any shapes (one dtype, bf16 or fp32; fp32 moments), one launch per 256 tensors."""
+def _check_adamw(W, G, m, v):
     import torch
-    lib = load_library()
     if not (len(W) == len(G) == len(m) == len(v)) or len(W) == 0:
         raise ValueError("W, G, m and v must be non-empty lists of equal length")
     dt = W[0].dtype
@@ -395,15 +393,39 @@ def adamw_step(W, G, m, v, step, lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8, weigh
             raise ValueError("tensors must be contiguous")
         if not (w.numel() == g.numel() == a.numel() == b.numel()):
             raise ValueError("W, G, m and v must match in size")
-    hp = AdamWHparams(float(lr), float(beta1), float(beta2), float(eps), float(weight_decay), int(step))
-    for c0 in range(0, len(W), MAX_BATCH):
-        sl = slice(c0, c0 + MAX_BATCH)
-        ws, gs, ms, vs = W[sl], G[sl], m[sl], v[sl]
-        numel = (ctypes.c_longlong * len(ws))(*[t.numel() for t in ws])
-        st = lib.muon_adamw_step(_ptrs(ws), _ptrs(gs), _ptrs(ms), _ptrs(vs), numel, len(ws), _dtype_code(ws[0]),
-                                 ctypes.byref(hp), _stream_handle(stream))
-        if st != MUON_OK:
-            raise MuonError(st, "muon_adamw_step")
+
+
+class AdamWGroup:
+    """AdamW over a fixed list of tensors: validated and marshalled once, so a step costs
+    one C call per MAX_BATCH tensors (the tensors must stay alive and in place)."""
+
+    def __init__(self, W, G, m, v):
+        _check_adamw(W, G, m, v)
+        self.lib = load_library()
+        self._tensors = (list(W), list(G), list(m), list(v))  # keep the storage alive
+        self._calls = []
+        for c0 in range(0, len(W), MAX_BATCH):
+            sl = slice(c0, c0 + MAX_BATCH)
+            ws = W[sl]
+            numel = (ctypes.c_longlong * len(ws))(*[t.numel() for t in ws])
+            self._calls.append((_ptrs(ws), _ptrs(G[sl]), _ptrs(m[sl]), _ptrs(v[sl]), numel, len(ws),
+                                _dtype_code(ws[0])))
+
+    def step(self, step, lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, stream=None):
+        hp = AdamWHparams(float(lr), float(beta1), float(beta2), float(eps), float(weight_decay), int(step))
+        sh = _stream_handle(stream)
+        for pw, pg, pm, pv, numel, n, dt in self._calls:
+            st = self.lib.muon_adamw_step(pw, pg, pm, pv, numel, n, dt, ctypes.byref(hp), sh)
+            if st != MUON_OK:
+                raise MuonError(st, "muon_adamw_step")
+
+
+def adamw_step(W, G, m, v, step, lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, stream=None):
+    """AdamW on tensors of any shapes (one dtype, bf16 or fp32; fp32 moments), one launch per
+    MAX_BATCH tensors.  For a fixed set of tensors stepped repeatedly, AdamWGroup does the
+    checks once."""
+    AdamWGroup(W, G, m, v).step(step, lr=lr, beta1=beta1, beta2=beta2, eps=eps, weight_decay=weight_decay,
+                                stream=stream)
 
 
 def shape_scale(rows: int, cols: int, mode: int = SCALE_SQRT_RATIO) -> float:

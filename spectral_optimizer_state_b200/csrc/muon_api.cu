@@ -133,6 +133,15 @@ struct muon_ctx {
   float* d_partials = nullptr;
   int* d_status = nullptr;
   unsigned* d_done = nullptr;  // [kMaxProblems][MUON_MAX_BATCH] phase-completion counters
+  // MUON_OVERLAP=1: momentum passes of later groups and applies of earlier groups run on a side
+  // stream beside the Newton-Schulz launches of other groups.  Off by default: on B200 the
+  // co-running elementwise passes slow the GEMM by as much time as they hide (both draw on the
+  // same L2 -> SM bandwidth), and one persistent launch for all groups has no gap between them.
+  bool overlap = false;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  cudaEvent_t ev_k1[MUON_MAX_GROUPS] = {};
+  cudaEvent_t ev_gemm[MUON_MAX_GROUPS] = {};
   int gemm_kind = GEMM_SINGLE;  // MUON_GEMM=pair selects the CTA-pair kernel
   bool per_phase = false;       // MUON_LAUNCH=phase: one launch per phase (same work; per-phase timing)
   int last_count = 0;
@@ -398,8 +407,8 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
   for (auto& p : plans) total += p.batch;
   MUON_CUDA(cudaMemsetAsync(c->d_status, 0, sizeof(int), s), "clear status");
 
-  // K1: momentum / look-ahead / norm, one launch per group.
-  for (auto& p : plans) {
+  // K1: momentum / look-ahead / norm of one group.
+  auto k1 = [&](const GroupPlan& p, cudaStream_t strm) -> muon_status {
     MomentumParams mp;
     std::memset(static_cast<void*>(&mp), 0, sizeof(mp));
     for (int l = 0; l < p.batch; ++l) {
@@ -422,11 +431,11 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
     mp.scale1 = c->d_s1 + p.mat_off;
     mp.scale2 = c->d_s2 + p.mat_off;
     mp.flags = c->d_flags + p.mat_off;
-    const int slot = prof_begin(c, MUON_KERNEL_MOMENTUM, s);
-    MUON_CUDA(launch_momentum(mp, p.batch, p.f32 != 0, step, p.planes, s), "momentum kernel");
-    prof_end(c, slot, s);
-  }
-
+    const int slot = prof_begin(c, MUON_KERNEL_MOMENTUM, strm);
+    MUON_CUDA(launch_momentum(mp, p.batch, p.f32 != 0, step, p.planes, strm), "momentum kernel");
+    prof_end(c, slot, strm);
+    return MUON_OK;
+  };
   // k Newton-Schulz iterations.  The single-CTA kernel runs every phase of
   // every group in one persistent launch (as many as fit in one parameter
   // block), ordered phase by phase; per-(phase, matrix) counters let a tile
@@ -455,7 +464,24 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
   // kernel runs one launch per phase covering every group.
   struct Item { int g, pi; };
   std::vector<std::vector<Item>> launches;
-  if (persistent) {
+  // Pipelined schedule (two or more groups, persistent kernel): one launch per group on the
+  // caller's stream; the momentum pass of group g+1 and the apply of group g run on the side
+  // stream beside them.  Groups whose momentum pass is transposed (tall W, shared-memory
+  // tiles that cannot sit beside a GEMM CTA) go first, so the passes that overlap are the
+  // ones that fit.
+  const bool pipelined = c->overlap && persistent && ng >= 2 && cap == nullptr && c->side != nullptr;
+  std::vector<int> order;
+  for (int g = 0; g < ng; ++g)
+    if (plans[g].transposed) order.push_back(g);
+  for (int g = 0; g < ng; ++g)
+    if (!plans[g].transposed) order.push_back(g);
+  if (pipelined) {
+    for (int g : order) {
+      std::vector<Item> cur;
+      for (int pi = 0; pi < nph; ++pi) cur.push_back({g, pi});
+      launches.push_back(cur);
+    }
+  } else if (persistent) {
     std::vector<Item> cur;
     for (int g = 0; g < ng; ++g) {
       for (int pi = 0; pi < nph; ++pi) {
@@ -475,7 +501,7 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
     }
   }
   GemmParams gp;
-  for (const auto& items : launches) {
+  auto run_launch = [&](const std::vector<Item>& items, cudaStream_t strm) -> muon_status {
     std::memset(static_cast<void*>(&gp), 0, sizeof(gp));
     gp.status = c->d_status;
     int tiles = 0;
@@ -500,42 +526,19 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
     }
     gp.total_tiles = tiles;
     if (persistent)
-      MUON_CUDA(cudaMemsetAsync(c->d_done, 0, sizeof(unsigned) * gp.nprob * MUON_MAX_BATCH, s), "clear counters");
+      MUON_CUDA(cudaMemsetAsync(c->d_done, 0, sizeof(unsigned) * gp.nprob * MUON_MAX_BATCH, strm), "clear counters");
     const int units = std::min(tiles, pair ? c->sm_count / 2 : c->sm_count);
     const int kind = items.size() > static_cast<size_t>(ng) || persistent
                          ? MUON_KERNEL_NS_FUSED
                          : MUON_KERNEL_GRAM + (seq_ph[items[0].pi] - PH_GRAM);
-    const int slot = prof_begin(c, kind, s);
-    MUON_CUDA(launch_gemm(gp, c->gemm_kind, units, s), "newton-schulz gemm");
-    prof_end(c, slot, s);
-  }
+    const int slot = prof_begin(c, kind, strm);
+    MUON_CUDA(launch_gemm(gp, c->gemm_kind, units, strm), "newton-schulz gemm");
+    prof_end(c, slot, strm);
+    return MUON_OK;
+  };
 
-  // Spectral cap: alpha_l = u_l^T O_l v_l from the final iterate (one group).
-  if (cap != nullptr) {
-    const GroupPlan& p = plans[0];
-    CapParams cp;
-    std::memset(static_cast<void*>(&cp), 0, sizeof(cp));
-    for (int l = 0; l < p.batch; ++l) {
-      cp.a[l] = p.transposed ? cap->v[l] : cap->u[l];  // wide rows are W's columns when tall
-      cp.b[l] = p.transposed ? cap->u[l] : cap->v[l];
-    }
-    cp.o = ws_at(c, p.off_x[c->k & 1]);
-    cp.o_plane = p.x_plane;
-    cp.o_mat = p.x_mat;
-    cp.pitch = p.pitch_n;
-    cp.m = p.m_rows;
-    cp.n = p.n_cols;
-    cp.planes = p.planes;
-    cp.rows_per_block = 8;
-    const size_t need = sizeof(double) * p.batch * ((p.m_rows + 7) / 8);
-    st = ensure_aux(c, need);
-    if (st != MUON_OK) return st;
-    cp.partial = static_cast<double*>(c->d_aux);
-    MUON_CUDA(launch_cap_alpha(cp, p.batch, cap->alpha, s), "cap coefficient");
-  }
-
-  // K5: scale + decoupled decay applied to W (or the plain copy to Out).
-  for (auto& p : plans) {
+  // K5: scale + decoupled decay applied to W (or the plain copy to Out) for one group.
+  auto k5 = [&](const GroupPlan& p, cudaStream_t strm) -> muon_status {
     ApplyParams ap;
     std::memset(static_cast<void*>(&ap), 0, sizeof(ap));
     for (int l = 0; l < p.batch; ++l) ap.w[l] = p.w[l];
@@ -560,9 +563,75 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
       }
       ap.alpha = cap->alpha;
     }
-    const int slot = prof_begin(c, MUON_KERNEL_APPLY, s);
-    MUON_CUDA(launch_apply(ap, p.batch, p.f32 != 0, s), "apply kernel");
-    prof_end(c, slot, s);
+    const int slot = prof_begin(c, MUON_KERNEL_APPLY, strm);
+    MUON_CUDA(launch_apply(ap, p.batch, p.f32 != 0, strm), "apply kernel");
+    prof_end(c, slot, strm);
+    return MUON_OK;
+  };
+
+  if (pipelined) {
+    // caller's stream: K1(first), GEMM(first), GEMM(second) ..., K5(last)
+    // side stream:     K1(second) ..., K5(first) ...
+    st = k1(plans[order[0]], s);
+    if (st != MUON_OK) return st;
+    MUON_CUDA(cudaEventRecord(c->ev_fork, s), "fork");
+    MUON_CUDA(cudaStreamWaitEvent(c->side, c->ev_fork, 0), "fork");
+    for (int i = 1; i < ng; ++i) {
+      st = k1(plans[order[i]], c->side);
+      if (st != MUON_OK) return st;
+      MUON_CUDA(cudaEventRecord(c->ev_k1[i], c->side), "momentum done");
+    }
+    for (int i = 0; i < ng; ++i) {
+      if (i > 0) MUON_CUDA(cudaStreamWaitEvent(s, c->ev_k1[i], 0), "wait momentum");
+      st = run_launch(launches[i], s);
+      if (st != MUON_OK) return st;
+      if (i + 1 < ng) {
+        MUON_CUDA(cudaEventRecord(c->ev_gemm[i], s), "gemm done");
+        MUON_CUDA(cudaStreamWaitEvent(c->side, c->ev_gemm[i], 0), "wait gemm");
+        st = k5(plans[order[i]], c->side);
+        if (st != MUON_OK) return st;
+      }
+    }
+    st = k5(plans[order[ng - 1]], s);
+    if (st != MUON_OK) return st;
+    MUON_CUDA(cudaEventRecord(c->ev_join, c->side), "join");
+    MUON_CUDA(cudaStreamWaitEvent(s, c->ev_join, 0), "join");
+  } else {
+    for (auto& p : plans) {
+      st = k1(p, s);
+      if (st != MUON_OK) return st;
+    }
+    for (const auto& items : launches) {
+      st = run_launch(items, s);
+      if (st != MUON_OK) return st;
+    }
+    // Spectral cap: alpha_l = u_l^T O_l v_l from the final iterate (one group).
+    if (cap != nullptr) {
+      const GroupPlan& p = plans[0];
+      CapParams cp;
+      std::memset(static_cast<void*>(&cp), 0, sizeof(cp));
+      for (int l = 0; l < p.batch; ++l) {
+        cp.a[l] = p.transposed ? cap->v[l] : cap->u[l];  // wide rows are W's columns when tall
+        cp.b[l] = p.transposed ? cap->u[l] : cap->v[l];
+      }
+      cp.o = ws_at(c, p.off_x[c->k & 1]);
+      cp.o_plane = p.x_plane;
+      cp.o_mat = p.x_mat;
+      cp.pitch = p.pitch_n;
+      cp.m = p.m_rows;
+      cp.n = p.n_cols;
+      cp.planes = p.planes;
+      cp.rows_per_block = 8;
+      const size_t need = sizeof(double) * p.batch * ((p.m_rows + 7) / 8);
+      st = ensure_aux(c, need);
+      if (st != MUON_OK) return st;
+      cp.partial = static_cast<double*>(c->d_aux);
+      MUON_CUDA(launch_cap_alpha(cp, p.batch, cap->alpha, s), "cap coefficient");
+    }
+    for (auto& p : plans) {
+      st = k5(p, s);
+      if (st != MUON_OK) return st;
+    }
   }
   c->last_count = total;
   c->last_stream = s;
@@ -631,6 +700,24 @@ muon_status muon_create(muon_ctx** out, int device) {
   if (const char* l = std::getenv("MUON_LAUNCH")) {
     if (std::strcmp(l, "phase") == 0) c->per_phase = true;
   }
+  if (const char* o = std::getenv("MUON_OVERLAP")) {
+    if (std::strcmp(o, "1") == 0) c->overlap = true;
+  }
+  {
+    int least = 0, greatest = 0;
+    bool ok = cudaDeviceGetStreamPriorityRange(&least, &greatest) == cudaSuccess &&
+              cudaStreamCreateWithPriority(&c->side, cudaStreamNonBlocking, least) == cudaSuccess &&
+              cudaEventCreateWithFlags(&c->ev_fork, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&c->ev_join, cudaEventDisableTiming) == cudaSuccess;
+    for (int g = 0; ok && g < MUON_MAX_GROUPS; ++g)
+      ok = cudaEventCreateWithFlags(&c->ev_k1[g], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&c->ev_gemm[g], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      if (c->side) cudaStreamDestroy(c->side);
+      c->side = nullptr;  // everything runs on the caller's stream
+    }
+  }
   if (cudaMalloc(&c->d_status, sizeof(int)) != cudaSuccess) {
     cudaGetLastError();
     delete c;
@@ -663,6 +750,13 @@ muon_status muon_destroy(muon_ctx* c) {
   cudaFree(c->d_stage);
   cudaFree(c->d_aux);
   for (cudaEvent_t e : c->events) cudaEventDestroy(e);
+  for (int g = 0; g < MUON_MAX_GROUPS; ++g) {
+    if (c->ev_k1[g]) cudaEventDestroy(c->ev_k1[g]);
+    if (c->ev_gemm[g]) cudaEventDestroy(c->ev_gemm[g]);
+  }
+  if (c->ev_fork) cudaEventDestroy(c->ev_fork);
+  if (c->ev_join) cudaEventDestroy(c->ev_join);
+  if (c->side) cudaStreamDestroy(c->side);
   delete c;
   return MUON_OK;
 }

@@ -358,6 +358,35 @@ def test_single_cta_and_pair_kernels_agree():
             assert rel_f(a, b) <= 5e-3
 
 
+def test_two_stream_schedule_is_bitwise_equal_to_serial():
+    """The pipelined schedule (momentum and apply passes of other groups on a side stream)
+    computes exactly what the one-stream schedule computes, over three groups and two steps."""
+    import os
+    import torch
+    from spectral_optimizer_state_b200 import Muon
+    shapes = [(200, 328), (328, 200), (768, 1536)]
+    results = {}
+    for mode in ("1", "0"):
+        os.environ["MUON_OVERLAP"] = mode
+        try:
+            m = Muon(0)
+        finally:
+            del os.environ["MUON_OVERLAP"]
+        m.set_coeffs(QUINTIC5)
+        W = [[to_device(w, "bf16") for w in group_weights(7, i, 3, r, c)] for i, (r, c) in enumerate(shapes)]
+        M = [[torch.zeros((r, c), dtype=torch.float32, device="cuda") for _ in range(3)] for (r, c) in shapes]
+        for step in range(2):
+            G = [[to_device(g, "bf16") for g in _inputs(shape, 3, seed=710 + 10 * step + i, kind="spike")]
+                 for i, shape in enumerate(shapes)]
+            m.step_groups([(W[i], G[i], M[i]) for i in range(len(shapes))])
+        assert m.status()[0] == 0
+        results[mode] = ([to_numpy(w) for ws in W for w in ws], [to_numpy(x) for ms in M for x in ms], m.norms())
+        m.close()
+    for a, b in zip(results["1"][0] + results["1"][1], results["0"][0] + results["0"][1]):
+        assert np.array_equal(a, b)
+    assert results["1"][2] == results["0"][2]
+
+
 def test_scaled_2k_model_full_size_sampled():
     """Scaled Mamba-2-style model (d_model 2048): 48 x 8768 x 2048 + 48 x 2048 x 4096 bf16 in one
     call, the same launches bench.py times; one matrix per group checked against the oracle.
