@@ -95,8 +95,8 @@ __device__ __forceinline__ void rmw1(void* dst, long long e, float v, bool apply
   }
 }
 
-// Wide W (rows <= cols): W(i, j) with O(i, j).
-template <bool F32, bool VEC>
+// Wide W (rows <= cols): W(i, j) with O(i, j).  CAP: O - alpha u v^T (spectral cap).
+template <bool F32, bool VEC, bool CAP>
 __global__ void __launch_bounds__(kThreads) apply_wide_kernel(const __grid_constant__ ApplyParams p) {
   const int l = blockIdx.y;
   if (p.flags != nullptr && p.flags[l] != 0) return;
@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(kThreads) apply_wide_kernel(const __grid_const
       const int j = static_cast<int>(v - i * per_row) * 8;
       float ov[8];
       load8_planes(o + i * p.pitch + j, p.o_plane, p.planes, ov);
-      if (p.alpha != nullptr) {
+      if (CAP) {
         const float au = p.alpha[l] * p.cu[l][i];
 #pragma unroll
         for (int t = 0; t < 8; ++t) ov[t] = fmaf(-au, p.cv[l][j + t], ov[t]);
@@ -131,14 +131,14 @@ __global__ void __launch_bounds__(kThreads) apply_wide_kernel(const __grid_const
       const long long i = e / C;
       const int j = static_cast<int>(e - i * C);
       float ov = load1_planes(o + i * p.pitch + j, p.o_plane, p.planes);
-      if (p.alpha != nullptr) ov = fmaf(-p.alpha[l] * p.cu[l][i], p.cv[l][j], ov);
+      if (CAP) ov = fmaf(-p.alpha[l] * p.cu[l][i], p.cv[l][j], ov);
       rmw1<F32>(w, e, ov, p.apply, p.decay, p.lrs);
     }
   }
 }
 
 // Tall W (rows > cols): W(r, c) with O(c, r), through a 64 x 64 tile.
-template <bool F32, bool VEC>
+template <bool F32, bool VEC, bool CAP>
 __global__ void __launch_bounds__(kThreads) apply_tall_kernel(const __grid_constant__ ApplyParams p) {
   __shared__ float tile[64][65];
   const int l = blockIdx.y;
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kThreads) apply_tall_kernel(const __grid_const
         float ov[8];
 #pragma unroll
         for (int t = 0; t < 8; ++t) ov[t] = tile[rl][cc + t];
-        if (p.alpha != nullptr) {
+        if (CAP) {
           const float au = p.alpha[l] * p.cu[l][r];
 #pragma unroll
           for (int t = 0; t < 8; ++t)
@@ -200,15 +200,15 @@ __global__ void __launch_bounds__(kThreads) apply_tall_kernel(const __grid_const
   }
 }
 
-template <bool F32>
+template <bool F32, bool CAP>
 cudaError_t launch_typed(const ApplyParams& p, int batch, bool tall, bool vec, cudaStream_t s) {
   dim3 grid(p.nblk, batch);
   if (tall) {
-    if (vec) apply_tall_kernel<F32, true><<<grid, kThreads, 0, s>>>(p);
-    else apply_tall_kernel<F32, false><<<grid, kThreads, 0, s>>>(p);
+    if (vec) apply_tall_kernel<F32, true, CAP><<<grid, kThreads, 0, s>>>(p);
+    else apply_tall_kernel<F32, false, CAP><<<grid, kThreads, 0, s>>>(p);
   } else {
-    if (vec) apply_wide_kernel<F32, true><<<grid, kThreads, 0, s>>>(p);
-    else apply_wide_kernel<F32, false><<<grid, kThreads, 0, s>>>(p);
+    if (vec) apply_wide_kernel<F32, true, CAP><<<grid, kThreads, 0, s>>>(p);
+    else apply_wide_kernel<F32, false, CAP><<<grid, kThreads, 0, s>>>(p);
   }
   return cudaGetLastError();
 }
@@ -220,8 +220,12 @@ cudaError_t launch_apply(const ApplyParams& p, int batch, bool w_f32, cudaStream
   bool vec = p.cols % 8 == 0;
   for (int l = 0; l < batch && vec; ++l)
     if (reinterpret_cast<uintptr_t>(p.w[l]) % 16) vec = false;
-  return w_f32 ? launch_typed<true>(p, batch, tall, vec, stream)
-               : launch_typed<false>(p, batch, tall, vec, stream);
+  // the cap term is its own instantiation: the plain pass keeps its register allocation
+  if (p.alpha != nullptr)
+    return w_f32 ? launch_typed<true, true>(p, batch, tall, vec, stream)
+                 : launch_typed<false, true>(p, batch, tall, vec, stream);
+  return w_f32 ? launch_typed<true, false>(p, batch, tall, vec, stream)
+               : launch_typed<false, false>(p, batch, tall, vec, stream);
 }
 
 }  // namespace muon
