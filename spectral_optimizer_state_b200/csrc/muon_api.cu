@@ -153,6 +153,14 @@ struct muon_ctx {
   // scratch of the spectral passes (GEMV partials, norms, cap partials)
   void* d_aux = nullptr;
   size_t aux_bytes = 0;
+  // results of the last call as muon_get_status / muon_get_norms report them: the per-matrix
+  // arrays of the last run, or the gathered copies of a slab-pipelined host call
+  const float* out_nu = nullptr;
+  const int* out_flags = nullptr;
+  float* d_nu_all = nullptr;
+  int* d_flags_all = nullptr;
+  int cap_all = 0;
+  std::vector<cudaEvent_t> copy_events;  // one per slab of a host call
   // per-launch timing
   bool profiling = false;
   std::vector<cudaEvent_t> events;  // pool, two per recorded launch
@@ -400,12 +408,12 @@ muon_status ensure_aux(muon_ctx* c, size_t bytes) {
 }
 
 muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* hp, bool step,
-                float eps, cudaStream_t s, const CapSpec* cap = nullptr) {
+                float eps, cudaStream_t s, const CapSpec* cap = nullptr, bool clear_status = true) {
   muon_status st = reserve(c, plans, s);
   if (st != MUON_OK) return st;
   int total = 0;
   for (auto& p : plans) total += p.batch;
-  MUON_CUDA(cudaMemsetAsync(c->d_status, 0, sizeof(int), s), "clear status");
+  if (clear_status) MUON_CUDA(cudaMemsetAsync(c->d_status, 0, sizeof(int), s), "clear status");
 
   // K1: momentum / look-ahead / norm of one group.
   auto k1 = [&](const GroupPlan& p, cudaStream_t strm) -> muon_status {
@@ -636,6 +644,8 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
   c->last_count = total;
   c->last_stream = s;
   c->pending = true;
+  c->out_nu = c->d_nu;
+  c->out_flags = c->d_flags;
   return MUON_OK;
 }
 
@@ -749,6 +759,9 @@ muon_status muon_destroy(muon_ctx* c) {
   cudaFree(c->d_done);
   cudaFree(c->d_stage);
   cudaFree(c->d_aux);
+  cudaFree(c->d_nu_all);
+  cudaFree(c->d_flags_all);
+  for (cudaEvent_t e : c->copy_events) cudaEventDestroy(e);
   for (cudaEvent_t e : c->events) cudaEventDestroy(e);
   for (int g = 0; g < MUON_MAX_GROUPS; ++g) {
     if (c->ev_k1[g]) cudaEventDestroy(c->ev_k1[g]);
@@ -832,7 +845,7 @@ muon_status muon_get_status(muon_ctx* c, int* flags, int capacity, int* count) {
   MUON_CUDA(cudaMemcpy(&status, c->d_status, sizeof(int), cudaMemcpyDeviceToHost), "read status");
   std::vector<int> f(c->last_count);
   if (c->last_count > 0)
-    MUON_CUDA(cudaMemcpy(f.data(), c->d_flags, sizeof(int) * c->last_count, cudaMemcpyDeviceToHost),
+    MUON_CUDA(cudaMemcpy(f.data(), c->out_flags, sizeof(int) * c->last_count, cudaMemcpyDeviceToHost),
               "read flags");
   if (flags) std::memcpy(flags, f.data(), sizeof(int) * std::min(capacity, c->last_count));
   if (status & kStatusTimeout) return MUON_ERR_TIMEOUT;
@@ -847,7 +860,7 @@ muon_status muon_get_norms(muon_ctx* c, float* nu, int capacity, int* count) {
   if (count) *count = c->last_count;
   if (!c->pending || c->last_count == 0) return MUON_OK;
   MUON_CUDA(cudaStreamSynchronize(c->last_stream), "stream synchronize");
-  MUON_CUDA(cudaMemcpy(nu, c->d_nu, sizeof(float) * std::min(capacity, c->last_count),
+  MUON_CUDA(cudaMemcpy(nu, c->out_nu, sizeof(float) * std::min(capacity, c->last_count),
                        cudaMemcpyDeviceToHost),
             "read norms");
   return MUON_OK;
@@ -879,32 +892,113 @@ muon_status muon_step_groups_host(muon_ctx* c, const muon_group* groups, int ngr
     }
     c->stage_bytes = need;
   }
-  // Device-side copies of the groups whose G pointers now point into the staging buffer.
+  // Staging slot of every matrix (256-byte aligned, group after group).
   std::vector<std::vector<const void*>> gptr(ngroups);
-  std::vector<muon_group> dev(groups, groups + ngroups);
+  std::vector<std::vector<size_t>> gbytes(ngroups);
   size_t off = 0;
+  int total = 0;
   for (int i = 0; i < ngroups; ++i) {
     const size_t eb = groups[i].dtype == MUON_F32 ? 4 : 2;
     const size_t bytes = static_cast<size_t>(groups[i].rows) * groups[i].cols * eb;
     gptr[i].resize(groups[i].batch);
+    gbytes[i].assign(groups[i].batch, bytes);
     for (int l = 0; l < groups[i].batch; ++l) {
-      void* dst = static_cast<char*>(c->d_stage) + off;
-      MUON_CUDA(cudaMemcpyAsync(dst, groups[i].G[l], bytes, cudaMemcpyHostToDevice, s), "gradient upload");
-      gptr[i][l] = dst;
+      gptr[i][l] = static_cast<char*>(c->d_stage) + off;
       off += align_up(bytes, 256);
     }
-    dev[i].G = gptr[i].data();
+    total += groups[i].batch;
   }
-  std::vector<GroupPlan> plans;
-  st = validate_and_plan(c, dev.data(), ngroups, true, plans);
-  if (st != MUON_OK) return st;
-  st = run(c, plans, hp, true, hp->eps, s);
-  if (st != MUON_OK) return st;
+  if (c->side == nullptr) {
+    // one stream: every upload, then one step over all groups
+    std::vector<muon_group> dev(groups, groups + ngroups);
+    for (int i = 0; i < ngroups; ++i) {
+      for (int l = 0; l < groups[i].batch; ++l)
+        MUON_CUDA(cudaMemcpyAsync(const_cast<void*>(gptr[i][l]), groups[i].G[l], gbytes[i][l],
+                                  cudaMemcpyHostToDevice, s),
+                  "gradient upload");
+      dev[i].G = gptr[i].data();
+    }
+    std::vector<GroupPlan> plans;
+    st = validate_and_plan(c, dev.data(), ngroups, true, plans);
+    if (st != MUON_OK) return st;
+    st = run(c, plans, hp, true, hp->eps, s);
+    if (st != MUON_OK) return st;
+  } else {
+    // Slab pipeline: the uploads run on the side stream (copy engine) slab after slab while the
+    // caller's stream steps each slab as soon as its gradients have landed, so the PCIe transfer of
+    // slab k+1 overlaps the step of slab k.  A slab is up to ~32 MB of one group's gradients.
+    constexpr size_t kSlabBytes = size_t(32) << 20;
+    struct Slab { int g, l0, n; };
+    std::vector<Slab> slabs;
+    for (int i = 0; i < ngroups; ++i) {
+      const size_t mb = std::max<size_t>(gbytes[i][0], 1);
+      const int per = static_cast<int>(std::max<size_t>(1, kSlabBytes / mb));
+      for (int l0 = 0; l0 < groups[i].batch; l0 += per)
+        slabs.push_back({i, l0, std::min(per, groups[i].batch - l0)});
+    }
+    while (c->copy_events.size() < slabs.size()) {
+      cudaEvent_t e;
+      MUON_CUDA(cudaEventCreateWithFlags(&e, cudaEventDisableTiming), "event");
+      c->copy_events.push_back(e);
+    }
+    if (total > c->cap_all) {
+      MUON_CUDA(cudaStreamSynchronize(s), "sync before result growth");
+      cudaFree(c->d_nu_all);
+      cudaFree(c->d_flags_all);
+      c->d_nu_all = nullptr;
+      c->d_flags_all = nullptr;
+      c->cap_all = 0;
+      if (cudaMalloc(&c->d_nu_all, sizeof(float) * total) != cudaSuccess ||
+          cudaMalloc(&c->d_flags_all, sizeof(int) * total) != cudaSuccess) {
+        cudaGetLastError();
+        return MUON_ERR_ALLOC;
+      }
+      c->cap_all = total;
+    }
+    // the uploads start once everything queued on the caller's stream (e.g. the previous step
+    // still reading the staging buffer) is done
+    MUON_CUDA(cudaEventRecord(c->ev_fork, s), "fork");
+    MUON_CUDA(cudaStreamWaitEvent(c->side, c->ev_fork, 0), "fork");
+    for (size_t k = 0; k < slabs.size(); ++k) {
+      const Slab& sl = slabs[k];
+      for (int l = sl.l0; l < sl.l0 + sl.n; ++l)
+        MUON_CUDA(cudaMemcpyAsync(const_cast<void*>(gptr[sl.g][l]), groups[sl.g].G[l], gbytes[sl.g][l],
+                                  cudaMemcpyHostToDevice, c->side),
+                  "gradient upload");
+      MUON_CUDA(cudaEventRecord(c->copy_events[k], c->side), "upload done");
+    }
+    int first = 0;
+    std::vector<int> first_of_group(ngroups, 0);
+    for (int i = 1; i < ngroups; ++i) first_of_group[i] = first_of_group[i - 1] + groups[i - 1].batch;
+    for (size_t k = 0; k < slabs.size(); ++k) {
+      const Slab& sl = slabs[k];
+      MUON_CUDA(cudaStreamWaitEvent(s, c->copy_events[k], 0), "wait upload");
+      muon_group sg = groups[sl.g];
+      sg.W = groups[sl.g].W + sl.l0;
+      sg.G = gptr[sl.g].data() + sl.l0;
+      sg.M = groups[sl.g].M + sl.l0;
+      sg.batch = sl.n;
+      std::vector<GroupPlan> plans;
+      st = validate_and_plan(c, &sg, 1, true, plans);
+      if (st != MUON_OK) return st;
+      st = run(c, plans, hp, true, hp->eps, s, nullptr, /*clear_status=*/k == 0);
+      if (st != MUON_OK) return st;
+      first = first_of_group[sl.g] + sl.l0;
+      MUON_CUDA(cudaMemcpyAsync(c->d_nu_all + first, c->d_nu, sizeof(float) * sl.n, cudaMemcpyDeviceToDevice, s),
+                "gather norms");
+      MUON_CUDA(cudaMemcpyAsync(c->d_flags_all + first, c->d_flags, sizeof(int) * sl.n, cudaMemcpyDeviceToDevice,
+                                s),
+                "gather flags");
+    }
+    c->last_count = total;
+    c->out_nu = c->d_nu_all;
+    c->out_flags = c->d_flags_all;
+  }
   if (nu_host)
-    MUON_CUDA(cudaMemcpyAsync(nu_host, c->d_nu, sizeof(float) * c->last_count, cudaMemcpyDeviceToHost, s),
+    MUON_CUDA(cudaMemcpyAsync(nu_host, c->out_nu, sizeof(float) * c->last_count, cudaMemcpyDeviceToHost, s),
               "norm download");
   if (flags_host)
-    MUON_CUDA(cudaMemcpyAsync(flags_host, c->d_flags, sizeof(int) * c->last_count, cudaMemcpyDeviceToHost, s),
+    MUON_CUDA(cudaMemcpyAsync(flags_host, c->out_flags, sizeof(int) * c->last_count, cudaMemcpyDeviceToHost, s),
               "flag download");
   MUON_CUDA(cudaStreamSynchronize(s), "stream synchronize");
   return muon_get_status(c, nullptr, 0, nullptr);

@@ -244,6 +244,38 @@ def test_host_gradient_entry_matches_device_entry(ctx):
         assert abs(n - 1.95 * np.linalg.norm(g.astype(np.float64))) <= 1e-5 * n
 
 
+def test_host_entry_slab_pipeline_matches_device_entry(ctx):
+    """Host gradients big enough to be uploaded in several slabs (in_proj matrices, ~32 MB per slab)
+    give bit-identical W and M, norms and flags in group order, and a non-finite matrix in a later
+    slab is flagged at its own index."""
+    import torch
+    shapes = [(3352, 768), (768, 1536)]
+    counts = [14, 5]
+    Gs = [_inputs(shapes[i], counts[i], seed=40 + i, kind="spike") for i in range(2)]
+    Gs[0][9] = Gs[0][9].copy()
+    Gs[0][9][5, 7] = np.nan  # third slab of the first group
+    W0 = [[to_device(w, "bf16") for w in group_weights(5, i, counts[i], *shapes[i])] for i in range(2)]
+    Wa = [[w.clone() for w in ws] for ws in W0]
+    Wb = [[w.clone() for w in ws] for ws in W0]
+    Ma = [[torch.zeros(shapes[i], device="cuda") for _ in range(counts[i])] for i in range(2)]
+    Mb = [[torch.zeros(shapes[i], device="cuda") for _ in range(counts[i])] for i in range(2)]
+    ctx.step_groups([(Wa[i], [to_device(g, "bf16") for g in Gs[i]], Ma[i]) for i in range(2)], **HP)
+    st_dev, flags_dev = ctx.status()
+    nu_dev = ctx.norms()
+    host = [[torch.from_numpy(g).to(torch.bfloat16).pin_memory() for g in Gs[i]] for i in range(2)]
+    nu, flags = ctx.step_groups_host([(Wb[i], host[i], Mb[i]) for i in range(2)], **HP)
+    assert st_dev == 5 and flags == flags_dev
+    assert [i for i, f in enumerate(flags) if f] == [9]
+    assert ctx.status() == (5, flags)
+    assert np.array_equal(np.asarray(ctx.norms()), np.asarray(nu), equal_nan=True)
+    assert np.array_equal(np.asarray(nu), np.asarray(nu_dev), equal_nan=True)
+    for i in range(2):
+        for a, b, ma, mb in zip(Wa[i], Wb[i], Ma[i], Mb[i]):
+            assert torch.equal(a, b)
+            assert torch.equal(ma.nan_to_num(), mb.nan_to_num())
+    assert torch.equal(Wb[0][9], W0[0][9])  # the flagged matrix keeps its weights
+
+
 def test_bad_arguments_raise(ctx):
     import torch
     from spectral_optimizer_state_b200 import MuonError
