@@ -334,6 +334,8 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
         const int nk = q.k_tiles * q.nseg;
         const bool narrow = !q.b_mn_major && ti.nw <= 128;
         const uint32_t bbytes = q.b_mn_major ? 4u * MNMAJ_BOX_BYTES : (narrow ? KMAJ_BOX_BYTES : 2u * KMAJ_BOX_BYTES);
+        // a symmetric tile that starts on the diagonal has A = the first 128 rows of B
+        const bool diag_tile = q.sym && ti.m0 == ti.n0;
         for (int kk = 0; kk < nk; ++kk, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -347,8 +349,9 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
           segment_planes(q.nseg, seg, pa, pb);
           const uint32_t sa = base + s * STAGE_BYTES;
           const uint32_t sb = sa + A_BYTES;
-          mbar_arrive_expect_tx(full_bar(s), A_BYTES + bbytes);
-          tma_load_4d(sa, &q.tmA, full_bar(s), kb * BK, ti.m0, ti.l, pa);
+          const bool a_in_b = diag_tile && pa == pb;  // the MMA reads A from B's first rows
+          mbar_arrive_expect_tx(full_bar(s), (a_in_b ? 0u : A_BYTES) + bbytes);
+          if (!a_in_b) tma_load_4d(sa, &q.tmA, full_bar(s), kb * BK, ti.m0, ti.l, pa);
           if (q.b_mn_major)
             tma_load_5d(sb, &q.tmB, full_bar(s), 0, kb * BK, ti.n0 / 64, ti.l, pb);
           else
@@ -380,6 +383,7 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
         const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
         const uint32_t idesc = instr_desc_bf16(BM, ti.nw, q.b_mn_major != 0);
         const int nk = q.k_tiles * q.nseg;
+        const bool diag_tile = q.sym && ti.m0 == ti.n0;
         for (int kk = 0; kk < nk; ++kk, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -387,8 +391,11 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
             ok = false;
             break;
           }
-          const uint32_t sa = base + s * STAGE_BYTES;
-          const uint32_t sb = sa + A_BYTES;
+          int pa, pb;
+          segment_planes(q.nseg, kk / q.k_tiles, pa, pb);
+          const uint32_t sb = base + s * STAGE_BYTES + A_BYTES;
+          // K-major, 128-byte swizzle: B's rows 0..127 are laid out exactly as an A tile
+          const uint32_t sa = diag_tile && pa == pb ? sb : base + s * STAGE_BYTES;
 #pragma unroll
           for (int k4 = 0; k4 < BK / 16; ++k4) {
             const uint64_t ad = smem_desc_sw128(sa + 32u * k4, 16u, 1024u);
