@@ -100,6 +100,7 @@ template <bool F32, bool VEC, bool CAP>
 __global__ void __launch_bounds__(kThreads) apply_wide_kernel(const __grid_constant__ ApplyParams p) {
   const int l = blockIdx.y;
   if (p.flags != nullptr && p.flags[l] != 0) return;
+  if (p.status != nullptr && (*p.status & kStatusTimeout)) return;  // the iterate is incomplete
   void* w = p.w[l];
   const uint16_t* o = p.o + static_cast<long long>(l) * p.o_mat;
   const int C = p.cols;
@@ -143,6 +144,7 @@ __global__ void __launch_bounds__(kThreads) apply_tall_kernel(const __grid_const
   __shared__ float tile[64][65];
   const int l = blockIdx.y;
   if (p.flags != nullptr && p.flags[l] != 0) return;
+  if (p.status != nullptr && (*p.status & kStatusTimeout)) return;  // the iterate is incomplete
   void* w = p.w[l];
   const uint16_t* o = p.o + static_cast<long long>(l) * p.o_mat;
   const int R = p.rows, C = p.cols;

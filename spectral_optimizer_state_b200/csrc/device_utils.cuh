@@ -114,6 +114,11 @@ __device__ __forceinline__ bool wait_counter_bounded(const unsigned* p, unsigned
     if (ld_acquire_gpu(p) >= target) return true;
     if ((i & 15u) == 0) {
       if (*abort_flag) return false;
+      // another CTA gave up (the counter may never complete): stop now, not after our own limit
+      if (status && (ld_relaxed_gpu(reinterpret_cast<const unsigned*>(status)) & kStatusTimeout)) {
+        *abort_flag = 1;
+        return false;
+      }
       if (global_timer_ns() - t0 > kWaitLimitNs) {
         *abort_flag = 1;
         if (status) atomicOr(status, kStatusTimeout);

@@ -439,7 +439,8 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
         if (lane == 0) {
           bulk_wait_group_all();
           fence_proxy_async_global();
-          red_release_gpu_add(q.done_self + ti.l, 1u);
+          if (!(P.drop_signal && blockIdx.x == 0 && e == 0 && local == 0))
+            red_release_gpu_add(q.done_self + ti.l, 1u);
         }
         __syncwarp();
       }

@@ -48,6 +48,7 @@ struct ApplyParams {
   int apply;                // 1: W <- decay*W - lrs*O ; 0: W <- O
   float decay, lrs;
   const int* flags;         // matrices with a nonzero flag are left unchanged (null: none)
+  const int* status;        // device status word: nothing is written after a timeout (null: none)
   int nblk;                 // blocks per matrix
   // spectral cap (null alpha: none): O is replaced by O - alpha_l u_l v_l^T,
   // u_l of length rows and v_l of length cols of W
@@ -130,6 +131,9 @@ struct GemmParams {
   int nprob;
   int total_tiles;
   int* status;
+  // test hook: CTA 0's first epilogue warp does not count its first finished tile, so the
+  // tiles that depend on it can only end through their bounded waits (MUON_ERR_TIMEOUT)
+  int drop_signal;
 };
 
 // Two kernels share the problem description:

@@ -138,6 +138,9 @@ struct muon_ctx {
   // co-running elementwise passes slow the GEMM by as much time as they hide (both draw on the
   // same L2 -> SM bandwidth), and one persistent launch for all groups has no gap between them.
   bool overlap = false;
+  // MUON_TEST_DROP_SIGNAL=1 at creation: the next persistent Newton-Schulz launch drops one
+  // completion signal (test of the bounded waits; used once, then cleared)
+  bool drop_signal_once = false;
   cudaStream_t side = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   cudaEvent_t ev_k1[MUON_MAX_GROUPS] = {};
@@ -533,6 +536,10 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
       ++gp.nprob;
     }
     gp.total_tiles = tiles;
+    if (persistent && c->drop_signal_once && c->gemm_kind == GEMM_SINGLE && gp.nprob > 1) {
+      gp.drop_signal = 1;
+      c->drop_signal_once = false;
+    }
     if (persistent)
       MUON_CUDA(cudaMemsetAsync(c->d_done, 0, sizeof(unsigned) * gp.nprob * MUON_MAX_BATCH, strm), "clear counters");
     const int units = std::min(tiles, pair ? c->sm_count / 2 : c->sm_count);
@@ -563,6 +570,7 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
       ap.lrs = hp->lr * shape_scale(p.rows, p.cols, hp->scale_mode);
       ap.flags = c->d_flags + p.mat_off;
     }
+    ap.status = c->d_status;
     ap.nblk = momentum_blocks_per_matrix(p.rows, p.cols);
     if (cap != nullptr) {
       for (int l = 0; l < p.batch; ++l) {
@@ -709,6 +717,9 @@ muon_status muon_create(muon_ctx** out, int device) {
   }
   if (const char* l = std::getenv("MUON_LAUNCH")) {
     if (std::strcmp(l, "phase") == 0) c->per_phase = true;
+  }
+  if (const char* d = std::getenv("MUON_TEST_DROP_SIGNAL")) {
+    if (std::strcmp(d, "1") == 0) c->drop_signal_once = true;
   }
   if (const char* o = std::getenv("MUON_OVERLAP")) {
     if (std::strcmp(o, "1") == 0) c->overlap = true;
