@@ -199,3 +199,40 @@ def test_golden_fixture_regression():
     assert np.allclose(O, np.array(cases["cubic10_5x3"]), rtol=0, atol=1e-15)
     O, _ = oracle.orthogonalize(G.T, QUINTIC5)
     assert np.allclose(O, np.array(cases["quintic5_3x5"]), rtol=0, atol=1e-15)
+
+
+def _loops_step(W, G, M, coeffs, lr, beta, wd, eps, scale):
+    """The whole step with explicit Python loops over scalars (no NumPy arithmetic)."""
+    R, C = len(W), len(W[0])
+    Mn = [[beta * M[i][j] + G[i][j] for j in range(C)] for i in range(R)]
+    U = [[G[i][j] + beta * Mn[i][j] for j in range(C)] for i in range(R)]
+    nu = sum(U[i][j] ** 2 for i in range(R) for j in range(C)) ** 0.5
+    X = [[U[i][j] / (nu + eps) for j in range(C)] for i in range(R)]
+    tall = R > C
+    if tall:
+        X = [[X[i][j] for i in range(R)] for j in range(C)]
+    m, n = len(X), len(X[0])
+    for a, b, c in coeffs:
+        A = [[sum(X[i][k] * X[j][k] for k in range(n)) for j in range(m)] for i in range(m)]
+        AA = [[sum(A[i][k] * A[k][j] for k in range(m)) for j in range(m)] for i in range(m)]
+        B = [[b * A[i][j] + c * AA[i][j] for j in range(m)] for i in range(m)]
+        X = [[a * X[i][j] + sum(B[i][k] * X[k][j] for k in range(m)) for j in range(n)] for i in range(m)]
+    O = [[X[j][i] for j in range(m)] for i in range(n)] if tall else X
+    Wn = [[W[i][j] * (1 - lr * wd) - lr * scale * O[i][j] for j in range(C)] for i in range(R)]
+    return Wn, Mn
+
+
+@pytest.mark.parametrize("shape", [(2, 3), (3, 5), (5, 3)])
+def test_brute_force_loops_tiny(shape):
+    """T6: the oracle's step equals a scalar-loop transcription of the definitions on tiny inputs."""
+    R, C = shape
+    rng = rng_for(77, R * 10 + C)
+    W = rng.standard_normal(shape) * 0.02
+    G = rng.standard_normal(shape)
+    M = rng.standard_normal(shape) * 0.1
+    coeffs = [oracle.QUINTIC] * 3 + [oracle.CUBIC] * 2
+    s = oracle.shape_scale(R, C, oracle.SCALE_SQRT_RATIO)
+    r = oracle.muon_step(W, G, M, coeffs, lr=0.02, beta=0.95, weight_decay=0.1, eps=1e-7)
+    Wl, Ml = _loops_step(W.tolist(), G.tolist(), M.tolist(), coeffs, 0.02, 0.95, 0.1, 1e-7, s)
+    assert np.allclose(r["W"], np.array(Wl), rtol=0, atol=1e-13)
+    assert np.allclose(r["M"], np.array(Ml), rtol=0, atol=1e-13)
