@@ -390,20 +390,24 @@ def test_single_cta_and_pair_kernels_agree():
             assert rel_f(a, b) <= 5e-3
 
 
-def test_two_stream_schedule_is_bitwise_equal_to_serial():
-    """The pipelined schedule (momentum and apply passes of other groups on a side stream)
-    computes exactly what the one-stream schedule computes, over three groups and two steps."""
+@pytest.mark.parametrize("env", [{"MUON_OVERLAP": "1"}, {"MUON_LAUNCH": "phase"}])
+def test_alternative_schedules_are_bitwise_equal_to_the_default(env):
+    """The two-stream schedule (momentum and apply passes of other groups on a side stream)
+    and the one-launch-per-phase schedule compute exactly what the default single persistent
+    launch computes, over three groups and two steps."""
     import os
     import torch
     from spectral_optimizer_state_b200 import Muon
     shapes = [(200, 328), (328, 200), (768, 1536)]
     results = {}
-    for mode in ("1", "0"):
-        os.environ["MUON_OVERLAP"] = mode
+    for mode in ("alt", "default"):
+        if mode == "alt":
+            os.environ.update(env)
         try:
             m = Muon(0)
         finally:
-            del os.environ["MUON_OVERLAP"]
+            for k in env:
+                os.environ.pop(k, None)
         m.set_coeffs(QUINTIC5)
         W = [[to_device(w, "bf16") for w in group_weights(7, i, 3, r, c)] for i, (r, c) in enumerate(shapes)]
         M = [[torch.zeros((r, c), dtype=torch.float32, device="cuda") for _ in range(3)] for (r, c) in shapes]
@@ -414,9 +418,9 @@ def test_two_stream_schedule_is_bitwise_equal_to_serial():
         assert m.status()[0] == 0
         results[mode] = ([to_numpy(w) for ws in W for w in ws], [to_numpy(x) for ms in M for x in ms], m.norms())
         m.close()
-    for a, b in zip(results["1"][0] + results["1"][1], results["0"][0] + results["0"][1]):
+    for a, b in zip(results["alt"][0] + results["alt"][1], results["default"][0] + results["default"][1]):
         assert np.array_equal(a, b)
-    assert results["1"][2] == results["0"][2]
+    assert results["alt"][2] == results["default"][2]
 
 
 def test_scaled_2k_model_full_size_sampled():
