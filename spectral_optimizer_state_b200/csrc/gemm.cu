@@ -214,10 +214,17 @@ __device__ __forceinline__ void store_chunk(const CUtensorMap* map, uint32_t sta
 // (this warp's lane quarter), 32-column chunks c_first, c_first + 64, ...
 // v = alpha s_l acc + beta cin + diag on the diagonal, split into planes and
 // stored through TMA; columns from `mirror_from` on are also stored transposed.
+// `release()` hands the accumulator back to the MMA issuer: it runs once, right after this
+// warp's last TMEM read of the tile (the stores that follow work from registers).
+template <class Release>
 __device__ __forceinline__ void epilogue_warp_tile(const GemmProblem& q, const Tile& ti, uint32_t tbase,
                                                    int row0, int lane, int c_first, int mirror_from,
-                                                   uint32_t my_stage, int& sb) {
-  if (row0 >= q.M) return;
+                                                   uint32_t my_stage, int& sb, Release&& release) {
+  if (row0 >= q.M) {
+    release();
+    return;
+  }
+  bool released = false;
   const int row = row0 + lane;
   const float scale = q.alpha * (q.mat_scale != nullptr ? q.mat_scale[ti.l] : 1.0f);
   for (int c = c_first; c < ti.nw; c += 64) {
@@ -228,6 +235,10 @@ __device__ __forceinline__ void epilogue_warp_tile(const GemmProblem& q, const T
     __syncwarp();  // tcgen05.ld is warp-collective
     tmem_load_32cols(tbase + c, r);
     tmem_load_wait();
+    if (c + 64 >= ti.nw || j0 + 64 >= q.N) {  // this warp's last chunk of the tile
+      release();
+      released = true;
+    }
     float v[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = scale * __uint_as_float(r[i]);
@@ -249,6 +260,7 @@ __device__ __forceinline__ void epilogue_warp_tile(const GemmProblem& q, const T
       if (mirror) store_chunk<true>(&q.tmOut, my_stage, sb, lane, b, row0, j0, ti.l, p);
     }
   }
+  if (!released) release();
 }
 
 // ------------------------------------------------------------------ kernel
@@ -433,7 +445,10 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
         // cin was written earlier in this launch: acquire it for this warp's plain loads
         if (!wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status)) break;
       }
-      epilogue_warp_tile(q, ti, tbase, ti.m0 + 32 * quarter, lane, 32 * half, ti.m0 + BM, my_stage, sb);
+      epilogue_warp_tile(q, ti, tbase, ti.m0 + 32 * quarter, lane, 32 * half, ti.m0 + BM, my_stage, sb, [&] {
+        tc_fence_before();
+        mbar_arrive(tempty_bar(acc));
+      });
       if (q.done_self != nullptr) {
         // this warp's stores of the tile are complete and visible: count it done
         if (lane == 0) {
@@ -444,8 +459,6 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
         }
         __syncwarp();
       }
-      tc_fence_before();
-      mbar_arrive(tempty_bar(acc));
     }
     if (lane == 0) bulk_wait_group_all();
   }
@@ -664,7 +677,11 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_c
         if (!wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status)) break;
       }
       epilogue_warp_tile(q, ti, tbase, ti.m0 + 128 * static_cast<int>(rank) + 32 * quarter, lane,
-                         32 * half, ti.m0 + PBM, my_stage, sb);
+                         32 * half, ti.m0 + PBM, my_stage, sb, [&] {
+                           tc_fence_before();
+                           __syncwarp();
+                           if (lane == 0) mbar_arrive_remote(map_shared_rank(tempty_bar(acc), 0));
+                         });
       if (q.done_self != nullptr) {
         if (lane == 0) {
           bulk_wait_group_all();
@@ -673,9 +690,6 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_c
         }
         __syncwarp();
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(map_shared_rank(tempty_bar(acc), 0));
     }
     if (lane == 0) bulk_wait_group_all();
   }
