@@ -25,6 +25,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -98,11 +99,23 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _code_only(text):
+    """Source without comments, trailing blanks or empty lines (a capture stays valid across comment edits)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = []
+    for line in text.splitlines():
+        line = re.sub(r"//.*$", "", line).rstrip()
+        if line:
+            out.append(line)
+    return "\n".join(out)
+
+
 def gemm_source_hash():
+    """sha256 (16 hex digits) of the NS kernel's code: gemm.cu, device_utils.cuh, internal.h without comments."""
     h = hashlib.sha256()
     for f in ("gemm.cu", "device_utils.cuh", "internal.h"):
-        with open(os.path.join(ROOT, "spectral_optimizer_state_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "spectral_optimizer_state_b200", "csrc", f)) as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

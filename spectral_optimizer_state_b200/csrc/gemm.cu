@@ -9,16 +9,22 @@
 // Newton-Schulz step: the orthogonalisation is matrix products only, no SVD;
 // Muon Meets Mamba, abstract: one orthogonalised update per weight matrix.)
 //
-// One persistent kernel serves all three: a CTA owns a 128-row M tile and up
-// to 256 N columns, loops over a static round-robin list of tiles (every
-// matrix of one or two same-phase problems), and runs
-//   warp 0      TMA producer (one thread) into a 4-stage ring of 48 KB stages,
+// One persistent kernel serves all three: a launch carries every (group,
+// iteration, phase) problem of a step, a CTA owns a 128-row M tile and up to
+// 256 N columns, walks a static round-robin list of tiles (group by group,
+// phase by phase, matrix by matrix), and runs
+//   warp 0      TMA producer (one thread) into a 4-stage ring of 48 KB stages;
+//               before a tile it waits for the previous phase of that tile's
+//               matrix (per-(problem, matrix) completion counters),
 //   warp 1      TMEM allocation + UMMA issuer (one thread),
 //   warps 2..9  epilogue: TMEM -> registers -> fused arithmetic -> 32 x 32
-//               swizzled shared-memory tiles -> TMA tensor stores.
+//               swizzled shared-memory tiles -> TMA tensor stores; each warp
+//               hands the accumulator back after its last TMEM read and counts
+//               the tile done once its stores have landed.
 // Two TMEM accumulators (2 x 256 fp32 columns) let the epilogue of one tile
 // overlap the main loop of the next.  Symmetric outputs are computed on the
-// upper 128 x 128 blocks only (tiles start at the diagonal block); the lower
+// upper 128 x 128 blocks only (tiles start at the diagonal block, and such a
+// tile reads its A operand from the first rows of its B stage); the lower
 // blocks are written by transposing the staged tile (a second TMA store).
 // The update's aX term is folded into the polynomial (B' = aI + bA + cA^2),
 // so the update epilogue only scales, converts and stores.
