@@ -68,3 +68,13 @@ def test_work_counts():
     assert bench.ns_flops(g) == 1146617856000
     assert bench.elements(g) == 24 * 768 * 1536 + 24 * 3352 * 768
     assert bench.momentum_bytes(g) == 12 * bench.elements(g)
+
+
+def test_kernel_hash_ignores_comments_but_not_code():
+    import bench
+    a = "int x = 1; // one\n/* block\ncomment */\n\nint y = 2;\n"
+    b = "int x = 1;   // a different note\n\nint y = 2;  \n"
+    c = "int x = 3; // one\nint y = 2;\n"
+    assert bench._code_only(a) == bench._code_only(b) == "int x = 1;\nint y = 2;"
+    assert bench._code_only(c) != bench._code_only(a)
+    assert len(bench.gemm_source_hash()) == 16
