@@ -107,3 +107,21 @@ def test_tma_coordinates_aligned(m, n, kind):
                     x = n0 + rank * half + 64 * c
                     assert (x * 2) % 16 == 0  # MN-major B: x = n
                     assert half % 64 == 0
+
+
+@pytest.mark.parametrize("m,n", SHAPES)
+def test_diagonal_tiles_have_a_inside_b(m, n):
+    """Single-CTA symmetric problems: exactly the first tile of each 128-row block starts on the
+    diagonal (n0 == m0), and its B box ({64, 256} or, for tiles <= 128 wide, {64, 128}) holds at
+    least the 128 rows of the A tile, so the kernel may read A from the first rows of B."""
+    BM = KINDS["single"][0]
+    firsts = {}
+    for r in range(tiles_per_matrix(m, m, 1, "single")):
+        m0, n0, nw = decode(m, m, 1, r, "single")
+        firsts.setdefault(m0, (n0, nw))
+        if n0 == m0:
+            assert firsts[m0] == (n0, nw)  # only the block's first tile
+            box_rows = 256 if nw > 128 else 128
+            assert box_rows >= BM
+    assert sorted(firsts) == list(range(0, m, BM))
+    assert all(n0 == m0 for m0, (n0, _) in firsts.items())
