@@ -79,3 +79,22 @@ def test_shape_scale_matches_readings():
     assert sos.shape_scale(768, 1536) == 1.0
     assert abs(sos.shape_scale(3352, 768) - (3352 / 768) ** 0.5) < 1e-12
     assert sos.shape_scale(10, 10, sos.SCALE_NONE) == 1.0
+
+
+def declared_arities():
+    """name -> number of parameters, from the prototypes in include/muon.h."""
+    text = open(os.path.join(ROOT, "include", "muon.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(muon_[a-z_]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argtypes_match_the_prototypes(lib):
+    arities = declared_arities()
+    assert sorted(arities) == declared_symbols()
+    for name, n in arities.items():
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None and len(fn.argtypes) == n, (name, n, fn.argtypes)
