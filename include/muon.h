@@ -142,10 +142,15 @@ muon_status muon_step_groups(muon_ctx* ctx, const muon_group* groups, int ngroup
 
 /* End-to-end variant for callers whose gradients live in (preferably pinned)
  * HOST memory: each group's G entries are HOST pointers.  The gradients are
- * copied to a context-owned device staging buffer on `stream`, the step runs,
- * and the per-matrix ||U||_F (nu_host, may be NULL) and flags (flags_host, may
- * be NULL), in group order, are copied back.  Returns after the stream has
- * been synchronised; the return value includes device-side status. */
+ * uploaded to a context-owned device staging buffer in slabs of about 32 MB on
+ * an internal copy stream (ordered after the work already queued on `stream`);
+ * each slab is stepped on `stream` as soon as its upload has landed, so the
+ * transfer of the next slab overlaps the step of this one.  Results equal
+ * muon_step_groups on the same gradients bit for bit.  The per-matrix ||U||_F
+ * (nu_host, may be NULL) and flags (flags_host, may be NULL), in group order,
+ * are copied back.  Returns after the stream has been synchronised; the return
+ * value includes device-side status.  With pageable host memory the uploads do
+ * not overlap; pin the gradients. */
 muon_status muon_step_groups_host(muon_ctx* ctx, const muon_group* groups, int ngroups,
                                   const muon_hparams* hp, float* nu_host, int* flags_host,
                                   void* stream);
