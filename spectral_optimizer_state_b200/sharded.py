@@ -144,6 +144,27 @@ class ShardedMuon:
                 "reduce_scatter_bytes": self.world * self.seg * e,
                 "all_gather_bytes": self.world * self.seg * e}
 
+    def state_dict(self) -> dict:
+        """This rank's optimizer state: its momentum buffers by matrix index, and the ownership they follow.
+
+        Save one per rank (e.g. ``torch.save(opt.state_dict(), f"muon_rank{rank}.pt")``); the
+        weights are the model's and are saved with it.
+        """
+        return {"shapes": list(self.shapes), "world": self.world, "owner": list(self.owner),
+                "momenta": {i: m.detach().clone() for i, m in self.momenta.items()}}
+
+    def load_state_dict(self, state: dict):
+        """Restore the momentum buffers saved by ``state_dict`` on the same rank of a job with the
+        same shapes and world size (ownership is a pure function of both, so it matches)."""
+        if [tuple(x) for x in state["shapes"]] != self.shapes or state["world"] != self.world:
+            raise ValueError("checkpoint was written for different shapes or a different world size")
+        if list(state["owner"]) != self.owner:
+            raise ValueError("checkpoint ownership differs from this job's")
+        if sorted(state["momenta"]) != sorted(self.momenta):
+            raise ValueError("checkpoint holds another rank's matrices")
+        for i, m in state["momenta"].items():
+            self.momenta[i].copy_(m)
+
     def step(self, stream=None):
         """One data-parallel Muon step: reduce-scatter G, local step on owned matrices, all-gather W."""
         import torch.distributed as dist

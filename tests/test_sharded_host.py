@@ -119,3 +119,69 @@ def test_sharded_step_matches_single_process_oracle_on_averaged_gradients(world)
             assert np.allclose(Ws[i], W[i], rtol=0, atol=1e-12)
     if world == 2:
         assert set(owner) == {0, 1}
+
+
+def _resume_worker(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+    from spectral_optimizer_state_b200.sharded import ShardedMuon
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        def make():
+            return ShardedMuon(SHAPES, dtype=torch.float64, device="cpu", local_step=_oracle_step,
+                               state_dtype=torch.float64, **HP)
+
+        W0 = [torch.from_numpy(weights(rng_for(800, i), r, c)) for i, (r, c) in enumerate(SHAPES)]
+
+        def run(opt, first, last):
+            for s in range(first, last):
+                for g, G in zip(opt.grads, _grads(rank, s)):
+                    g.copy_(torch.from_numpy(G))
+                opt.step()
+
+        straight = make()
+        straight.load_weights(W0)
+        run(straight, 0, 3)
+        first = make()
+        first.load_weights(W0)
+        run(first, 0, 2)
+        ck = {"W": [w.clone() for w in first.weights], "state": first.state_dict()}
+        resumed = make()
+        resumed.load_weights(ck["W"])
+        resumed.load_state_dict(ck["state"])
+        run(resumed, 2, 3)
+        same = all(torch.equal(a, b) for a, b in zip(straight.weights, resumed.weights)) and \
+            all(torch.equal(straight.momenta[i], resumed.momenta[i]) for i in straight.momenta)
+        q.put((rank, same))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_checkpoint_resume_equals_straight_run():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_resume_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=300) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(same for _, same in out)
+
+
+def test_state_dict_rejects_another_layout():
+    import torch
+    from spectral_optimizer_state_b200.sharded import ShardedMuon
+    opt = ShardedMuon(SHAPES, dtype=torch.float64, device="cpu", local_step=_oracle_step,
+                      state_dtype=torch.float64, **HP)
+    st = opt.state_dict()
+    other = ShardedMuon(SHAPES[:-1], dtype=torch.float64, device="cpu", local_step=_oracle_step,
+                        state_dtype=torch.float64, **HP)
+    with pytest.raises(ValueError):
+        other.load_state_dict(st)
+    opt.load_state_dict(st)  # round trip on the same layout
