@@ -74,5 +74,25 @@ class MuonAdamW:
             adamw_step(W, G, [m for _, _, m, _ in entries], [v for _, _, _, v in entries], self.t,
                        stream=stream, **self.adamw_hp)
 
+    def state_dict(self) -> dict:
+        """Optimizer state by parameter name: Muon momentum, AdamW moments, and the step count."""
+        return {"t": self.t,
+                "muon": {n: m.detach().clone() for entries in self.muon.values() for (n, _, m) in entries},
+                "adamw": {n: (m.detach().clone(), v.detach().clone())
+                          for entries in self.adam.values() for (n, _, m, v) in entries}}
+
+    def load_state_dict(self, state: dict):
+        """Restore the state saved by ``state_dict`` for the same parameter names and shapes."""
+        muon = {n: m for entries in self.muon.values() for (n, _, m) in entries}
+        adam = {n: (m, v) for entries in self.adam.values() for (n, _, m, v) in entries}
+        if set(state["muon"]) != set(muon) or set(state["adamw"]) != set(adam):
+            raise ValueError("checkpoint holds a different parameter split")
+        for n, m in state["muon"].items():
+            muon[n].copy_(m)
+        for n, (m, v) in state["adamw"].items():
+            adam[n][0].copy_(m)
+            adam[n][1].copy_(v)
+        self.t = int(state["t"])
+
     def close(self):
         self.ctx.close()

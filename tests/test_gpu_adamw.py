@@ -77,3 +77,41 @@ def test_muon_adamw_split_small_mamba_like(mode):
         bound = 2e-2 * np.linalg.norm(ref - W0[n]) + np.linalg.norm(half_ulp_bf16(ref))
         assert np.linalg.norm(to_numpy(w) - ref) <= bound, n
     opt.close()
+
+
+def test_muon_adamw_checkpoint_resume_equals_straight_run():
+    """Three steps straight equal two steps, a state_dict round trip into a new optimizer, one more."""
+    import io
+    import torch
+    from spectral_optimizer_state_b200 import MuonAdamW
+    names = [("layers.0.mixer.in_proj.weight", (424, 96)), ("layers.0.mixer.out_proj.weight", (96, 192)),
+             ("layers.0.mixer.A_log", (3,)), ("embeddings.weight", (500, 96))]
+    rng = rng_for(63, 0)
+    W0 = {n: round_bf16(rng.standard_normal(s).astype(np.float32) * 0.02) for n, s in names}
+    Gs = [{n: torch.from_numpy(round_bf16(rng.standard_normal(s).astype(np.float32))).to(torch.bfloat16).cuda()
+           for n, s in names} for _ in range(3)]
+
+    def fresh():
+        params = [(n, torch.from_numpy(W0[n]).to(torch.bfloat16).cuda()) for n, _ in names]
+        return params, MuonAdamW(params, mode="both", coeffs=[oracle.QUINTIC] * 5)
+
+    pa, a = fresh()
+    for g in Gs:
+        a.step(g)
+    pb, b = fresh()
+    for g in Gs[:2]:
+        b.step(g)
+    buf = io.BytesIO()
+    torch.save({"params": {n: w.cpu() for n, w in pb}, "opt": b.state_dict()}, buf)
+    b.close()
+    buf.seek(0)
+    ck = torch.load(buf)
+    pc = [(n, ck["params"][n].cuda()) for n, _ in names]
+    c = MuonAdamW(pc, mode="both", coeffs=[oracle.QUINTIC] * 5)
+    c.load_state_dict(ck["opt"])
+    c.step(Gs[2])
+    torch.cuda.synchronize()
+    for (n, wa), (_, wc) in zip(pa, pc):
+        assert torch.equal(wa, wc), n
+    a.close()
+    c.close()
