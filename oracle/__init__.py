@@ -12,11 +12,16 @@ iteration, i.e. steepest descent under the spectral norm) together with the
 plainest reading of the steps they leave open; each reading is listed in the
 function that takes it.
 
-Pins (tests/test_oracle_pins.py) tie it to things other than itself: the
-SVD closed form U f_k(S) V^T of the iteration, the polar factor U V^T, the
+Pins tie it to things other than itself.  tests/test_oracle_pins.py: the SVD
+closed form U f_k(S) V^T of the iteration, the polar factor U V^T, the
 fixed-point scaling of semi-orthogonal inputs, the singular-value band of the
-polynomial, invariances, exact rational arithmetic on diagonal inputs, and
-closed forms of momentum and the decoupled update.
+polynomial, invariances, exact rational arithmetic on diagonal inputs, closed
+forms of momentum and the decoupled update, and a scalar-loop transcription of
+the whole step on tiny inputs.  tests/test_oracle_mutants.py: planted mistakes
+are rejected.  tests/test_oracle_adamw.py: AdamW's first step, moment closed
+forms, decay-only and scale cases, and the parameter selection.
+tests/test_oracle_spectral.py: power iteration and the smallest singular value
+against LAPACK and exact cases, and the cap's vanishing first-order growth.
 
 Parity unpinned (parameters, not facts of the pages): the quintic coefficient
 triple and the shape-scale convention.  Parity holds for whichever values are
