@@ -243,6 +243,31 @@ def blas_threads():
         return os.cpu_count()
 
 
+def blas_vendor():
+    try:
+        from threadpoolctl import threadpool_info
+        for d in threadpool_info():
+            if d.get("user_api") == "blas":
+                return f"{d.get('internal_api')} {d.get('version')}"
+    except Exception:
+        pass
+    return "unknown"
+
+
+def oracle_one_thread_seconds(groups):
+    """Seconds of the fp64 oracle for one matrix of the first group with BLAS held to one thread."""
+    import oracle
+    from synthetic import group_inputs, group_weights
+    from threadpoolctl import threadpool_limits
+    _, _, R, C = groups[0]
+    G = group_inputs(3, 0, 0, 1, R, C)[0].astype(np.float64)
+    W = group_weights(3, 0, 1, R, C)[0].astype(np.float64)
+    with threadpool_limits(limits=1, user_api="blas"):
+        t0 = time.perf_counter()
+        oracle.muon_step(W, G, np.zeros((R, C)), [QUINTIC] * K_ITERS, **HP)
+        return time.perf_counter() - t0
+
+
 def oracle_sample(groups, budget_s=12.0, max_per_group=96):
     """Time the fp64 oracle on whole matrices of one step until ~budget_s; returns steps/s and a label."""
     import oracle
@@ -430,7 +455,8 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, sample, spent = oracle_sample(groups)
         cpu = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample,
-               "seconds": round(spent, 2)}
+               "seconds": round(spent, 2), "blas": blas_vendor(),
+               "one_thread_seconds_per_matrix": {groups[0][0]: round(oracle_one_thread_seconds(groups), 3)}}
 
     mu = Muon(local)
     mu.set_coeffs([QUINTIC] * K_ITERS)

@@ -78,3 +78,10 @@ def test_kernel_hash_ignores_comments_but_not_code():
     assert bench._code_only(a) == bench._code_only(b) == "int x = 1;\nint y = 2;"
     assert bench._code_only(c) != bench._code_only(a)
     assert len(bench.gemm_source_hash()) == 16
+
+
+def test_cpu_baseline_reports_blas_and_a_one_thread_figure():
+    import bench
+    assert bench.blas_vendor() != ""
+    t = bench.oracle_one_thread_seconds([("small", 2, 96, 160)])
+    assert 0.0 < t < 30.0
