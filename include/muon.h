@@ -33,7 +33,11 @@
  *     (non-finite norm, a kernel wait that ran out) are reported by
  *     muon_get_status() after the stream has been synchronised.
  *   - Two calls on the same context must not run concurrently on different
- *     streams: they share the workspace.
+ *     streams: they share the workspace.  A context is used from one host
+ *     thread at a time; separate contexts are independent.
+ *   - Work a call puts on the context's internal streams (the uploads of
+ *     muon_step_groups_host) starts after what is already queued on `stream`
+ *     and joins back into `stream` before the call's last kernel.
  *   - No C++ exception crosses this interface.
  */
 #ifndef LIBMUON_MUON_H
