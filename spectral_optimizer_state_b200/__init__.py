@@ -8,4 +8,4 @@ from .binding import (  # noqa: F401
     SCALE_NONE, SCALE_RMS_MATCH, SCALE_SQRT_RATIO, AdamWGroup, Muon, MuonError, adamw_step, load_library,
     momentum_norm_noalloc, shape_scale,
 )
-from .optim import MuonAdamW, takes_muon  # noqa: F401,E402
+from .optim import MuonAdamW, takes_muon, torch_optimizer  # noqa: F401,E402

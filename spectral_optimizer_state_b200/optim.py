@@ -96,3 +96,39 @@ class MuonAdamW:
 
     def close(self):
         self.ctx.close()
+
+
+def torch_optimizer(named_params, mode="both", inner=None, **kw):
+    """A ``torch.optim.Optimizer`` over MuonAdamW: ``step()`` reads each parameter's ``.grad``.
+
+    named_params: (name, parameter) pairs, e.g. ``model.named_parameters()``.  Parameters whose
+    ``.grad`` is None at ``step()`` are given a zero gradient (their decay still applies, as in
+    ``torch.optim.AdamW``).  ``inner`` replaces the MuonAdamW instance (host-side tests only).
+    """
+    import torch
+
+    named = [(n, p) for n, p in named_params]
+
+    class MuonAdamWOptimizer(torch.optim.Optimizer):
+        def __init__(self):
+            super().__init__([p for _, p in named], defaults={})
+            self.inner = inner if inner is not None else MuonAdamW(named, mode=mode, **kw)
+            self.names = [n for n, _ in named]
+
+        @torch.no_grad()
+        def step(self, closure=None):
+            loss = None
+            if closure is not None:
+                with torch.enable_grad():
+                    loss = closure()
+            grads = {n: (p.grad if p.grad is not None else torch.zeros_like(p)) for n, p in named}
+            self.inner.step(grads)
+            return loss
+
+        def state_dict(self):
+            return self.inner.state_dict()
+
+        def load_state_dict(self, state):
+            self.inner.load_state_dict(state)
+
+    return MuonAdamWOptimizer()
