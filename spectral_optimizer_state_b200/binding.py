@@ -9,7 +9,6 @@ call raises.
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 from typing import Iterable, Sequence
 
@@ -427,11 +426,3 @@ def adamw_step(W, G, m, v, step, lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8, weigh
     AdamWGroup(W, G, m, v).step(step, lr=lr, beta1=beta1, beta2=beta2, eps=eps, weight_decay=weight_decay,
                                 stream=stream)
 
-
-def shape_scale(rows: int, cols: int, mode: int = SCALE_SQRT_RATIO) -> float:
-    """The scale the library applies (mirrors the C side, for callers' bookkeeping)."""
-    if mode == SCALE_NONE:
-        return 1.0
-    if mode == SCALE_RMS_MATCH:
-        return 0.2 * math.sqrt(max(rows, cols))
-    return math.sqrt(max(1.0, rows / cols))

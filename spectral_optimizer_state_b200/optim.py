@@ -50,6 +50,9 @@ class MuonAdamW:
                 z = lambda: torch.zeros(p.numel(), dtype=torch.float32, device=p.device)  # noqa: E731
                 self.adam.setdefault(p.dtype, []).append((name, p, z(), z()))
         self.t = 0
+        # AdamW bias correction counts the steps each parameter actually took (a parameter
+        # without a gradient in some step keeps its count, as in torch.optim.AdamW)
+        self.adam_t = {n: 0 for entries in self.adam.values() for (n, _, _, _) in entries}
 
     def muon_names(self):
         return [n for entries in self.muon.values() for (n, _, _) in entries]
@@ -58,25 +61,38 @@ class MuonAdamW:
         return [n for entries in self.adam.values() for (n, _, _, _) in entries]
 
     def step(self, grads, stream=None):
-        """grads: mapping name -> gradient tensor (same shape and dtype as the parameter)."""
+        """grads: mapping name -> gradient tensor (same shape and dtype as the parameter).
+
+        A parameter whose name is missing from ``grads`` or maps to None (frozen, or unused
+        in this backward pass) is left untouched: its weights get no decay, its Muon momentum
+        no step and its AdamW moments and step count stay as they are.
+        """
         self.t += 1
         groups = []
         for entries in self.muon.values():
-            for c0 in range(0, len(entries), MAX_BATCH):
-                chunk = entries[c0:c0 + MAX_BATCH]
+            live = [e for e in entries if grads.get(e[0]) is not None]
+            for c0 in range(0, len(live), MAX_BATCH):
+                chunk = live[c0:c0 + MAX_BATCH]
                 groups.append(([w for _, w, _ in chunk], [grads[n].contiguous() for n, _, _ in chunk],
                                [mbuf for _, _, mbuf in chunk]))
         for g0 in range(0, len(groups), MAX_GROUPS):
             self.ctx.step_groups(groups[g0:g0 + MAX_GROUPS], stream=stream, **self.muon_hp)
         for entries in self.adam.values():
-            W = [w.view(-1) for _, w, _, _ in entries]
-            G = [grads[n].contiguous().view(-1) for n, _, _, _ in entries]
-            adamw_step(W, G, [m for _, _, m, _ in entries], [v for _, _, _, v in entries], self.t,
-                       stream=stream, **self.adamw_hp)
+            by_count = OrderedDict()  # one launch per distinct step count (normally exactly one)
+            for e in entries:
+                if grads.get(e[0]) is None:
+                    continue
+                self.adam_t[e[0]] += 1
+                by_count.setdefault(self.adam_t[e[0]], []).append(e)
+            for t, live in by_count.items():
+                W = [w.view(-1) for _, w, _, _ in live]
+                G = [grads[n].contiguous().view(-1) for n, _, _, _ in live]
+                adamw_step(W, G, [m for _, _, m, _ in live], [v for _, _, _, v in live], t,
+                           stream=stream, **self.adamw_hp)
 
     def state_dict(self) -> dict:
         """Optimizer state by parameter name: Muon momentum, AdamW moments, and the step count."""
-        return {"t": self.t,
+        return {"t": self.t, "adamw_t": dict(self.adam_t),
                 "muon": {n: m.detach().clone() for entries in self.muon.values() for (n, _, m) in entries},
                 "adamw": {n: (m.detach().clone(), v.detach().clone())
                           for entries in self.adam.values() for (n, _, m, v) in entries}}
@@ -93,6 +109,8 @@ class MuonAdamW:
             adam[n][0].copy_(m)
             adam[n][1].copy_(v)
         self.t = int(state["t"])
+        counts = state.get("adamw_t", {n: self.t for n in adam})
+        self.adam_t = {n: int(counts[n]) for n in adam}
 
     def close(self):
         self.ctx.close()
@@ -102,8 +120,9 @@ def torch_optimizer(named_params, mode="both", inner=None, **kw):
     """A ``torch.optim.Optimizer`` over MuonAdamW: ``step()`` reads each parameter's ``.grad``.
 
     named_params: (name, parameter) pairs, e.g. ``model.named_parameters()``.  Parameters whose
-    ``.grad`` is None at ``step()`` are given a zero gradient (their decay still applies, as in
-    ``torch.optim.AdamW``).  ``inner`` replaces the MuonAdamW instance (host-side tests only).
+    ``.grad`` is None at ``step()`` are skipped, as ``torch.optim.AdamW`` skips them: no decay,
+    no momentum step, no moment update.  ``inner`` replaces the MuonAdamW instance (host-side
+    tests only).
     """
     import torch
 
@@ -121,7 +140,7 @@ def torch_optimizer(named_params, mode="both", inner=None, **kw):
             if closure is not None:
                 with torch.enable_grad():
                     loss = closure()
-            grads = {n: (p.grad if p.grad is not None else torch.zeros_like(p)) for n, p in named}
+            grads = {n: p.grad for n, p in named}
             self.inner.step(grads)
             return loss
 

@@ -75,12 +75,6 @@ def test_binding_validates_before_calling():
         binding._check_same([torch.zeros(2, 3)], (2, 2), torch.float32, "cpu", "W")
 
 
-def test_shape_scale_matches_readings():
-    assert sos.shape_scale(768, 1536) == 1.0
-    assert abs(sos.shape_scale(3352, 768) - (3352 / 768) ** 0.5) < 1e-12
-    assert sos.shape_scale(10, 10, sos.SCALE_NONE) == 1.0
-
-
 def declared_arities():
     """name -> number of parameters, from the prototypes in include/muon.h."""
     text = open(os.path.join(ROOT, "include", "muon.h")).read()
