@@ -2,7 +2,7 @@
 """Throughput of the Muon weight update on B200: full Mamba-2 130M optimizer steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload mamba2-130m|mamba2-2k]
+                    [--workload mamba2-130m|mamba2-2k] [--mode replicas|sharded]
 
 One step = the whole hot path over every in_proj (24 x 3352 x 768) and
 out_proj (24 x 768 x 1536) matrix of a Mamba-2 130M model, in one
@@ -14,7 +14,9 @@ resident in HBM; W and M persist across steps.
 
 Multi-GPU (torchrun): every rank runs its own full step on its own GPU (the
 matrices of different models/ranks are independent -- weak scaling, no
-collective on the data path); time is the max over ranks.
+collective on the data path); time is the max over ranks.  `--mode sharded`
+instead splits ONE model's step over the ranks by matrix ownership
+(reduce-scatter of gradients, owned step, all-gather of weights; strong scaling).
 
 Prints ONE JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
 (the baseline arm) on rank 0 over a bounded sample of the same workload.
@@ -88,6 +90,18 @@ def momentum_bytes(groups):
 def apply_bytes(groups):
     """Algorithmic bytes of the apply pass: O 2 (read) + W 2 (read) + W 2 (write) per element (bf16)."""
     return 6 * elements(groups)
+
+
+def step_bytes_algorithmic(groups):
+    """Algorithmic HBM bytes of the elementwise part of one step: G 2 + M 4 (read) + M 4 + U 2 (write)
+    + W 2 (read) + W 2 (write) = 16 B per element (the un-normalised U is the Newton-Schulz input)."""
+    return 16 * elements(groups)
+
+
+def roofline_step_ms(groups, tflops, hbm_gbs):
+    """Shortest possible step: the Newton-Schulz flops at the tensor peak plus the elementwise bytes at
+    the HBM peak (the two cannot overlap less than this, and need not overlap more)."""
+    return ns_flops(groups) / (tflops * 1e12) * 1e3 + step_bytes_algorithmic(groups) / (hbm_gbs * 1e9) * 1e3
 
 
 def load_peaks():
@@ -218,16 +232,29 @@ def make_inputs(groups, device, sets=GRAD_SETS, pinned_host=False):
     return Ws, Ms, Gsets, Ghost
 
 
+def device_spike_gradient(R, C, gen, device, std=1e-3, rank=4, factor=10.0, dtype=None):
+    """Gaussian N(0, std^2) bulk plus a rank-4 spike at `factor` times the bulk's top edge
+    std (sqrt(R) + sqrt(C)), drawn on the device (the host recipe's distribution, another stream)."""
+    import torch
+    g = torch.randn((R, C), device=device, generator=gen) * std
+    u, ru = torch.linalg.qr(torch.randn((R, rank), device=device, generator=gen))
+    v, rv = torch.linalg.qr(torch.randn((C, rank), device=device, generator=gen))
+    u = u * torch.sign(torch.diagonal(ru))
+    v = v * torch.sign(torch.diagonal(rv))
+    g += factor * std * (R ** 0.5 + C ** 0.5) * (u @ v.T)
+    return g.to(dtype if dtype is not None else torch.bfloat16)
+
+
 def make_inputs_device(groups, device, sets, pinned_host):
-    """Large workloads: seeded Gaussian weights and gradients drawn on the device
-    (the host generator would take minutes for 1.3 G elements), one gradient set."""
+    """Large workloads: seeded weights and spike gradients drawn on the device (the host generator
+    would take minutes for 1.3 G elements), one gradient set."""
     import torch
     gen = torch.Generator(device=device).manual_seed(3000)
     Ws, Ms, G1, Ghost = [], [], [], []
     for g, (_, L, R, C) in enumerate(groups):
         Ws.append([(torch.randn((R, C), device=device, generator=gen) * 0.02).to(torch.bfloat16) for _ in range(L)])
         Ms.append([torch.zeros((R, C), dtype=torch.float32, device=device) for _ in range(L)])
-        G1.append([(torch.randn((R, C), device=device, generator=gen) * 1e-3).to(torch.bfloat16) for _ in range(L)])
+        G1.append([device_spike_gradient(R, C, gen, device) for _ in range(L)])
         if pinned_host:
             Ghost.append([t.cpu().pin_memory() for t in G1[-1]])
     return Ws, Ms, [G1] * sets, Ghost
@@ -360,6 +387,84 @@ def measure_spectral(mu, Ws, Gs, Ms, groups, stream, peaks, pi_iters=8, min_iter
     }
 
 
+GEMM_KINDS = ("gram", "poly", "update", "ns_fused")
+
+
+def measure_fp32(mu, groups, device, stream, peaks, reps=20):
+    """The fp32 path on the same shapes: fp32 W and G, every Newton-Schulz operand split into three
+    bf16 planes and six plane products accumulated per contraction (so 6x the bf16 tensor work)."""
+    import torch
+    gen = torch.Generator(device=device).manual_seed(3100)
+    W = [[torch.randn((R, C), device=device, generator=gen) * 0.02 for _ in range(L)] for _, L, R, C in groups]
+    G = [[device_spike_gradient(R, C, gen, device, dtype=torch.float32) for _ in range(L)] for _, L, R, C in groups]
+    M = [[torch.zeros((R, C), device=device) for _ in range(L)] for _, L, R, C in groups]
+
+    def step():
+        mu.step_groups([(W[g], G[g], M[g]) for g in range(len(groups))], stream=stream, **HP)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    mu.profile_read(reset=True)
+    mu.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    mu.profile_enable(False)
+    prof = mu.profile_read(reset=True)
+    st, _ = mu.status()
+    assert st == 0, f"device status {st}"
+    ms = e0.elapsed_time(e1) / reps
+    ns_ms = sum(prof[k][1] for k in GEMM_KINDS) / reps
+    alg = ns_flops(groups)
+    plane_tf = 6 * alg / (ns_ms / 1e3) / 1e12
+    del W, G, M
+    return {"steps_per_s": 1000.0 / ms, "ms_per_step": ms, "ns_ms_per_step": ns_ms,
+            "ns_algorithmic_tflops": alg / (ns_ms / 1e3) / 1e12,
+            "plane_product_tflops": plane_tf,
+            "plane_product_frac_of_bf16_peak": {"burst": plane_tf / peaks["bf16_tflops"],
+                                                "sustained": plane_tf / peaks["bf16_tflops_sustained"]},
+            "steps": reps,
+            "note": ("fp32 W, G and M; each Newton-Schulz operand as three bf16 planes, six plane products "
+                     "per contraction on the bf16 tensor cores (6x the algorithmic flops)")}
+
+
+def steady_state_run(step_fn, stream, mu, gpu_id, ms_per_step, groups, peaks, min_s=1.0, max_steps=20000):
+    """The same step repeated for at least `min_s` seconds after the timed region, with the SM clock
+    sampled meanwhile: the steady state under the power cap, for reading the short timed region."""
+    import torch
+    n = int(min(max_steps, max(1, min_s * 1.2 * 1000.0 / max(ms_per_step, 1e-3))))
+    clocks = ClockSampler(gpu_id)
+    mu.profile_read(reset=True)
+    mu.profile_enable(True)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.25)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        step_fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    mu.profile_enable(False)
+    prof = mu.profile_read(reset=True)
+    ms = e0.elapsed_time(e1)
+    ns_ms = sum(prof[k][1] for k in GEMM_KINDS)
+    tf = ns_flops(groups) * n / (ns_ms / 1e3) / 1e12
+    out = {"steps": n, "seconds": ms / 1e3, "steps_per_s": n / (ms / 1e3), "ns_tflops": tf,
+           "ns_frac_of_bf16_peak": {"burst": tf / peaks["bf16_tflops"],
+                                    "sustained": tf / peaks["bf16_tflops_sustained"]},
+           "clocks": clk}
+    if clk.get("sm_mhz"):
+        # work per SM clock, which the power cap's clock changes do not move
+        out["ns_flop_per_sm_clock"] = ns_flops(groups) * n / (ns_ms / 1e3) / (clk["sm_mhz"] * 1e6) / 148
+    return out
+
+
 def run_reference(args, groups, rank):
     if rank != 0:
         return
@@ -382,14 +487,19 @@ def run_reference(args, groups, rank):
             per_step.append(dt)
     frac = len(mats) / total_mats
     value = frac * len(per_step) / sum(per_step)
-    labels = " + ".join(f"1 {m[1]}" for m in mats) + " matrix per step (oracle.muon_step, fp64 NumPy)"
+    labels = (" + ".join(f"1 {m[1]}" for m in mats) + f" matrix per step (oracle.muon_step, fp64 NumPy); "
+              f"steps/s extrapolated from {len(mats)} of the step's {total_mats} matrices")
     cores = blas_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / value, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_dict(args),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": labels},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": labels,
+                         "extrapolated": True, "matrices_timed_per_step": len(mats),
+                         "matrices_per_step": total_mats,
+                         "seconds_per_timed_step": sum(per_step) / max(len(per_step), 1)},
+        "extrapolated": True,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -401,6 +511,76 @@ def config_dict(args):
             "grad_sets_in_hbm": GRAD_SETS,
             "l2": "inputs larger than L2: each step streams G, M and W (%.2f GB)" % (
                 elements(WORKLOADS[args.workload]) * 8 / 1e9)}
+
+
+# ---------------------------------------------------------------- sharded data parallelism
+def run_sharded(args, groups, world, rank, local, device):
+    """Strong scaling of one model: ShardedMuon over `world` ranks -- an in-place NCCL reduce-scatter
+    of the gradients to the matrices' owners, the owners' libmuon step (the 1/N average folded into
+    its momentum pass), an in-place all-gather of the weights.  Each rank's local gradient is
+    refreshed from a resident copy before every step (a backward pass would write it there); only
+    opt.step() is timed, per part, with CUDA events on the launching stream."""
+    import torch
+    import torch.distributed as dist
+    from spectral_optimizer_state_b200.sharded import ShardedMuon
+    shapes = [(R, C) for _, L, R, C in groups for _ in range(L)]
+    opt = ShardedMuon(shapes, dtype=torch.bfloat16, device=device, coeffs=[QUINTIC] * K_ITERS, **HP)
+    gen = torch.Generator(device=device).manual_seed(3000)  # identical weights on every rank
+    for w in opt.weights:
+        w.copy_((torch.randn(w.shape, device=device, generator=gen) * 0.02).to(torch.bfloat16))
+    gen_r = torch.Generator(device=device).manual_seed(3300 + rank)  # this rank's own gradients
+    local_g = [device_spike_gradient(R, C, gen_r, device) for (R, C) in shapes]
+    stream = torch.cuda.current_stream()
+    parts = ("reduce_scatter", "local_step", "all_gather")
+    n_ev = args.steps * 4
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+
+    def refresh():
+        for g, src in zip(opt.grads, local_g):
+            g.copy_(src)
+
+    for _ in range(args.warmup):
+        refresh()
+        opt.step()
+    st, _ = opt.local_step.muon.status() if opt.owned else (0, [])
+    assert st == 0, f"device status {st}"
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        refresh()
+        marks = iter(evs[4 * i:4 * i + 4])
+        opt.step(mark=lambda phase: next(marks).record(stream))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    per_part = {p: 0.0 for p in parts}
+    for i in range(args.steps):
+        e = evs[4 * i:4 * i + 4]
+        for j, p in enumerate(parts):
+            per_part[p] += e[j].elapsed_time(e[j + 1])
+    ms_local = sum(per_part.values())
+    ms = max_over_ranks(ms_local, world, device)
+    parts_max = {p: max_over_ranks(v, world, device) / args.steps for p, v in per_part.items()}
+    nbytes = opt.owned_bytes()
+    line = {
+        "metric": METRIC, "value": args.steps / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(config_dict(args), parallelism=f"sharded x{world} (reduce-scatter -> owned step -> all-gather)"),
+        "matrices_per_s": args.steps / (ms / 1e3) * len(shapes),
+        "ms_per_step_by_part": parts_max,
+        "owned_matrices": len(opt.owned),
+        "bytes_per_rank": {"reduce_scatter_in": nbytes["reduce_scatter_bytes"],
+                           "all_gather_out": nbytes["all_gather_bytes"],
+                           "momentum_state": nbytes["momentum_bytes"]},
+        "note": "one model's step, total work fixed as N grows; timed region = opt.step() only",
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    opt.local_step.muon.close()
 
 
 # ---------------------------------------------------------------- ranks
@@ -427,6 +607,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-spectral", dest="spectral", action="store_false",
                     help="skip the power-iteration / min-singular / capped-step measurements")
+    ap.add_argument("--no-fp32", dest="fp32", action="store_false", help="skip the fp32-path measurement")
+    ap.add_argument("--mode", choices=["replicas", "sharded"], default="replicas",
+                    help="replicas: every rank steps its own model (weak scaling, the default); sharded: one "
+                         "model's step split over the ranks by matrix ownership (strong scaling)")
+    ap.add_argument("--no-long-run", dest="long_run", action="store_false",
+                    help="skip the >= 1 s steady-state repeat after the timed region")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     groups = WORKLOADS[args.workload]
@@ -449,6 +635,13 @@ def main():
     device = torch.device("cuda", local)
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+
+    if args.mode == "sharded":
+        run_sharded(args, groups, world, rank, local, device)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
 
     # cpu baseline first (rank 0, N = 1), before any pools or threads touch the GPU
     cpu = None
@@ -473,7 +666,7 @@ def main():
 
     peaks, peak_src = load_peaks()
     uuid = str(torch.cuda.get_device_properties(device).uuid)
-    clocks = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    clocks = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")  # during the timed region
 
     mu.profile_read(reset=True)
     mu.profile_enable(True)
@@ -499,6 +692,8 @@ def main():
     st, flags = mu.status()
     assert st == 0, f"device status {st}"
     ms = max_over_ranks(t0.elapsed_time(t1), world, device)
+    gpu_id = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+    steady = steady_state_run(step, stream, mu, gpu_id, ms / args.steps, groups, peaks) if args.long_run else None
 
     # e2e through the host-gradient entry point (pinned host G in, norms + flags out)
     e2e_steps = max(3, min(args.e2e_steps, args.steps))
@@ -548,12 +743,14 @@ def main():
         del aw, ag, am, av
 
     spectral = measure_spectral(mu, Ws, Gsets[0], Ms, groups, stream, peaks) if args.spectral else None
+    fp32 = None
+    if args.fp32 and args.workload == "mamba2-130m":
+        fp32 = measure_fp32(mu, groups, device, stream, peaks)
 
     n_mats = sum(L for _, L, _, _ in groups)
     steps_per_s = world * args.steps / (ms / 1e3)
-    gemm_kinds = ("gram", "poly", "update", "ns_fused")
-    gemm_launches = sum(prof[k][0] for k in gemm_kinds)
-    gemm_ms = sum(prof[k][1] for k in gemm_kinds)
+    gemm_launches = sum(prof[k][0] for k in GEMM_KINDS)
+    gemm_ms = sum(prof[k][1] for k in GEMM_KINDS)
     flops_timed = ns_flops(groups) * args.steps
     achieved_tf = flops_timed / (gemm_ms / 1e3) / 1e12
     burst, sustained = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
@@ -570,12 +767,20 @@ def main():
     mom_gbs = momentum_bytes(groups) * args.steps / (mom_ms / 1e3) / 1e9 if mom_ms > 0 else None
     h2d = sum(L * R * C * 2 for _, L, R, C in groups)
     d2h = n_mats * 8
+    roof_ms = roofline_step_ms(groups, peak, peaks["hbm_gbs"])
+    roof_steps = 1000.0 / roof_ms
 
     line = {
         "metric": METRIC, "value": steps_per_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(args),
         "matrices_per_s": steps_per_s * n_mats,
+        "step_roofline": {"ms": roof_ms, "steps_per_s": world * roof_steps, "matrices_per_s": world * roof_steps * n_mats,
+                          "tensor_peak_tflops": peak, "hbm_peak_gbs": peaks["hbm_gbs"],
+                          "ns_flops": ns_flops(groups), "elementwise_bytes": step_bytes_algorithmic(groups),
+                          "basis": "NS algorithmic flops at the tensor peak + 16 B/element at the HBM peak"},
+        "steps_per_s_frac": steps_per_s / (world * roof_steps),
+        "matrices_per_s_frac": steps_per_s / (world * roof_steps),
         "ns_tflops": achieved_tf,
         "ns_frac_of_bf16_peak": {"burst": achieved_tf / burst, "sustained": achieved_tf / sustained,
                                  "source": peak_src},
@@ -594,11 +799,14 @@ def main():
         "kernel_ms_per_step": {k: v[1] / args.steps for k, v in prof.items()},
         "adamw_kernel": adamw,
         "spectral": spectral,
+        "fp32_path": fp32,
+        "steady_state": steady,
         "cpu_baseline": cpu,
         "clocks": clk,
         "e2e": {"value": world * e2e_steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "entry": "muon_step_groups_host (pinned host G -> device, norms + flags -> host)"},
+                "entry": "muon_step_groups_host (pinned host G -> device, norms + flags -> host)",
+                "bound": "the host-to-device upload of every gradient each step (W and M stay resident)"},
         "gpu_launches": sum(v[0] for v in prof.values()),
     }
     if rank == 0:

@@ -3,6 +3,7 @@
  *
  * What is computed (per 2-D weight matrix W of shape rows x cols):
  *   M <- beta*M + G                      momentum buffer, fp32, updated in place
+ *                                        (G pre-scaled by hparams.grad_scale)
  *   U  = G + beta*M                      Nesterov look-ahead (U = M without it)
  *   X0 = U / (||U||_F + eps)             Frobenius normalisation
  *   X  = X0 or X0^T so that X is wide    (m = min(rows, cols) rows)
@@ -50,7 +51,7 @@
 extern "C" {
 #endif
 
-#define MUON_ABI_VERSION 1
+#define MUON_ABI_VERSION 2
 
 /* Largest number of Newton-Schulz iterations a coefficient table may hold. */
 #define MUON_MAX_ITERS 32
@@ -89,6 +90,10 @@ typedef struct {
   float eps;          /* added to ||U||_F before dividing, >= 0                        */
   int nesterov;       /* 1: U = G + beta*M (after the buffer update); 0: U = M         */
   int scale_mode;     /* muon_scale_mode                                               */
+  float grad_scale;   /* G is read as grad_scale*G (finite, > 0; 1 = as given).  A data- */
+                      /* parallel caller that reduce-scattered the SUM of N ranks'      */
+                      /* gradients passes 1/N to step on their average, with no extra   */
+                      /* pass over G.  0 (a struct from an older caller) is rejected.   */
 } muon_hparams;
 
 /* One group of same-shape matrices for muon_step_groups. */
@@ -277,6 +282,9 @@ muon_status muon_adamw_step(void* const* W, const void* const* G, float* const* 
  * elements of each matrix: batch * ceil(rows*cols / 8192) <= 65280, else
  * MUON_ERR_UNSUPPORTED_SHAPE.  The first call on a device looks the scratch
  * address up (cudaGetSymbolAddress), so make it before any stream capture.
+ * That address is kept for the life of the process: after cudaDeviceReset
+ * (or any destruction of the device's primary context) this entry point must
+ * not be called again on that device.
  * Every call shares the scratch: calls that overlap on the GPU race on it.
  * Asynchronous on `stream`; argument errors return before anything is queued. */
 muon_status muon_momentum_norm_noalloc(const void* const* G, float* const* M, float* nu, int batch,

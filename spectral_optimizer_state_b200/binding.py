@@ -52,7 +52,8 @@ class MuonError(RuntimeError):
 
 class Hparams(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_float), ("beta", ctypes.c_float), ("weight_decay", ctypes.c_float),
-                ("eps", ctypes.c_float), ("nesterov", ctypes.c_int), ("scale_mode", ctypes.c_int)]
+                ("eps", ctypes.c_float), ("nesterov", ctypes.c_int), ("scale_mode", ctypes.c_int),
+                ("grad_scale", ctypes.c_float)]
 
 
 class Profile(ctypes.Structure):
@@ -203,8 +204,10 @@ class Muon:
 
     # -------------------------------------------------------------- steps
     @staticmethod
-    def hparams(lr=0.02, beta=0.95, weight_decay=0.1, eps=1e-7, nesterov=True, scale_mode=SCALE_SQRT_RATIO):
-        return Hparams(float(lr), float(beta), float(weight_decay), float(eps), int(bool(nesterov)), int(scale_mode))
+    def hparams(lr=0.02, beta=0.95, weight_decay=0.1, eps=1e-7, nesterov=True, scale_mode=SCALE_SQRT_RATIO,
+                grad_scale=1.0):
+        return Hparams(float(lr), float(beta), float(weight_decay), float(eps), int(bool(nesterov)), int(scale_mode),
+                       float(grad_scale))
 
     def _group(self, W, G, M, g_device_type="cuda"):
         import torch

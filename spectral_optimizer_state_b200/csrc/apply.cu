@@ -8,6 +8,7 @@
 // scale and the decay taken from the pre-step W are the readings this library
 // uses for what the page leaves open.)
 //
+// One launch covers every group of a call (blocks cut into per-group ranges).
 // O is the last Newton-Schulz iterate in the workspace: wide orientation,
 // PLANES bf16 planes summed in fp32.  A wide W is updated row by row with
 // 16-byte vectors; a tall W (O stored transposed) goes through a 64 x 64
@@ -46,41 +47,47 @@ __device__ __forceinline__ float load1_planes(const uint16_t* o, long long ps, i
   return v;
 }
 
-// dst[0..8) <- f(dst, v), dst 16-byte aligned (bf16) or 32-byte (fp32).
+// The current W at dst[0..8) (16-byte aligned bf16, 32-byte fp32), when the pass applies a decay.
 template <bool F32>
-__device__ __forceinline__ void rmw8(void* dst, const float (&v)[8], bool apply, float decay, float lrs) {
+__device__ __forceinline__ void load8_w(const void* dst, int apply, float (&c)[8]) {
+  if (!apply) {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) c[t] = 0.f;
+    return;
+  }
+  if (F32) {
+    const float4* p = reinterpret_cast<const float4*>(dst);
+    const float4 a = p[0], b = p[1];
+    c[0] = a.x; c[1] = a.y; c[2] = a.z; c[3] = a.w; c[4] = b.x; c[5] = b.y; c[6] = b.z; c[7] = b.w;
+  } else {
+    const uint4 q = *reinterpret_cast<const uint4*>(dst);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      c[2 * i] = __uint_as_float(w[i] << 16);
+      c[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+}
+
+// dst[0..8) <- decay * c - lrs * v (apply) or v, in W's dtype.
+template <bool F32>
+__device__ __forceinline__ void store8_w(void* dst, const float (&v)[8], const float (&c)[8], int apply, float decay,
+                                         float lrs) {
+  float o[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) o[t] = apply ? fmaf(decay, c[t], -lrs * v[t]) : v[t];
   if (F32) {
     float4* p = reinterpret_cast<float4*>(dst);
-    float c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (apply) {
-      const float4 a = p[0], b = p[1];
-      c[0] = a.x; c[1] = a.y; c[2] = a.z; c[3] = a.w; c[4] = b.x; c[5] = b.y; c[6] = b.z; c[7] = b.w;
-    }
-    float o[8];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) o[t] = apply ? fmaf(decay, c[t], -lrs * v[t]) : v[t];
     p[0] = make_float4(o[0], o[1], o[2], o[3]);
     p[1] = make_float4(o[4], o[5], o[6], o[7]);
   } else {
-    uint4* p = reinterpret_cast<uint4*>(dst);
-    float c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (apply) {
-      const uint4 q = *p;
-      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        c[2 * i] = __uint_as_float(w[i] << 16);
-        c[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-      }
-    }
     uint32_t w[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float a = apply ? fmaf(decay, c[2 * i], -lrs * v[2 * i]) : v[2 * i];
-      const float b = apply ? fmaf(decay, c[2 * i + 1], -lrs * v[2 * i + 1]) : v[2 * i + 1];
-      w[i] = static_cast<uint32_t>(float_to_bf16_bits(a)) | (static_cast<uint32_t>(float_to_bf16_bits(b)) << 16);
-    }
-    *p = make_uint4(w[0], w[1], w[2], w[3]);
+    for (int i = 0; i < 4; ++i)
+      w[i] = static_cast<uint32_t>(float_to_bf16_bits(o[2 * i])) |
+             (static_cast<uint32_t>(float_to_bf16_bits(o[2 * i + 1])) << 16);
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -95,80 +102,164 @@ __device__ __forceinline__ void rmw1(void* dst, long long e, float v, bool apply
   }
 }
 
-// Wide W (rows <= cols): W(i, j) with O(i, j).  CAP: O - alpha u v^T (spectral cap).
-template <bool F32, bool VEC, bool CAP>
-__global__ void __launch_bounds__(kThreads) apply_wide_kernel(const __grid_constant__ ApplyParams p) {
-  const int l = blockIdx.y;
-  if (p.flags != nullptr && p.flags[l] != 0) return;
-  if (p.status != nullptr && (*p.status & kStatusTimeout)) return;  // the iterate is incomplete
-  void* w = p.w[l];
-  const uint16_t* o = p.o + static_cast<long long>(l) * p.o_mat;
-  const int C = p.cols;
-  if (VEC) {
-    const long long per_row = C / 8;
-    const long long total = static_cast<long long>(p.rows) * per_row;
-    const long long chunk = (total + p.nblk - 1) / p.nblk;
-    const long long beg = chunk * blockIdx.x;
-    const long long end = min(total, beg + chunk);
-    for (long long v = beg + threadIdx.x; v < end; v += kThreads) {
-      const long long i = v / per_row;
-      const int j = static_cast<int>(v - i * per_row) * 8;
-      float ov[8];
-      load8_planes(o + i * p.pitch + j, p.o_plane, p.planes, ov);
-      if (CAP) {
-        const float au = p.alpha[l] * p.cu[l][i];
+// 16-byte raw vectors of one wide-path step: O and W.  A bf16 W has a one-plane iterate (one
+// vector of each); an fp32 W has three planes and two vectors of W.
+template <bool F32>
+struct Raw8 {
+  static constexpr int kPlanes = F32 ? 3 : 1;
+  uint4 o[kPlanes];
+  uint4 w[F32 ? 2 : 1];
+};
+
+template <bool F32>
+__device__ __forceinline__ void load_raw8(Raw8<F32>& r, const uint16_t* o, long long ps, const void* w, int apply) {
 #pragma unroll
-        for (int t = 0; t < 8; ++t) ov[t] = fmaf(-au, p.cv[l][j + t], ov[t]);
-      }
-      char* dst = static_cast<char*>(w) + (i * C + j) * (F32 ? 4 : 2);
-      rmw8<F32>(dst, ov, p.apply, p.decay, p.lrs);
+  for (int p = 0; p < Raw8<F32>::kPlanes; ++p) r.o[p] = __ldcs(reinterpret_cast<const uint4*>(o + p * ps));
+  if (apply) {
+#pragma unroll
+    for (int i = 0; i < (F32 ? 2 : 1); ++i) r.w[i] = reinterpret_cast<const uint4*>(w)[i];
+  }
+}
+
+// Unpack a raw step: ov = sum of the O planes, cw = the current W (zeros when not applying).
+template <bool F32>
+__device__ __forceinline__ void unpack_raw8(const Raw8<F32>& r, int apply, float (&ov)[8], float (&cw)[8]) {
+#pragma unroll
+  for (int t = 0; t < 8; ++t) ov[t] = 0.f;
+#pragma unroll
+  for (int p = 0; p < Raw8<F32>::kPlanes; ++p) {
+    const uint32_t w[4] = {r.o[p].x, r.o[p].y, r.o[p].z, r.o[p].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ov[2 * i] += __uint_as_float(w[i] << 16);
+      ov[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+  if (!apply) {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) cw[t] = 0.f;
+  } else if (F32) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      cw[4 * i + 0] = __uint_as_float(r.w[i].x);
+      cw[4 * i + 1] = __uint_as_float(r.w[i].y);
+      cw[4 * i + 2] = __uint_as_float(r.w[i].z);
+      cw[4 * i + 3] = __uint_as_float(r.w[i].w);
     }
   } else {
-    const long long total = static_cast<long long>(p.rows) * C;
-    const long long chunk = (total + p.nblk - 1) / p.nblk;
-    const long long beg = chunk * blockIdx.x;
+    const uint32_t w[4] = {r.w[0].x, r.w[0].y, r.w[0].z, r.w[0].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      cw[2 * i] = __uint_as_float(w[i] << 16);
+      cw[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+}
+
+// Wide W (rows <= cols): W(i, j) with O(i, j).  CAP: O - alpha u v^T (spectral cap).
+// Vector path: 8 elements per thread step, two steps in flight (both steps' loads are
+// issued, as packed 16-byte vectors, before either is used).
+template <bool F32, bool CAP>
+__device__ __forceinline__ void wide_body(const ApplyParams& p, const ApplyGroup& q, int l, int b) {
+  void* w = p.w[q.mat0 + l];
+  const uint16_t* o = q.o + static_cast<long long>(l) * q.o_mat;
+  const int C = q.cols;
+  const bool cap = CAP && q.alpha != nullptr;
+  if (q.vec) {
+    const long long per_row = C / 8;
+    const long long total = static_cast<long long>(q.rows) * per_row;
+    const long long chunk = (total + q.nblk - 1) / q.nblk;
+    const long long beg = chunk * b;
+    const long long end = min(total, beg + chunk);
+    for (long long v0 = beg + threadIdx.x; v0 < end; v0 += 2 * kThreads) {
+      const long long v1 = v0 + kThreads;
+      const bool two = v1 < end;
+      long long iv[2];
+      int jv[2];
+      Raw8<F32> raw[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const long long v = h ? v1 : v0;
+        iv[h] = v / per_row;
+        jv[h] = static_cast<int>(v - iv[h] * per_row) * 8;
+        if (h == 0 || two)
+          load_raw8<F32>(raw[h], o + iv[h] * q.pitch + jv[h], q.o_plane,
+                         static_cast<char*>(w) + (iv[h] * C + jv[h]) * (F32 ? 4 : 2), p.apply);
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (h == 1 && !two) break;
+        float ov[8], cw[8];
+        unpack_raw8<F32>(raw[h], p.apply, ov, cw);
+        if (cap) {
+          const float au = q.alpha[l] * p.cu[q.mat0 + l][iv[h]];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) ov[t] = fmaf(-au, p.cv[q.mat0 + l][jv[h] + t], ov[t]);
+        }
+        store8_w<F32>(static_cast<char*>(w) + (iv[h] * C + jv[h]) * (F32 ? 4 : 2), ov, cw, p.apply, p.decay,
+                      q.lrs);
+      }
+    }
+  } else {
+    const long long total = static_cast<long long>(q.rows) * C;
+    const long long chunk = (total + q.nblk - 1) / q.nblk;
+    const long long beg = chunk * b;
     const long long end = min(total, beg + chunk);
     for (long long e = beg + threadIdx.x; e < end; e += kThreads) {
       const long long i = e / C;
       const int j = static_cast<int>(e - i * C);
-      float ov = load1_planes(o + i * p.pitch + j, p.o_plane, p.planes);
-      if (CAP) ov = fmaf(-p.alpha[l] * p.cu[l][i], p.cv[l][j], ov);
-      rmw1<F32>(w, e, ov, p.apply, p.decay, p.lrs);
+      float ov = load1_planes(o + i * q.pitch + j, q.o_plane, p.planes);
+      if (cap) ov = fmaf(-q.alpha[l] * p.cu[q.mat0 + l][i], p.cv[q.mat0 + l][j], ov);
+      rmw1<F32>(w, e, ov, p.apply, p.decay, q.lrs);
     }
   }
 }
 
 // Tall W (rows > cols): W(r, c) with O(c, r), through a 64 x 64 tile.
-template <bool F32, bool VEC, bool CAP>
-__global__ void __launch_bounds__(kThreads) apply_tall_kernel(const __grid_constant__ ApplyParams p) {
+template <bool F32, bool CAP>
+__device__ __forceinline__ void tall_body(const ApplyParams& p, const ApplyGroup& q, int l, int b) {
   __shared__ float tile[64][65];
-  const int l = blockIdx.y;
-  if (p.flags != nullptr && p.flags[l] != 0) return;
-  if (p.status != nullptr && (*p.status & kStatusTimeout)) return;  // the iterate is incomplete
-  void* w = p.w[l];
-  const uint16_t* o = p.o + static_cast<long long>(l) * p.o_mat;
-  const int R = p.rows, C = p.cols;
+  void* w = p.w[q.mat0 + l];
+  const uint16_t* o = q.o + static_cast<long long>(l) * q.o_mat;
+  const int R = q.rows, C = q.cols;
+  const bool cap = CAP && q.alpha != nullptr;
   const int tiles_c = (C + 63) / 64;
   const int ntiles = ((R + 63) / 64) * tiles_c;
   const int rr = threadIdx.x >> 3;       // 0..31
   const int cc = (threadIdx.x & 7) * 8;  // 0..56
-  for (int tt = blockIdx.x; tt < ntiles; tt += gridDim.x) {
+  for (int tt = b; tt < ntiles; tt += q.nblk) {
     const int r0 = (tt / tiles_c) * 64, c0 = (tt % tiles_c) * 64;
     // O rows c (= W columns), 8 consecutive W rows r per thread: O(c, r..r+7)
+    float ov[2][8];
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
       const int c = c0 + rr + 32 * pass;
       const int r = r0 + cc;
-      float ov[8];
       if (c < C && r < R) {
         // the wide pitch is >= round_up(R, 8) and r % 8 == 0: the 8-wide read stays in the row
-        load8_planes(o + static_cast<long long>(c) * p.pitch + r, p.o_plane, p.planes, ov);
+        load8_planes(o + static_cast<long long>(c) * q.pitch + r, q.o_plane, p.planes, ov[pass]);
       } else {
 #pragma unroll
-        for (int t = 0; t < 8; ++t) ov[t] = 0.f;
+        for (int t = 0; t < 8; ++t) ov[pass][t] = 0.f;
       }
+    }
+    // this thread's W rows for the write-back, read (packed) before the tile exchange
+    uint4 cw_raw[2][F32 ? 2 : 1];
+    const bool wvec = q.vec && c0 + cc < C;
 #pragma unroll
-      for (int t = 0; t < 8; ++t) tile[cc + t][rr + 32 * pass] = ov[t];
+    for (int pass = 0; pass < 2; ++pass) {
+      const int r = r0 + rr + 32 * pass;
+      if (wvec && r < R && p.apply) {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<char*>(w) +
+                                                          (static_cast<long long>(r) * C + c0 + cc) * (F32 ? 4 : 2));
+#pragma unroll
+        for (int i = 0; i < (F32 ? 2 : 1); ++i) cw_raw[pass][i] = src[i];
+      }
+    }
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
+      for (int t = 0; t < 8; ++t) tile[cc + t][rr + 32 * pass] = ov[pass][t];
     }
     __syncthreads();
 #pragma unroll
@@ -177,24 +268,24 @@ __global__ void __launch_bounds__(kThreads) apply_tall_kernel(const __grid_const
       const int r = r0 + rl;
       const int c = c0 + cc;
       if (r < R) {
-        float ov[8];
+        float v[8];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) ov[t] = tile[rl][cc + t];
-        if (CAP) {
-          const float au = p.alpha[l] * p.cu[l][r];
+        for (int t = 0; t < 8; ++t) v[t] = tile[rl][cc + t];
+        if (cap) {
+          const float au = q.alpha[l] * p.cu[q.mat0 + l][r];
 #pragma unroll
           for (int t = 0; t < 8; ++t)
-            if (c + t < C) ov[t] = fmaf(-au, p.cv[l][c + t], ov[t]);
+            if (c + t < C) v[t] = fmaf(-au, p.cv[q.mat0 + l][c + t], v[t]);
         }
-        if (VEC) {
-          if (c < C) {
-            char* dst = static_cast<char*>(w) + (static_cast<long long>(r) * C + c) * (F32 ? 4 : 2);
-            rmw8<F32>(dst, ov, p.apply, p.decay, p.lrs);
-          }
+        if (wvec) {
+          float cw[8];
+          load8_w<F32>(cw_raw[pass], p.apply, cw);
+          store8_w<F32>(static_cast<char*>(w) + (static_cast<long long>(r) * C + c) * (F32 ? 4 : 2), v, cw,
+                        p.apply, p.decay, q.lrs);
         } else {
 #pragma unroll
           for (int t = 0; t < 8; ++t)
-            if (c + t < C) rmw1<F32>(w, static_cast<long long>(r) * C + c + t, ov[t], p.apply, p.decay, p.lrs);
+            if (c + t < C) rmw1<F32>(w, static_cast<long long>(r) * C + c + t, v[t], p.apply, p.decay, q.lrs);
         }
       }
     }
@@ -203,31 +294,45 @@ __global__ void __launch_bounds__(kThreads) apply_tall_kernel(const __grid_const
 }
 
 template <bool F32, bool CAP>
-cudaError_t launch_typed(const ApplyParams& p, int batch, bool tall, bool vec, cudaStream_t s) {
-  dim3 grid(p.nblk, batch);
-  if (tall) {
-    if (vec) apply_tall_kernel<F32, true, CAP><<<grid, kThreads, 0, s>>>(p);
-    else apply_tall_kernel<F32, false, CAP><<<grid, kThreads, 0, s>>>(p);
-  } else {
-    if (vec) apply_wide_kernel<F32, true, CAP><<<grid, kThreads, 0, s>>>(p);
-    else apply_wide_kernel<F32, false, CAP><<<grid, kThreads, 0, s>>>(p);
-  }
-  return cudaGetLastError();
+__global__ void __launch_bounds__(kThreads) apply_kernel(const __grid_constant__ ApplyParams p) {
+  int gi = 0;
+  while (gi + 1 < p.ngroups && static_cast<int>(blockIdx.x) >= p.grp[gi + 1].block0) ++gi;
+  const ApplyGroup& q = p.grp[gi];
+  const int local = static_cast<int>(blockIdx.x) - q.block0;
+  const int l = local / q.nblk;
+  const int b = local - l * q.nblk;
+  if (q.flags != nullptr && q.flags[l] != 0) return;
+  if (p.status != nullptr && (*p.status & kStatusTimeout)) return;  // the iterate is incomplete
+  if (q.rows > q.cols) tall_body<F32, CAP>(p, q, l, b);
+  else wide_body<F32, CAP>(p, q, l, b);
 }
 
 }  // namespace
 
-cudaError_t launch_apply(const ApplyParams& p, int batch, bool w_f32, cudaStream_t stream) {
-  const bool tall = p.rows > p.cols;
-  bool vec = p.cols % 8 == 0;
-  for (int l = 0; l < batch && vec; ++l)
-    if (reinterpret_cast<uintptr_t>(p.w[l]) % 16) vec = false;
+cudaError_t launch_apply(ApplyParams& p, bool w_f32, cudaStream_t stream) {
+  if (p.ngroups < 1 || p.ngroups > MUON_MAX_GROUPS) return cudaErrorInvalidValue;
+  long long blocks = 0;
+  bool cap = false;
+  for (int gi = 0; gi < p.ngroups; ++gi) {
+    ApplyGroup& q = p.grp[gi];
+    q.block0 = static_cast<int>(blocks);
+    q.vec = q.cols % 8 == 0;
+    for (int l = 0; l < q.batch && q.vec; ++l)
+      if (reinterpret_cast<uintptr_t>(p.w[q.mat0 + l]) % 16) q.vec = 0;
+    cap = cap || q.alpha != nullptr;
+    blocks += static_cast<long long>(q.batch) * q.nblk;
+  }
+  if (blocks < 1 || blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(blocks));
   // the cap term is its own instantiation: the plain pass keeps its register allocation
-  if (p.alpha != nullptr)
-    return w_f32 ? launch_typed<true, true>(p, batch, tall, vec, stream)
-                 : launch_typed<false, true>(p, batch, tall, vec, stream);
-  return w_f32 ? launch_typed<true, false>(p, batch, tall, vec, stream)
-               : launch_typed<false, false>(p, batch, tall, vec, stream);
+  if (cap) {
+    if (w_f32) apply_kernel<true, true><<<grid, kThreads, 0, stream>>>(p);
+    else apply_kernel<false, true><<<grid, kThreads, 0, stream>>>(p);
+  } else {
+    if (w_f32) apply_kernel<true, false><<<grid, kThreads, 0, stream>>>(p);
+    else apply_kernel<false, false><<<grid, kThreads, 0, stream>>>(p);
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace muon

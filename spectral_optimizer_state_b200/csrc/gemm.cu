@@ -64,20 +64,35 @@ struct Tile {
   int pi, l, m0, n0, nw;
 };
 
+// What decoding a tile index needs of each problem, copied into shared memory at launch: the
+// parameter block (up to 30 problems of four tensor maps each) is far larger than the constant
+// cache, and every role decodes every tile.
+struct TileMeta {
+  int tile_base, tiles_per_matrix, L, M, N, sym, reverse, pad;
+};
+constexpr uint32_t META_BYTES = kMaxProblems * sizeof(TileMeta);
+
+__device__ __forceinline__ void load_meta(const GemmParams& P, TileMeta* meta) {
+  for (int i = threadIdx.x; i < P.nprob; i += blockDim.x) {
+    const GemmProblem& q = P.prob[i];
+    meta[i] = TileMeta{q.tile_base, q.tiles_per_matrix, q.L, q.M, q.N, q.sym, q.reverse, 0};
+  }
+}
+
 // Tile t of the launch: problem, matrix, first row (multiple of TM), first
 // column and width (a multiple of NG, at most BN).  Symmetric outputs start
 // each TM-row block at its diagonal block.
 template <int TM, int NG>
-__device__ __forceinline__ Tile decode_tile(const GemmParams& P, int t) {
+__device__ __forceinline__ Tile decode_tile(const TileMeta* meta, int nprob, int t) {
   Tile ti;
-  int lo = 0, hi = P.nprob - 1;  // last problem whose first tile is <= t
+  int lo = 0, hi = nprob - 1;  // last problem whose first tile is <= t
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (P.prob[mid].tile_base <= t) lo = mid;
+    if (meta[mid].tile_base <= t) lo = mid;
     else hi = mid - 1;
   }
   ti.pi = lo;
-  const GemmProblem& q = P.prob[ti.pi];
+  const TileMeta q = meta[ti.pi];
   const int local = t - q.tile_base;
   const int lm = local / q.tiles_per_matrix;
   int r = local - lm * q.tiles_per_matrix;
@@ -279,6 +294,8 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
   const uint32_t bar0 = stage_area + EPI_WARPS * STAGING_BYTES_PER_WARP;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + (bar0 - base) + 8 * NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  TileMeta* meta = reinterpret_cast<TileMeta*>(gbase + (bar0 - base) + BAR_BYTES);
+  load_meta(P, meta);
 
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
@@ -328,11 +345,11 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
       // latency hides behind the current tile's loads
       unsigned dep_seen = 0;
       if (blockIdx.x < P.total_tiles) {
-        const Tile t0 = decode_tile<BM, 64>(P, blockIdx.x);
+        const Tile t0 = decode_tile<BM, 64>(meta, P.nprob, blockIdx.x);
         if (P.prob[t0.pi].done_dep != nullptr) dep_seen = ld_relaxed_gpu(P.prob[t0.pi].done_dep + t0.l);
       }
       for (int t = blockIdx.x; ok && t < P.total_tiles; t += gridDim.x) {
-        const Tile ti = decode_tile<BM, 64>(P, t);
+        const Tile ti = decode_tile<BM, 64>(meta, P.nprob, t);
         const GemmProblem& q = P.prob[ti.pi];
         if (q.done_dep != nullptr) {
           // the previous phase of this matrix must have landed before it is read
@@ -346,7 +363,7 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
         }
         const int tn = t + gridDim.x;
         if (tn < P.total_tiles) {
-          const Tile tin = decode_tile<BM, 64>(P, tn);
+          const Tile tin = decode_tile<BM, 64>(meta, P.nprob, tn);
           dep_seen = P.prob[tin.pi].done_dep != nullptr ? ld_relaxed_gpu(P.prob[tin.pi].done_dep + tin.l) : 0u;
         }
         const int nk = q.k_tiles * q.nseg;
@@ -389,7 +406,7 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
       int local = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < P.total_tiles; t += gridDim.x, ++local) {
-        const Tile ti = decode_tile<BM, 64>(P, t);
+        const Tile ti = decode_tile<BM, 64>(meta, P.nprob, t);
         const GemmProblem& q = P.prob[ti.pi];
         const int acc = local & 1;
         const uint32_t aph = (local >> 1) & 1;
@@ -440,7 +457,7 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
     int sb = 0;
     int local = 0;
     for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++local) {
-      const Tile ti = decode_tile<BM, 64>(P, t);
+      const Tile ti = decode_tile<BM, 64>(meta, P.nprob, t);
       const GemmProblem& q = P.prob[ti.pi];
       const int acc = local & 1;
       const uint32_t aph = (local >> 1) & 1;
@@ -507,6 +524,8 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_c
   const uint32_t bar0 = stage_area + EPI_WARPS * STAGING_BYTES_PER_WARP;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + (bar0 - base) + 8 * PNUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  TileMeta* meta = reinterpret_cast<TileMeta*>(gbase + (bar0 - base) + PBAR_BYTES);
+  load_meta(P, meta);
 
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (PSTAGES + s); };
@@ -558,11 +577,11 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_c
       bool ok = true;
       unsigned dep_seen = 0;  // next tile's dependency counter, read a tile ahead
       if (pair < P.total_tiles) {
-        const Tile t0 = decode_tile<PBM, 128>(P, pair);
+        const Tile t0 = decode_tile<PBM, 128>(meta, P.nprob, pair);
         if (P.prob[t0.pi].done_dep != nullptr) dep_seen = ld_relaxed_gpu(P.prob[t0.pi].done_dep + t0.l);
       }
       for (int t = pair; ok && t < P.total_tiles; t += npairs) {
-        const Tile ti = decode_tile<PBM, 128>(P, t);
+        const Tile ti = decode_tile<PBM, 128>(meta, P.nprob, t);
         const GemmProblem& q = P.prob[ti.pi];
         if (q.done_dep != nullptr) {
           // both CTAs load, so both acquire the previous phase of this matrix
@@ -576,7 +595,7 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_c
         }
         const int tn = t + npairs;
         if (tn < P.total_tiles) {
-          const Tile tin = decode_tile<PBM, 128>(P, tn);
+          const Tile tin = decode_tile<PBM, 128>(meta, P.nprob, tn);
           dep_seen = P.prob[tin.pi].done_dep != nullptr ? ld_relaxed_gpu(P.prob[tin.pi].done_dep + tin.l) : 0u;
         }
         const int nk = q.k_tiles * q.nseg;
@@ -626,7 +645,7 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_c
       int local = 0;
       bool ok = true;
       for (int t = pair; ok && t < P.total_tiles; t += npairs, ++local) {
-        const Tile ti = decode_tile<PBM, 128>(P, t);
+        const Tile ti = decode_tile<PBM, 128>(meta, P.nprob, t);
         const GemmProblem& q = P.prob[ti.pi];
         const int acc = local & 1;
         const uint32_t aph = (local >> 1) & 1;
@@ -672,7 +691,7 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_c
     int sb = 0;
     int local = 0;
     for (int t = pair; t < P.total_tiles; t += npairs, ++local) {
-      const Tile ti = decode_tile<PBM, 128>(P, t);
+      const Tile ti = decode_tile<PBM, 128>(meta, P.nprob, t);
       const GemmProblem& q = P.prob[ti.pi];
       const int acc = local & 1;
       const uint32_t aph = (local >> 1) & 1;
@@ -711,8 +730,9 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_c
 }  // namespace
 
 size_t gemm_smem_bytes(int kind) {
-  if (kind == GEMM_PAIR) return PSTAGES * PSTAGE_BYTES + EPI_WARPS * STAGING_BYTES_PER_WARP + PBAR_BYTES + 1024;
-  return STAGES * STAGE_BYTES + EPI_WARPS * STAGING_BYTES_PER_WARP + BAR_BYTES + 1024;
+  if (kind == GEMM_PAIR)
+    return PSTAGES * PSTAGE_BYTES + EPI_WARPS * STAGING_BYTES_PER_WARP + PBAR_BYTES + META_BYTES + 1024;
+  return STAGES * STAGE_BYTES + EPI_WARPS * STAGING_BYTES_PER_WARP + BAR_BYTES + META_BYTES + 1024;
 }
 
 int gemm_tiles_per_matrix(int kind, int M, int N, int sym) {

@@ -11,19 +11,18 @@ namespace muon {
 
 // ------------------------------------------------------------------ K1
 // Momentum + Nesterov + Frobenius norm, writes X0 (un-normalised U) in the
-// wide orientation into the workspace as PLANES bf16 planes.
-struct MomentumParams {
-  const void* g[MUON_MAX_BATCH];  // rows x cols, bf16 or fp32
-  float* m[MUON_MAX_BATCH];       // rows x cols fp32 (null when no momentum)
+// wide orientation into the workspace as PLANES bf16 planes.  One launch
+// covers several same-dtype groups: the launch's blocks are cut into
+// consecutive ranges, one per group, `nblk` blocks per matrix.
+struct MomentumGroup {
+  int mat0;                       // first matrix of the group in the launch's pointer tables
+  int batch, rows, cols;          // of G / M (row-major)
+  int nblk;                       // blocks per matrix
+  int block0;                     // first block of the group in the launch
+  int vec;                        // 16-byte vector path (cols % 8 == 0, aligned pointers)
+  int pitch;                      // wide row pitch of x (elements), multiple of 8
   uint16_t* x;                    // [planes][batch][mrows][pitch] bf16 bits
-  long long x_plane;              // elements between planes
-  long long x_mat;                // elements between matrices
-  int pitch;                      // wide row pitch (elements), multiple of 8
-  int rows, cols;                 // of G / M (row-major)
-  float beta;
-  int nesterov;
-  float eps;
-  int nblk;                       // blocks per matrix (gridDim.x)
+  long long x_plane, x_mat;       // elements between planes / matrices
   float* partials;                // [batch][nblk]
   unsigned int* counters;         // [batch], zero between calls
   float* nu;                      // [batch] ||U||_F
@@ -32,32 +31,51 @@ struct MomentumParams {
   int* flags;                     // [batch]
 };
 
-// Launch K1 for one group; mode bits choose the kernel instance.
-cudaError_t launch_momentum(const MomentumParams& p, int batch, bool g_is_f32, bool momentum,
-                            int planes, cudaStream_t stream);
+struct MomentumParams {
+  const void* g[MUON_MAX_BATCH];  // rows x cols, bf16 or fp32 (launch-wide index)
+  float* m[MUON_MAX_BATCH];       // rows x cols fp32 (null when no momentum)
+  MomentumGroup grp[MUON_MAX_GROUPS];
+  int ngroups;
+  float beta;
+  float gscale;                   // G is read as gscale * G
+  int nesterov;
+  float eps;
+};
+
+// One launch over p.ngroups groups (at most MUON_MAX_BATCH matrices in all);
+// the caller fills every field but block0 / vec, which this sets.
+cudaError_t launch_momentum(MomentumParams& p, bool g_is_f32, bool momentum, int planes, cudaStream_t stream);
 
 // Number of blocks per matrix K1 uses for a rows x cols matrix.
 int momentum_blocks_per_matrix(int rows, int cols);
 
 // ------------------------------------------------------------------ K5 apply
-struct ApplyParams {
-  void* w[MUON_MAX_BATCH];  // caller matrices rows x cols (W, or Out)
+struct ApplyGroup {
+  int mat0, batch, rows, cols, nblk, block0, vec;
   const uint16_t* o;        // final iterate [planes][batch][m][pitch] bf16 bits (wide)
   long long o_plane, o_mat; // elements
-  int pitch, rows, cols, planes;
-  int apply;                // 1: W <- decay*W - lrs*O ; 0: W <- O
-  float decay, lrs;
-  const int* flags;         // matrices with a nonzero flag are left unchanged (null: none)
-  const int* status;        // device status word: nothing is written after a timeout (null: none)
-  int nblk;                 // blocks per matrix
-  // spectral cap (null alpha: none): O is replaced by O - alpha_l u_l v_l^T,
-  // u_l of length rows and v_l of length cols of W
-  const float* cu[MUON_MAX_BATCH];
-  const float* cv[MUON_MAX_BATCH];
-  const float* alpha;
+  int pitch;
+  float lrs;                // lr * s(rows, cols)
+  const int* flags;         // [batch] matrices with a nonzero flag are left unchanged (null: none)
+  const float* alpha;       // spectral cap coefficients [batch] (null: none)
 };
 
-cudaError_t launch_apply(const ApplyParams& p, int batch, bool w_f32, cudaStream_t stream);
+struct ApplyParams {
+  void* w[MUON_MAX_BATCH];  // caller matrices rows x cols (W, or Out), launch-wide index
+  // spectral cap: O is replaced by O - alpha_l u_l v_l^T, u_l of length rows and
+  // v_l of length cols of W (used by groups whose alpha is set)
+  const float* cu[MUON_MAX_BATCH];
+  const float* cv[MUON_MAX_BATCH];
+  ApplyGroup grp[MUON_MAX_GROUPS];
+  int ngroups;
+  int planes;
+  int apply;                // 1: W <- decay*W - lrs*O ; 0: W <- O
+  float decay;
+  const int* status;        // device status word: nothing is written after a timeout (null: none)
+};
+
+// One launch over p.ngroups groups of one W dtype; sets block0 / vec.
+cudaError_t launch_apply(ApplyParams& p, bool w_f32, cudaStream_t stream);
 
 // ------------------------------------------------------------------ spectral
 struct GemvParams {

@@ -1,12 +1,15 @@
 // K1: momentum, Nesterov look-ahead and the Frobenius norm in one HBM pass.
 //
 //   M <- beta*M + G ;  U = G + beta*M (or U = M) ;  nu = ||U||_F
+//   (G read as gscale * G: a data-parallel caller's 1/N average, folded into this pass)
 //
 // (Muon Meets Mamba: Spectral Optimization for State Space Models, abstract:
 // the update of each weight matrix is orthogonalised; the momentum, look-ahead
 // and normalisation that precede the Newton-Schulz iteration are the optimizer
 // state this pass maintains.)
 //
+// One launch covers every group of a call (blocks cut into per-group ranges),
+// so the step has one momentum launch instead of one per shape.
 // U is written, un-normalised, into the workspace in the WIDE orientation
 // (min(rows, cols) rows): a wide matrix is copied row by row with 16-byte
 // vectors, a tall one is transposed through a 64 x 64 shared-memory tile so
@@ -119,151 +122,176 @@ __device__ __forceinline__ T block_sum(T v, T* scratch) {
 }
 
 // Write this block's partial, and let the last block of the matrix finish the norm.
-__device__ void finish_norm(const MomentumParams& p, int l, float local) {
+__device__ void finish_norm(const MomentumGroup& q, float eps, int l, int b, float local) {
   __shared__ float fscratch[kThreads / 32];
   __shared__ double dscratch[kThreads / 32];
   __shared__ int is_last;
   const float blk = block_sum<float>(local, fscratch);
   if (threadIdx.x == 0) {
-    p.partials[static_cast<long long>(l) * p.nblk + blockIdx.x] = blk;
+    q.partials[static_cast<long long>(l) * q.nblk + b] = blk;
     __threadfence();
-    const unsigned prev = atomicAdd(&p.counters[l], 1u);
-    is_last = (prev == static_cast<unsigned>(p.nblk) - 1u);
+    const unsigned prev = atomicAdd(&q.counters[l], 1u);
+    is_last = (prev == static_cast<unsigned>(q.nblk) - 1u);
   }
   __syncthreads();
   if (!is_last) return;
   __threadfence();
   double acc = 0.0;
-  for (int b = threadIdx.x; b < p.nblk; b += kThreads)
-    acc += static_cast<double>(__ldcg(&p.partials[static_cast<long long>(l) * p.nblk + b]));
+  for (int i = threadIdx.x; i < q.nblk; i += kThreads)
+    acc += static_cast<double>(__ldcg(&q.partials[static_cast<long long>(l) * q.nblk + i]));
   const double tot = block_sum<double>(acc, dscratch);
   if (threadIdx.x == 0) {
     const float nu = static_cast<float>(sqrt(tot));
-    const float s1 = 1.0f / (nu + p.eps);
+    const float s1 = 1.0f / (nu + eps);
     const float s2 = s1 * s1;
-    p.nu[l] = nu;
-    p.scale1[l] = s1;
-    p.scale2[l] = s2;
+    q.nu[l] = nu;
+    q.scale1[l] = s1;
+    q.scale2[l] = s2;
     const bool ok = isfinite(nu) && isfinite(s2);
-    p.flags[l] = ok ? 0 : MUON_FLAG_NONFINITE;
-    p.counters[l] = 0u;  // ready for the next call
+    q.flags[l] = ok ? 0 : MUON_FLAG_NONFINITE;
+    q.counters[l] = 0u;  // ready for the next call
   }
 }
 
-// Wide matrices (rows <= cols): X(i, j) = U(i, j).  VEC: cols % 8 == 0 and
-// 16-byte aligned rows, 8 elements per thread step; else one element.
-template <typename TG, bool MOM, int PLANES, bool VEC>
-__global__ void __launch_bounds__(kThreads) momentum_wide_kernel(const __grid_constant__ MomentumParams p) {
-  const int l = blockIdx.y;
-  const TG* __restrict__ g = static_cast<const TG*>(p.g[l]);
-  float* __restrict__ m = MOM ? p.m[l] : nullptr;
-  uint16_t* __restrict__ x = p.x + static_cast<long long>(l) * p.x_mat;
-  const int C = p.cols;
+// M, U of 8 consecutive elements from G (and M): one vector step of the wide path.
+template <typename TG, bool MOM>
+__device__ __forceinline__ void lookahead8(const MomentumParams& p, float (&gv)[8], float (&mv)[8], float (&u)[8]) {
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    gv[t] *= p.gscale;
+    if (MOM) {
+      mv[t] = fmaf(p.beta, mv[t], gv[t]);
+      u[t] = p.nesterov ? fmaf(p.beta, mv[t], gv[t]) : mv[t];
+    } else {
+      u[t] = gv[t];
+    }
+  }
+}
+
+// Wide matrices (rows <= cols): X(i, j) = U(i, j).  Vector path: 8 elements per
+// thread step, two steps in flight (both loads issued before either is used).
+template <typename TG, bool MOM, int PLANES>
+__device__ __forceinline__ void wide_body(const MomentumParams& p, const MomentumGroup& q, int l, int b) {
+  const TG* __restrict__ g = static_cast<const TG*>(p.g[q.mat0 + l]);
+  float* __restrict__ m = MOM ? p.m[q.mat0 + l] : nullptr;
+  uint16_t* __restrict__ x = q.x + static_cast<long long>(l) * q.x_mat;
+  const int C = q.cols;
   float ss = 0.f;
-  if (VEC) {
+  if (q.vec) {
     const long long per_row = C / 8;
-    const long long total = static_cast<long long>(p.rows) * per_row;
-    const long long chunk = (total + p.nblk - 1) / p.nblk;
-    const long long beg = chunk * blockIdx.x;
+    const long long total = static_cast<long long>(q.rows) * per_row;
+    const long long chunk = (total + q.nblk - 1) / q.nblk;
+    const long long beg = chunk * b;
     const long long end = min(total, beg + chunk);
-    for (long long v = beg + threadIdx.x; v < end; v += kThreads) {
-      const long long i = v / per_row;
-      const int j = static_cast<int>(v - i * per_row) * 8;
-      const long long e = i * C + j;
-      float gv[8], u[8];
-      load8<TG>(g + e, gv);
-      if (MOM) {
-        float mv[8];
-        load8_f32(m + e, mv);
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          mv[t] = fmaf(p.beta, mv[t], gv[t]);
-          u[t] = p.nesterov ? fmaf(p.beta, mv[t], gv[t]) : mv[t];
-        }
-        store8_f32(m + e, mv);
-      } else {
-#pragma unroll
-        for (int t = 0; t < 8; ++t) u[t] = gv[t];
+    for (long long v0 = beg + threadIdx.x; v0 < end; v0 += 2 * kThreads) {
+      const long long v1 = v0 + kThreads;
+      const bool two = v1 < end;
+      const long long i0 = v0 / per_row, i1 = v1 / per_row;
+      const int j0 = static_cast<int>(v0 - i0 * per_row) * 8, j1 = static_cast<int>(v1 - i1 * per_row) * 8;
+      const long long e0 = i0 * C + j0, e1 = i1 * C + j1;
+      float ga[8], gb[8], ma[8], mb[8], ua[8], ub[8];
+      load8<TG>(g + e0, ga);
+      if (MOM) load8_f32(m + e0, ma);
+      if (two) {
+        load8<TG>(g + e1, gb);
+        if (MOM) load8_f32(m + e1, mb);
       }
+      lookahead8<TG, MOM>(p, ga, ma, ua);
+      if (MOM) store8_f32(m + e0, ma);
 #pragma unroll
-      for (int t = 0; t < 8; ++t) ss = fmaf(u[t], u[t], ss);
-      store8_planes<PLANES>(x + i * p.pitch + j, p.x_plane, u);
+      for (int t = 0; t < 8; ++t) ss = fmaf(ua[t], ua[t], ss);
+      store8_planes<PLANES>(x + i0 * q.pitch + j0, q.x_plane, ua);
+      if (two) {
+        lookahead8<TG, MOM>(p, gb, mb, ub);
+        if (MOM) store8_f32(m + e1, mb);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) ss = fmaf(ub[t], ub[t], ss);
+        store8_planes<PLANES>(x + i1 * q.pitch + j1, q.x_plane, ub);
+      }
     }
   } else {
-    const long long total = static_cast<long long>(p.rows) * C;
-    const long long chunk = (total + p.nblk - 1) / p.nblk;
-    const long long beg = chunk * blockIdx.x;
+    const long long total = static_cast<long long>(q.rows) * C;
+    const long long chunk = (total + q.nblk - 1) / q.nblk;
+    const long long beg = chunk * b;
     const long long end = min(total, beg + chunk);
     for (long long e = beg + threadIdx.x; e < end; e += kThreads) {
       const long long i = e / C;
       const int j = static_cast<int>(e - i * C);
-      const float gv = load_elem<TG>(g + e);
+      const float gv = p.gscale * load_elem<TG>(g + e);
       const float u = MOM ? momentum_lookahead(gv, m + e, p.beta, p.nesterov) : gv;
       ss = fmaf(u, u, ss);
-      store1_planes<PLANES>(x + i * p.pitch + j, p.x_plane, u);
+      store1_planes<PLANES>(x + i * q.pitch + j, q.x_plane, u);
     }
   }
-  finish_norm(p, l, ss);
+  finish_norm(q, p.eps, l, b, ss);
 }
 
 // Tall matrices (rows > cols): X(j, i) = U(i, j) through a 64 x 64 tile.
-template <typename TG, bool MOM, int PLANES, bool VEC>
-__global__ void __launch_bounds__(kThreads) momentum_tall_kernel(const __grid_constant__ MomentumParams p) {
+template <typename TG, bool MOM, int PLANES>
+__device__ __forceinline__ void tall_body(const MomentumParams& p, const MomentumGroup& q, int l, int b) {
   __shared__ float tile[64][65];
-  const int l = blockIdx.y;
-  const TG* __restrict__ g = static_cast<const TG*>(p.g[l]);
-  float* __restrict__ m = MOM ? p.m[l] : nullptr;
-  uint16_t* __restrict__ x = p.x + static_cast<long long>(l) * p.x_mat;
-  const int R = p.rows, C = p.cols;
+  const TG* __restrict__ g = static_cast<const TG*>(p.g[q.mat0 + l]);
+  float* __restrict__ m = MOM ? p.m[q.mat0 + l] : nullptr;
+  uint16_t* __restrict__ x = q.x + static_cast<long long>(l) * q.x_mat;
+  const int R = q.rows, C = q.cols;
   const int tiles_c = (C + 63) / 64;
   const int ntiles = ((R + 63) / 64) * tiles_c;
   const int rr = threadIdx.x >> 3;        // 0..31
   const int cc = (threadIdx.x & 7) * 8;   // 0..56
   float ss = 0.f;
-  for (int tt = blockIdx.x; tt < ntiles; tt += gridDim.x) {
+  for (int tt = b; tt < ntiles; tt += q.nblk) {
     const int r0 = (tt / tiles_c) * 64, c0 = (tt % tiles_c) * 64;
+    float u[2][8];
+    if (q.vec) {
+      // both passes' loads first: two rows of 8 in flight per thread
+      float gv[2][8], mv[2][8];
+      bool in[2];
 #pragma unroll
-    for (int pass = 0; pass < 2; ++pass) {
-      const int i = r0 + rr + 32 * pass;
-      const int j = c0 + cc;
-      float u[8];
-      if (VEC) {
-        if (i < R && j < C) {
+      for (int pass = 0; pass < 2; ++pass) {
+        const int i = r0 + rr + 32 * pass;
+        const int j = c0 + cc;
+        in[pass] = i < R && j < C;
+        if (in[pass]) {
           const long long e = static_cast<long long>(i) * C + j;
-          float gv[8];
-          load8<TG>(g + e, gv);
-          if (MOM) {
-            float mv[8];
-            load8_f32(m + e, mv);
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              mv[t] = fmaf(p.beta, mv[t], gv[t]);
-              u[t] = p.nesterov ? fmaf(p.beta, mv[t], gv[t]) : mv[t];
-            }
-            store8_f32(m + e, mv);
-          } else {
-#pragma unroll
-            for (int t = 0; t < 8; ++t) u[t] = gv[t];
-          }
-        } else {
-#pragma unroll
-          for (int t = 0; t < 8; ++t) u[t] = 0.f;
-        }
-      } else {
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          u[t] = 0.f;
-          if (i < R && j + t < C) {
-            const long long e = static_cast<long long>(i) * C + j + t;
-            const float gv = load_elem<TG>(g + e);
-            u[t] = MOM ? momentum_lookahead(gv, m + e, p.beta, p.nesterov) : gv;
-          }
+          load8<TG>(g + e, gv[pass]);
+          if (MOM) load8_f32(m + e, mv[pass]);
         }
       }
 #pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        if (in[pass]) {
+          lookahead8<TG, MOM>(p, gv[pass], mv[pass], u[pass]);
+          if (MOM) {
+            const long long e = static_cast<long long>(r0 + rr + 32 * pass) * C + c0 + cc;
+            store8_f32(m + e, mv[pass]);
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) u[pass][t] = 0.f;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        const int i = r0 + rr + 32 * pass;
+        const int j = c0 + cc;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          u[pass][t] = 0.f;
+          if (i < R && j + t < C) {
+            const long long e = static_cast<long long>(i) * C + j + t;
+            const float gv = p.gscale * load_elem<TG>(g + e);
+            u[pass][t] = MOM ? momentum_lookahead(gv, m + e, p.beta, p.nesterov) : gv;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
       for (int t = 0; t < 8; ++t) {
-        ss = fmaf(u[t], u[t], ss);
-        tile[rr + 32 * pass][cc + t] = u[t];
+        ss = fmaf(u[pass][t], u[pass][t], ss);
+        tile[rr + 32 * pass][cc + t] = u[pass][t];
       }
     }
     __syncthreads();
@@ -273,35 +301,35 @@ __global__ void __launch_bounds__(kThreads) momentum_tall_kernel(const __grid_co
       const int j = c0 + jl;
       const int i = r0 + cc;              // first of 8 consecutive W rows
       if (j < C && i < R) {
-        float u[8];
+        float uo[8];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) u[t] = tile[cc + t][jl];
+        for (int t = 0; t < 8; ++t) uo[t] = tile[cc + t][jl];
         // pitch >= round_up(R, 8) and i % 8 == 0, so the 8-wide store stays in the row
-        store8_planes<PLANES>(x + static_cast<long long>(j) * p.pitch + i, p.x_plane, u);
+        store8_planes<PLANES>(x + static_cast<long long>(j) * q.pitch + i, q.x_plane, uo);
       }
     }
     __syncthreads();
   }
-  finish_norm(p, l, ss);
+  finish_norm(q, p.eps, l, b, ss);
 }
 
+// Every group of the launch: the block range of group g starts at grp[g].block0.
 template <typename TG, bool MOM, int PLANES>
-cudaError_t launch_typed(const MomentumParams& p, int batch, bool tall, bool vec, cudaStream_t s) {
-  dim3 grid(p.nblk, batch);
-  if (tall) {
-    if (vec) momentum_tall_kernel<TG, MOM, PLANES, true><<<grid, kThreads, 0, s>>>(p);
-    else momentum_tall_kernel<TG, MOM, PLANES, false><<<grid, kThreads, 0, s>>>(p);
-  } else {
-    if (vec) momentum_wide_kernel<TG, MOM, PLANES, true><<<grid, kThreads, 0, s>>>(p);
-    else momentum_wide_kernel<TG, MOM, PLANES, false><<<grid, kThreads, 0, s>>>(p);
-  }
-  return cudaGetLastError();
+__global__ void __launch_bounds__(kThreads) momentum_kernel(const __grid_constant__ MomentumParams p) {
+  int gi = 0;
+  while (gi + 1 < p.ngroups && static_cast<int>(blockIdx.x) >= p.grp[gi + 1].block0) ++gi;
+  const MomentumGroup& q = p.grp[gi];
+  const int local = static_cast<int>(blockIdx.x) - q.block0;
+  const int l = local / q.nblk;
+  const int b = local - l * q.nblk;
+  if (q.rows > q.cols) tall_body<TG, MOM, PLANES>(p, q, l, b);
+  else wide_body<TG, MOM, PLANES>(p, q, l, b);
 }
 
-bool pointers_aligned(const MomentumParams& p, int batch, bool mom) {
-  for (int l = 0; l < batch; ++l) {
-    if (reinterpret_cast<uintptr_t>(p.g[l]) % 16) return false;
-    if (mom && reinterpret_cast<uintptr_t>(p.m[l]) % 16) return false;
+bool pointers_aligned(const MomentumParams& p, const MomentumGroup& q, bool mom) {
+  for (int l = 0; l < q.batch; ++l) {
+    if (reinterpret_cast<uintptr_t>(p.g[q.mat0 + l]) % 16) return false;
+    if (mom && reinterpret_cast<uintptr_t>(p.m[q.mat0 + l]) % 16) return false;
   }
   return true;
 }
@@ -320,18 +348,27 @@ int momentum_blocks_per_matrix(int rows, int cols) {
   return static_cast<int>(b < 1 ? 1 : (b > 4096 ? 4096 : b));
 }
 
-cudaError_t launch_momentum(const MomentumParams& p, int batch, bool g_is_f32, bool momentum,
-                            int planes, cudaStream_t stream) {
-  const bool tall = p.rows > p.cols;
-  const bool vec = (p.cols % 8 == 0) && pointers_aligned(p, batch, momentum);
+cudaError_t launch_momentum(MomentumParams& p, bool g_is_f32, bool momentum, int planes, cudaStream_t stream) {
+  if (p.ngroups < 1 || p.ngroups > MUON_MAX_GROUPS) return cudaErrorInvalidValue;
+  long long blocks = 0;
+  for (int gi = 0; gi < p.ngroups; ++gi) {
+    MomentumGroup& q = p.grp[gi];
+    q.block0 = static_cast<int>(blocks);
+    q.vec = (q.cols % 8 == 0) && pointers_aligned(p, q, momentum);
+    blocks += static_cast<long long>(q.batch) * q.nblk;
+  }
+  if (blocks < 1 || blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(blocks));
   if (g_is_f32) {
     if (planes != 3) return cudaErrorInvalidValue;
-    return momentum ? launch_typed<float, true, 3>(p, batch, tall, vec, stream)
-                    : launch_typed<float, false, 3>(p, batch, tall, vec, stream);
+    if (momentum) momentum_kernel<float, true, 3><<<grid, kThreads, 0, stream>>>(p);
+    else momentum_kernel<float, false, 3><<<grid, kThreads, 0, stream>>>(p);
+  } else {
+    if (planes != 1) return cudaErrorInvalidValue;
+    if (momentum) momentum_kernel<uint16_t, true, 1><<<grid, kThreads, 0, stream>>>(p);
+    else momentum_kernel<uint16_t, false, 1><<<grid, kThreads, 0, stream>>>(p);
   }
-  if (planes != 1) return cudaErrorInvalidValue;
-  return momentum ? launch_typed<uint16_t, true, 1>(p, batch, tall, vec, stream)
-                  : launch_typed<uint16_t, false, 1>(p, batch, tall, vec, stream);
+  return cudaGetLastError();
 }
 
 }  // namespace muon

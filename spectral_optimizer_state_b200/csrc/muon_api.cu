@@ -209,6 +209,7 @@ muon_status check_hparams(const muon_hparams* hp) {
   if (!finite(hp->lr) || !finite(hp->beta) || !finite(hp->weight_decay) || !finite(hp->eps))
     return MUON_ERR_INVALID_ARG;
   if (hp->eps < 0.f) return MUON_ERR_INVALID_ARG;
+  if (!finite(hp->grad_scale) || !(hp->grad_scale > 0.f)) return MUON_ERR_INVALID_ARG;
   if (hp->scale_mode < MUON_SCALE_SQRT_RATIO || hp->scale_mode > MUON_SCALE_RMS_MATCH)
     return MUON_ERR_INVALID_ARG;
   return MUON_OK;
@@ -418,35 +419,52 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
   for (auto& p : plans) total += p.batch;
   if (clear_status) MUON_CUDA(cudaMemsetAsync(c->d_status, 0, sizeof(int), s), "clear status");
 
-  // K1: momentum / look-ahead / norm of one group.
-  auto k1 = [&](const GroupPlan& p, cudaStream_t strm) -> muon_status {
-    MomentumParams mp;
-    std::memset(static_cast<void*>(&mp), 0, sizeof(mp));
-    for (int l = 0; l < p.batch; ++l) {
-      mp.g[l] = p.g[l];
-      mp.m[l] = step ? p.m[l] : nullptr;
+  // K1: momentum / look-ahead / norm over the groups `gs` (one launch per run of groups that share
+  // a dtype and fit the launch's pointer tables).
+  auto k1 = [&](const std::vector<int>& gs, cudaStream_t strm) -> muon_status {
+    size_t i = 0;
+    while (i < gs.size()) {
+      MomentumParams mp;
+      std::memset(static_cast<void*>(&mp), 0, sizeof(mp));
+      mp.beta = step ? hp->beta : 0.f;
+      mp.gscale = step ? hp->grad_scale : 1.f;
+      mp.nesterov = step ? hp->nesterov : 0;
+      mp.eps = eps;
+      const int f32 = plans[gs[i]].f32;
+      int mats = 0;
+      for (; i < gs.size() && mp.ngroups < MUON_MAX_GROUPS; ++i) {
+        const GroupPlan& p = plans[gs[i]];
+        if (p.f32 != f32 || mats + p.batch > MUON_MAX_BATCH) break;
+        MomentumGroup& q = mp.grp[mp.ngroups++];
+        q.mat0 = mats;
+        for (int l = 0; l < p.batch; ++l) {
+          mp.g[mats + l] = p.g[l];
+          mp.m[mats + l] = step ? p.m[l] : nullptr;
+        }
+        mats += p.batch;
+        q.batch = p.batch;
+        q.rows = p.rows;
+        q.cols = p.cols;
+        q.nblk = p.nblk;
+        q.pitch = p.pitch_n;
+        q.x = ws_at(c, p.off_x[0]);
+        q.x_plane = p.x_plane;
+        q.x_mat = p.x_mat;
+        q.partials = c->d_partials + p.part_off;
+        q.counters = c->d_counters + p.mat_off;
+        q.nu = c->d_nu + p.mat_off;
+        q.scale1 = c->d_s1 + p.mat_off;
+        q.scale2 = c->d_s2 + p.mat_off;
+        q.flags = c->d_flags + p.mat_off;
+      }
+      const int slot = prof_begin(c, MUON_KERNEL_MOMENTUM, strm);
+      MUON_CUDA(launch_momentum(mp, f32 != 0, step, f32 ? 3 : 1, strm), "momentum kernel");
+      prof_end(c, slot, strm);
     }
-    mp.x = ws_at(c, p.off_x[0]);
-    mp.x_plane = p.x_plane;
-    mp.x_mat = p.x_mat;
-    mp.pitch = p.pitch_n;
-    mp.rows = p.rows;
-    mp.cols = p.cols;
-    mp.beta = step ? hp->beta : 0.f;
-    mp.nesterov = step ? hp->nesterov : 0;
-    mp.eps = eps;
-    mp.nblk = p.nblk;
-    mp.partials = c->d_partials + p.part_off;
-    mp.counters = c->d_counters + p.mat_off;
-    mp.nu = c->d_nu + p.mat_off;
-    mp.scale1 = c->d_s1 + p.mat_off;
-    mp.scale2 = c->d_s2 + p.mat_off;
-    mp.flags = c->d_flags + p.mat_off;
-    const int slot = prof_begin(c, MUON_KERNEL_MOMENTUM, strm);
-    MUON_CUDA(launch_momentum(mp, p.batch, p.f32 != 0, step, p.planes, strm), "momentum kernel");
-    prof_end(c, slot, strm);
     return MUON_OK;
   };
+  std::vector<int> all_groups;
+  for (int g = 0; g < static_cast<int>(plans.size()); ++g) all_groups.push_back(g);
   // k Newton-Schulz iterations.  The single-CTA kernel runs every phase of
   // every group in one persistent launch (as many as fit in one parameter
   // block), ordered phase by phase; per-(phase, matrix) counters let a tile
@@ -552,48 +570,59 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
     return MUON_OK;
   };
 
-  // K5: scale + decoupled decay applied to W (or the plain copy to Out) for one group.
-  auto k5 = [&](const GroupPlan& p, cudaStream_t strm) -> muon_status {
-    ApplyParams ap;
-    std::memset(static_cast<void*>(&ap), 0, sizeof(ap));
-    for (int l = 0; l < p.batch; ++l) ap.w[l] = p.w[l];
-    ap.o = ws_at(c, p.off_x[c->k & 1]);
-    ap.o_plane = p.x_plane;
-    ap.o_mat = p.x_mat;
-    ap.pitch = p.pitch_n;
-    ap.rows = p.rows;
-    ap.cols = p.cols;
-    ap.planes = p.planes;
-    ap.apply = step ? 1 : 0;
-    if (step) {
-      ap.decay = 1.0f - hp->lr * hp->weight_decay;
-      ap.lrs = hp->lr * shape_scale(p.rows, p.cols, hp->scale_mode);
-      ap.flags = c->d_flags + p.mat_off;
-    }
-    ap.status = c->d_status;
-    ap.nblk = momentum_blocks_per_matrix(p.rows, p.cols);
-    if (cap != nullptr) {
-      for (int l = 0; l < p.batch; ++l) {
-        ap.cu[l] = cap->u[l];
-        ap.cv[l] = cap->v[l];
+  // K5: scale + decoupled decay applied to W (or the plain copy to Out) over the groups `gs`.
+  auto k5 = [&](const std::vector<int>& gs, cudaStream_t strm) -> muon_status {
+    size_t i = 0;
+    while (i < gs.size()) {
+      ApplyParams ap;
+      std::memset(static_cast<void*>(&ap), 0, sizeof(ap));
+      const int f32 = plans[gs[i]].f32;
+      ap.planes = plans[gs[i]].planes;
+      ap.apply = step ? 1 : 0;
+      ap.decay = step ? 1.0f - hp->lr * hp->weight_decay : 1.0f;
+      ap.status = c->d_status;
+      int mats = 0;
+      for (; i < gs.size() && ap.ngroups < MUON_MAX_GROUPS; ++i) {
+        const GroupPlan& p = plans[gs[i]];
+        if (p.f32 != f32 || mats + p.batch > MUON_MAX_BATCH) break;
+        ApplyGroup& q = ap.grp[ap.ngroups++];
+        q.mat0 = mats;
+        for (int l = 0; l < p.batch; ++l) {
+          ap.w[mats + l] = p.w[l];
+          if (cap != nullptr) {
+            ap.cu[mats + l] = cap->u[l];
+            ap.cv[mats + l] = cap->v[l];
+          }
+        }
+        mats += p.batch;
+        q.batch = p.batch;
+        q.rows = p.rows;
+        q.cols = p.cols;
+        q.nblk = momentum_blocks_per_matrix(p.rows, p.cols);
+        q.o = ws_at(c, p.off_x[c->k & 1]);
+        q.o_plane = p.x_plane;
+        q.o_mat = p.x_mat;
+        q.pitch = p.pitch_n;
+        q.lrs = step ? hp->lr * shape_scale(p.rows, p.cols, hp->scale_mode) : 0.f;
+        q.flags = step ? c->d_flags + p.mat_off : nullptr;
+        q.alpha = cap != nullptr ? cap->alpha : nullptr;
       }
-      ap.alpha = cap->alpha;
+      const int slot = prof_begin(c, MUON_KERNEL_APPLY, strm);
+      MUON_CUDA(launch_apply(ap, f32 != 0, strm), "apply kernel");
+      prof_end(c, slot, strm);
     }
-    const int slot = prof_begin(c, MUON_KERNEL_APPLY, strm);
-    MUON_CUDA(launch_apply(ap, p.batch, p.f32 != 0, strm), "apply kernel");
-    prof_end(c, slot, strm);
     return MUON_OK;
   };
 
   if (pipelined) {
     // caller's stream: K1(first), GEMM(first), GEMM(second) ..., K5(last)
     // side stream:     K1(second) ..., K5(first) ...
-    st = k1(plans[order[0]], s);
+    st = k1({order[0]}, s);
     if (st != MUON_OK) return st;
     MUON_CUDA(cudaEventRecord(c->ev_fork, s), "fork");
     MUON_CUDA(cudaStreamWaitEvent(c->side, c->ev_fork, 0), "fork");
     for (int i = 1; i < ng; ++i) {
-      st = k1(plans[order[i]], c->side);
+      st = k1({order[i]}, c->side);
       if (st != MUON_OK) return st;
       MUON_CUDA(cudaEventRecord(c->ev_k1[i], c->side), "momentum done");
     }
@@ -604,19 +633,17 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
       if (i + 1 < ng) {
         MUON_CUDA(cudaEventRecord(c->ev_gemm[i], s), "gemm done");
         MUON_CUDA(cudaStreamWaitEvent(c->side, c->ev_gemm[i], 0), "wait gemm");
-        st = k5(plans[order[i]], c->side);
+        st = k5({order[i]}, c->side);
         if (st != MUON_OK) return st;
       }
     }
-    st = k5(plans[order[ng - 1]], s);
+    st = k5({order[ng - 1]}, s);
     if (st != MUON_OK) return st;
     MUON_CUDA(cudaEventRecord(c->ev_join, c->side), "join");
     MUON_CUDA(cudaStreamWaitEvent(s, c->ev_join, 0), "join");
   } else {
-    for (auto& p : plans) {
-      st = k1(p, s);
-      if (st != MUON_OK) return st;
-    }
+    st = k1(all_groups, s);
+    if (st != MUON_OK) return st;
     for (const auto& items : launches) {
       st = run_launch(items, s);
       if (st != MUON_OK) return st;
@@ -644,10 +671,8 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
       cp.partial = static_cast<double*>(c->d_aux);
       MUON_CUDA(launch_cap_alpha(cp, p.batch, cap->alpha, s), "cap coefficient");
     }
-    for (auto& p : plans) {
-      st = k5(p, s);
-      if (st != MUON_OK) return st;
-    }
+    st = k5(all_groups, s);
+    if (st != MUON_OK) return st;
   }
   c->last_count = total;
   c->last_stream = s;
@@ -1031,6 +1056,8 @@ muon_status muon_power_iteration(muon_ctx* c, const void* const* W, float* const
   std::memset(static_cast<void*>(&gp), 0, sizeof(gp));
   gp.rows = rows;
   gp.cols = cols;
+  const bool f32 = dtype == MUON_F32;
+  for (int l = 0; l < batch; ++l) gp.w[l] = W[l];
   gp.rows_per_chunk = 64;
   gp.row_chunks = (rows + 63) / 64;
   const size_t part_bytes = align_up(sizeof(float) * batch * gp.row_chunks * cols, 256);
@@ -1038,8 +1065,6 @@ muon_status muon_power_iteration(muon_ctx* c, const void* const* W, float* const
   if (st != MUON_OK) return st;
   gp.partial = static_cast<float*>(c->d_aux);
   float* norms = reinterpret_cast<float*>(static_cast<char*>(c->d_aux) + part_bytes);
-  const bool f32 = dtype == MUON_F32;
-  for (int l = 0; l < batch; ++l) gp.w[l] = W[l];
   MUON_CUDA(launch_normalize(v, batch, cols, norms, s), "normalise start vector");
   for (int i = 0; i < iters; ++i) {
     for (int l = 0; l < batch; ++l) {

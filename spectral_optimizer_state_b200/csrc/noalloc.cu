@@ -70,10 +70,30 @@ __device__ __forceinline__ T block_sum(T v, T* scratch) {
   return r;
 }
 
+// 8 consecutive elements of G (16-byte aligned bf16, or 32-byte aligned fp32) as floats.
+template <bool F32>
+__device__ __forceinline__ void load_g8(const void* g, long long e, float (&v)[8]) {
+  if (F32) {
+    const float4* q = reinterpret_cast<const float4*>(static_cast<const float*>(g) + e);
+    const float4 a = __ldcs(q), b = __ldcs(q + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    const uint4 q = __ldcs(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(g) + e));
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+}
+
 // grid (nblk, batch): block b of matrix l updates elements
 // [b*chunk, (b+1)*chunk) of M and sums U^2; the last block of the matrix adds
-// the partials in a fixed order (fp64) and writes ||U||_F.
-template <bool F32>
+// the partials in a fixed order (fp64) and writes ||U||_F.  VEC: rows*cols is a
+// multiple of 8 and every pointer is 16-byte aligned, so each thread step moves
+// 8 elements with 16-byte loads and stores (chunks are whole vectors).
+template <bool F32, bool VEC>
 __global__ void __launch_bounds__(kThreads) momentum_norm_noalloc_kernel(const __grid_constant__ NoAllocParams p) {
   __shared__ float fs[kThreads / 32];
   __shared__ double ds[kThreads / 32];
@@ -81,16 +101,40 @@ __global__ void __launch_bounds__(kThreads) momentum_norm_noalloc_kernel(const _
   const int l = blockIdx.y;
   const void* g = p.g[l];
   float* m = p.m[l];
-  const long long chunk = (p.elems + p.nblk - 1) / p.nblk;
-  const long long beg = chunk * blockIdx.x;
-  const long long end = min(p.elems, beg + chunk);
   float ss = 0.f;
-  for (long long e = beg + threadIdx.x; e < end; e += kThreads) {
-    const float gv = load_g<F32>(g, e);
-    const float mn = fmaf(p.beta, m[e], gv);
-    m[e] = mn;
-    const float u = p.nesterov ? fmaf(p.beta, mn, gv) : mn;
-    ss = fmaf(u, u, ss);
+  if (VEC) {
+    const long long nv = p.elems / 8;
+    const long long chunk = (nv + p.nblk - 1) / p.nblk;
+    const long long beg = chunk * blockIdx.x;
+    const long long end = min(nv, beg + chunk);
+    for (long long v = beg + threadIdx.x; v < end; v += kThreads) {
+      const long long e = v * 8;
+      float gv[8], mv[8];
+      load_g8<F32>(g, e, gv);
+      const float4* mq = reinterpret_cast<const float4*>(m + e);
+      const float4 a = __ldcs(mq), b = __ldcs(mq + 1);
+      mv[0] = a.x; mv[1] = a.y; mv[2] = a.z; mv[3] = a.w; mv[4] = b.x; mv[5] = b.y; mv[6] = b.z; mv[7] = b.w;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        mv[t] = fmaf(p.beta, mv[t], gv[t]);
+        const float u = p.nesterov ? fmaf(p.beta, mv[t], gv[t]) : mv[t];
+        ss = fmaf(u, u, ss);
+      }
+      float4* mo = reinterpret_cast<float4*>(m + e);
+      __stcs(mo, make_float4(mv[0], mv[1], mv[2], mv[3]));
+      __stcs(mo + 1, make_float4(mv[4], mv[5], mv[6], mv[7]));
+    }
+  } else {
+    const long long chunk = (p.elems + p.nblk - 1) / p.nblk;
+    const long long beg = chunk * blockIdx.x;
+    const long long end = min(p.elems, beg + chunk);
+    for (long long e = beg + threadIdx.x; e < end; e += kThreads) {
+      const float gv = load_g<F32>(g, e);
+      const float mn = fmaf(p.beta, m[e], gv);
+      m[e] = mn;
+      const float u = p.nesterov ? fmaf(p.beta, mn, gv) : mn;
+      ss = fmaf(u, u, ss);
+    }
   }
   const float blk = block_sum<float>(ss, fs);
   if (threadIdx.x == 0) {
@@ -108,7 +152,9 @@ __global__ void __launch_bounds__(kThreads) momentum_norm_noalloc_kernel(const _
   if (threadIdx.x == 0) p.nu[l] = static_cast<float>(sqrt(tot));
 }
 
-// Device address of the scratch array, looked up once per device.
+// Device address of the scratch array, looked up once per device and kept for the life of the
+// process: it belongs to the device's context as it was at the lookup, so it must not be used
+// after that context is destroyed (cudaDeviceReset).
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
@@ -166,9 +212,17 @@ extern "C" muon_status muon_momentum_norm_noalloc(const void* const* G, float* c
     cudaGetLastError();
     return MUON_ERR_CUDA;
   }
+  bool vec = elems % 8 == 0;
+  for (int l = 0; l < batch && vec; ++l)
+    vec = reinterpret_cast<uintptr_t>(G[l]) % 16 == 0 && reinterpret_cast<uintptr_t>(M[l]) % 16 == 0;
   const dim3 grid(p.nblk, batch);
-  if (dtype == MUON_F32) momentum_norm_noalloc_kernel<true><<<grid, kThreads, 0, s>>>(p);
-  else momentum_norm_noalloc_kernel<false><<<grid, kThreads, 0, s>>>(p);
+  if (dtype == MUON_F32) {
+    if (vec) momentum_norm_noalloc_kernel<true, true><<<grid, kThreads, 0, s>>>(p);
+    else momentum_norm_noalloc_kernel<true, false><<<grid, kThreads, 0, s>>>(p);
+  } else {
+    if (vec) momentum_norm_noalloc_kernel<false, true><<<grid, kThreads, 0, s>>>(p);
+    else momentum_norm_noalloc_kernel<false, false><<<grid, kThreads, 0, s>>>(p);
+  }
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
 }

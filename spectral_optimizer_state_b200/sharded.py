@@ -6,7 +6,8 @@ orthogonalises the update of each weight matrix on its own).  With N
 data-parallel ranks that each hold a full gradient, one step is therefore
 
   1. reduce-scatter of the gradients: rank r receives the sum, over ranks, of
-     the gradients of the matrices it owns (then divides by N);
+     the gradients of the matrices it owns (the 1/N of the average is folded
+     into the momentum pass as libmuon's gradient scale, not a separate pass);
   2. the local Muon step (momentum, Newton-Schulz, apply) on the owned
      matrices only, through libmuon;
   3. all-gather of the updated weights, so every rank holds the new W.
@@ -85,8 +86,9 @@ class ShardedMuon:
     weights / grads: views (one per shape) into the flat weight / gradient
     buffers; write each step's local gradient into ``grads[i]`` and read the
     model's weights from ``weights[i]``.  ``local_step(groups, hp)`` performs
-    Muon steps on [(W list, G list, M list), ...] same-shape groups; it defaults
-    to libmuon on this rank's GPU and is replaceable only for host-side tests.
+    Muon steps on [(W list, G list, M list), ...] same-shape groups, reading each
+    G as ``hp["grad_scale"] * G``; it defaults to libmuon on this rank's GPU and is
+    replaceable only for host-side tests.
     """
 
     def __init__(self, shapes: Sequence[tuple], dtype=None, device=None, process_group=None,
@@ -165,16 +167,25 @@ class ShardedMuon:
         for i, m in state["momenta"].items():
             self.momenta[i].copy_(m)
 
-    def step(self, stream=None):
-        """One data-parallel Muon step: reduce-scatter G, local step on owned matrices, all-gather W."""
+    def step(self, stream=None, mark=None):
+        """One data-parallel Muon step: reduce-scatter G, local step on owned matrices, all-gather W.
+
+        ``mark(phase)``, if given, is called before each part ("reduce_scatter", "local_step",
+        "all_gather") and at the end ("end"), e.g. to record CUDA events for a per-part timing.
+        """
         import torch.distributed as dist
+        mark = mark or (lambda phase: None)
         mine_g = self.segment(self.flat_g)
+        mark("reduce_scatter")
         if self.world > 1:
             dist.reduce_scatter_tensor(mine_g, self.flat_g, op=dist.ReduceOp.SUM, group=self.group)
-            mine_g.mul_(1.0 / self.world)
         groups = [([self.weights[i] for i in idx], [self.grads[i] for i in idx], [self.momenta[i] for i in idx])
                   for idx in self._groups]
+        mark("local_step")
         if groups:
-            self.local_step(groups, self.hp, stream)
+            # the owned gradients hold the SUM over ranks; the step reads grad_scale * G
+            self.local_step(groups, dict(self.hp, grad_scale=1.0 / self.world), stream)
+        mark("all_gather")
         if self.world > 1:
             dist.all_gather_into_tensor(self.flat_w, self.segment(self.flat_w), group=self.group)
+        mark("end")

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(lib):
 def test_status_strings(lib):
     for code, name in binding.STATUS_NAMES.items():
         assert lib.muon_status_string(code).decode() == name
-    assert lib.muon_abi_version() == 1
+    assert lib.muon_abi_version() == 2
 
 
 def test_argument_errors_need_no_device(lib):
@@ -43,7 +43,7 @@ def test_argument_errors_need_no_device(lib):
     assert lib.muon_create(None, 0) == 1
     assert lib.muon_set_coeffs(None, None, 5) == 1
     assert lib.muon_get_coeffs(None, None, None) == 1
-    hp = binding.Hparams(0.02, 0.95, 0.1, 1e-7, 1, 0)
+    hp = binding.Hparams(0.02, 0.95, 0.1, 1e-7, 1, 0, 1.0)
     assert lib.muon_step(None, None, None, None, 1, 8, 8, 0, ctypes.byref(hp), None) == 1
     assert lib.muon_step_groups(None, None, 1, ctypes.byref(hp), None) == 1
     assert lib.muon_ns_orthogonalize(None, None, None, 1, 8, 8, 0, 1e-7, None) == 1

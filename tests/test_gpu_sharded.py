@@ -37,3 +37,28 @@ def test_sharded_world_one_equals_plain_grouped_step_bitwise():
         assert torch.equal(opt.weights[i], Wp[i])
         assert torch.equal(opt.momenta[i], Mp[i])
     assert opt.local_step.muon.status()[0] == 0
+
+
+def test_gradient_scale_equals_prescaled_gradients_bitwise():
+    """grad_scale = 1/2 on G gives exactly what grad_scale = 1 gives on G/2 (halving is exact in
+    bf16 and fp32), so the data-parallel 1/N average folded into the momentum pass changes nothing
+    but the extra pass; a zero scale (an uninitialised field) is rejected."""
+    import torch
+    from spectral_optimizer_state_b200 import Muon, MuonError
+    shape = (320, 192)
+    G = [torch.from_numpy(round_bf16(gaussian_spike(rng_for(650, i), *shape))).to(torch.bfloat16).cuda()
+         for i in range(3)]
+    W0 = [torch.from_numpy(round_bf16(weights(rng_for(651, i), *shape))).to(torch.bfloat16).cuda() for i in range(3)]
+    out = []
+    with Muon() as mu:
+        for gs, Gs in ((0.5, G), (1.0, [g / 2 for g in G])):
+            W = [w.clone() for w in W0]
+            M = [torch.zeros(shape, device="cuda") for _ in range(3)]
+            for _ in range(2):
+                mu.step(W, Gs, M, grad_scale=gs)
+            assert mu.status()[0] == 0
+            out.append((W, M))
+        with pytest.raises(MuonError):
+            mu.step([w.clone() for w in W0], G, [torch.zeros(shape, device="cuda") for _ in range(3)], grad_scale=0.0)
+    for a, b in zip(out[0][0] + out[0][1], out[1][0] + out[1][1]):
+        assert torch.equal(a, b)

@@ -48,10 +48,13 @@ def test_layout_is_owner_major_aligned_and_disjoint():
 
 
 def _oracle_step(groups, hp, stream=None):
+    """Stand-in for libmuon's step on CPU: reads G as grad_scale * G, as the library does."""
     import torch
+    hp = dict(hp)
+    gs = hp.pop("grad_scale", 1.0)
     for Ws, Gs, Ms in groups:
         for W, G, M in zip(Ws, Gs, Ms):
-            r = oracle.muon_step(W.numpy(), G.numpy(), M.numpy(), COEFFS, **hp)
+            r = oracle.muon_step(W.numpy(), gs * G.numpy(), M.numpy(), COEFFS, **hp)
             W.copy_(torch.from_numpy(r["W"]))
             M.copy_(torch.from_numpy(r["M"]))
 

@@ -1,5 +1,6 @@
 """The allocation-free momentum / norm entry point (for callers that cannot
-call cudaMalloc) against the same pass inside muon_step.
+call cudaMalloc) against the same pass inside muon_step, and against the fp64
+oracle's momentum and look-ahead norm.
 
 Collected last on purpose: the GPU test also passes after every other test
 has used the library in the same process.
@@ -9,6 +10,7 @@ import ctypes
 import numpy as np
 import pytest
 
+import oracle
 from synthetic import gaussian_spike, rng_for, round_bf16
 
 
@@ -40,6 +42,7 @@ def test_noalloc_matches_muon_step_two_calls(shape, dtype):
     M_ref = [torch.zeros(shape, dtype=torch.float32, device="cuda") for _ in range(batch)]
     M_new = [torch.zeros(shape, dtype=torch.float32, device="cuda") for _ in range(batch)]
     nu = torch.full((batch,), -1.0, dtype=torch.float32, device="cuda")
+    M_or = [np.zeros(shape) for _ in range(batch)]
     for call in range(2):
         G = []
         for l in range(batch):
@@ -55,4 +58,10 @@ def test_noalloc_matches_muon_step_two_calls(shape, dtype):
             b = M_ref[l].double().cpu().numpy()
             assert np.linalg.norm(a - b) <= 1e-6 * np.linalg.norm(b)
             assert abs(float(nu[l]) - ref_nu[l]) <= 1e-5 * ref_nu[l]
+            # and against the fp64 oracle's momentum and look-ahead norm
+            g64 = G[l].double().cpu().numpy()
+            M_or[l] = oracle.momentum_update(M_or[l], g64, beta)
+            nu_or = oracle.frobenius_norm(oracle.nesterov_lookahead(g64, M_or[l], beta))
+            assert np.linalg.norm(a - M_or[l]) <= 1e-6 * np.linalg.norm(M_or[l])
+            assert abs(float(nu[l]) - nu_or) <= 1e-5 * nu_or
     mu.close()
