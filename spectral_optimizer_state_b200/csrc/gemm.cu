@@ -212,16 +212,42 @@ __device__ __forceinline__ void stage_as_col(uint32_t buf, int lane, const uint1
   for (int t = 0; t < 32; ++t) st_shared_u16(buf + stage_offset(t, lane >> 3) + 2 * (lane & 7), b[t]);
 }
 
+// This lane's 32 values, already packed as 16 bf16 pairs, become row `lane` of the staging tile.
+__device__ __forceinline__ void stage_packed_row(uint32_t buf, int lane, const uint32_t (&w)[16]) {
+#pragma unroll
+  for (int h = 0; h < 4; ++h)
+    st_shared_v4(buf + stage_offset(lane, h), w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]);
+}
+
+__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// This lane's 32 values (packed pairs) become column `lane` of the staging tile (the mirror).
+// Lanes 2k and 2k+1 trade their pairs, so each writes whole 32-bit words holding columns 2k and
+// 2k+1: the even lane rows 2i, the odd lane rows 2i+1.  Each store then fills two adjacent 64-byte
+// rows (one shared-memory wavefront) instead of one 2-byte slot per lane and row.
+__device__ __forceinline__ void stage_packed_col(uint32_t buf, int lane, const uint32_t (&w)[16]) {
+  const bool odd = lane & 1;
+  const int col = lane & ~1;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t other = __shfl_xor_sync(0xffffffffu, w[i], 1);
+    // even lane: (own low, other low) = row 2i; odd lane: (other high, own high) = row 2i + 1
+    const uint32_t word = odd ? __byte_perm(other, w[i], 0x7632) : __byte_perm(w[i], other, 0x5410);
+    st_shared_u32(buf + stage_offset(2 * i + (odd ? 1 : 0), col >> 3) + 2 * (col & 7), word);
+  }
+}
+
 // One 32 x 32 TMA store from the warp's next staging buffer.  Lane 0 first
 // makes sure the store that last read this buffer has finished reading it.
-template <bool AS_COL>
+template <typename Stage>
 __device__ __forceinline__ void store_chunk(const CUtensorMap* map, uint32_t stage_base, int& sb, int lane,
-                                            const uint16_t (&b)[32], int x, int y, int l, int p) {
+                                            Stage&& stage, int x, int y, int l, int p) {
   const uint32_t buf = stage_base + static_cast<uint32_t>(sb) * 2048u;
   if (lane == 0) bulk_wait_group_read<1>();
   __syncwarp();
-  if (AS_COL) stage_as_col(buf, lane, b);
-  else stage_as_row(buf, lane, b);
+  stage(buf);
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
@@ -270,15 +296,33 @@ __device__ __forceinline__ void epilogue_warp_tile(const GemmProblem& q, const T
         if (j0 + i == row) v[i] += q.diag;
     }
     const bool mirror = q.sym && (j0 >= mirror_from);
-    for (int p = 0; p < q.planes; ++p) {
-      uint16_t b[32];
+    if (q.planes == 1) {
+      // one bf16 plane: round to nearest even two values at a time, already packed for the stores
+      uint32_t w[16];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        b[i] = float_to_bf16_bits(v[i]);
-        v[i] -= bf16_bits_to_float(b[i]);  // residual for the next plane
+      for (int i = 0; i < 16; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        w[i] = *reinterpret_cast<const uint32_t*>(&h);
       }
-      store_chunk<false>(&q.tmOut, my_stage, sb, lane, b, j0, row0, ti.l, p);
-      if (mirror) store_chunk<true>(&q.tmOut, my_stage, sb, lane, b, row0, j0, ti.l, p);
+      store_chunk(&q.tmOut, my_stage, sb, lane, [&](uint32_t buf) { stage_packed_row(buf, lane, w); }, j0, row0,
+                  ti.l, 0);
+      if (mirror)
+        store_chunk(&q.tmOut, my_stage, sb, lane, [&](uint32_t buf) { stage_packed_col(buf, lane, w); }, row0, j0,
+                    ti.l, 0);
+    } else {
+      for (int p = 0; p < q.planes; ++p) {
+        uint16_t b[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          b[i] = float_to_bf16_bits(v[i]);
+          v[i] -= bf16_bits_to_float(b[i]);  // residual for the next plane
+        }
+        store_chunk(&q.tmOut, my_stage, sb, lane, [&](uint32_t buf) { stage_as_row(buf, lane, b); }, j0, row0,
+                    ti.l, p);
+        if (mirror)
+          store_chunk(&q.tmOut, my_stage, sb, lane, [&](uint32_t buf) { stage_as_col(buf, lane, b); }, row0, j0,
+                      ti.l, p);
+      }
     }
   }
   if (!released) release();
@@ -419,6 +463,13 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
         const uint32_t idesc = instr_desc_bf16(BM, ti.nw, q.b_mn_major != 0);
         const int nk = q.k_tiles * q.nseg;
         const bool diag_tile = q.sym && ti.m0 == ti.n0;
+        // Descriptors of stage 0, k-step 0; a stage or k-step only moves the start address (the
+        // low 14 bits, in 16-byte units, which never carry: shared addresses are below 256 KB).
+        // K-major operands advance 32 bytes per 16-deep k-step, the MN-major B 16 rows of 128 bytes.
+        const uint64_t a_desc0 = smem_desc_sw128(base, 16u, 1024u);
+        const uint64_t b_desc0 = q.b_mn_major ? smem_desc_sw128(base + A_BYTES, MNMAJ_BOX_BYTES, 1024u)
+                                              : smem_desc_sw128(base + A_BYTES, 16u, 1024u);
+        const uint32_t b_step = q.b_mn_major ? (2048u >> 4) : (32u >> 4);
         for (int kk = 0; kk < nk; ++kk, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -428,16 +479,13 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
           }
           int pa, pb;
           segment_planes(q.nseg, kk / q.k_tiles, pa, pb);
-          const uint32_t sb = base + s * STAGE_BYTES + A_BYTES;
+          const uint32_t stage_off = static_cast<uint32_t>(s) * (STAGE_BYTES >> 4);
           // K-major, 128-byte swizzle: B's rows 0..127 are laid out exactly as an A tile
-          const uint32_t sa = diag_tile && pa == pb ? sb : base + s * STAGE_BYTES;
+          const uint64_t ad = a_desc0 + stage_off + (diag_tile && pa == pb ? (A_BYTES >> 4) : 0u);
+          const uint64_t bd = b_desc0 + stage_off;
 #pragma unroll
-          for (int k4 = 0; k4 < BK / 16; ++k4) {
-            const uint64_t ad = smem_desc_sw128(sa + 32u * k4, 16u, 1024u);
-            const uint64_t bd = q.b_mn_major ? smem_desc_sw128(sb + 2048u * k4, MNMAJ_BOX_BYTES, 1024u)
-                                             : smem_desc_sw128(sb + 32u * k4, 16u, 1024u);
-            tc_mma_bf16(d_tmem, ad, bd, idesc, (kk | k4) != 0 ? 1u : 0u);
-          }
+          for (int k4 = 0; k4 < BK / 16; ++k4)
+            tc_mma_bf16(d_tmem, ad + 2u * k4, bd + b_step * k4, idesc, (kk | k4) != 0 ? 1u : 0u);
           tc_commit(empty_bar(s));
         }
         if (ok) tc_commit(tfull_bar(acc));

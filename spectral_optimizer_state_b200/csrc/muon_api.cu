@@ -1058,6 +1058,26 @@ muon_status muon_power_iteration(muon_ctx* c, const void* const* W, float* const
   gp.cols = cols;
   const bool f32 = dtype == MUON_F32;
   for (int l = 0; l < batch; ++l) gp.w[l] = W[l];
+  bool fused = cols % 8 == 0 && cols <= power_pass_max_cols();
+  for (int l = 0; l < batch && fused; ++l)
+    if (reinterpret_cast<uintptr_t>(W[l]) % 16) fused = false;
+  if (fused) {
+    // one pass over W per iteration (power_pass_kernel); 64 rows per block
+    const int rpb = 64;
+    const int nblk = (rows + rpb - 1) / rpb;
+    const size_t part_bytes = align_up(sizeof(float) * batch * nblk * cols, 256);
+    muon_status st = ensure_aux(c, part_bytes + sizeof(float) * batch * (nblk + (cols + 255) / 256));
+    if (st != MUON_OK) return st;
+    gp.partial = static_cast<float*>(c->d_aux);
+    float* tsq = reinterpret_cast<float*>(static_cast<char*>(c->d_aux) + part_bytes);
+    for (int l = 0; l < batch; ++l) {
+      gp.x[l] = v[l];
+      gp.y[l] = u[l];
+    }
+    for (int i = 0; i < iters; ++i)
+      MUON_CUDA(launch_power_iteration_fused(gp, batch, f32, tsq, nblk, rpb, sigma, s), "power iteration");
+    return MUON_OK;
+  }
   gp.rows_per_chunk = 64;
   gp.row_chunks = (rows + 63) / 64;
   const size_t part_bytes = align_up(sizeof(float) * batch * gp.row_chunks * cols, 256);

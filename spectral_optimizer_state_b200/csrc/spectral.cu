@@ -126,6 +126,155 @@ __global__ void __launch_bounds__(kThreads) gemv_cols_reduce_kernel(const __grid
   p.y[l][c] = s;
 }
 
+// 8 consecutive elements of W as packed 16-byte vectors (bf16: one, fp32: two) and their values.
+template <bool F32>
+struct Raw8w {
+  uint4 q[F32 ? 2 : 1];
+};
+
+template <bool F32>
+__device__ __forceinline__ void load_raw(const void* base, long long e, Raw8w<F32>& r) {
+  const uint4* p = F32 ? reinterpret_cast<const uint4*>(static_cast<const float*>(base) + e)
+                       : reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + e);
+#pragma unroll
+  for (int i = 0; i < (F32 ? 2 : 1); ++i) r.q[i] = p[i];
+}
+
+template <bool F32>
+__device__ __forceinline__ void unpack_raw(const Raw8w<F32>& r, float (&x)[8]) {
+  if (F32) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      x[4 * i] = __uint_as_float(r.q[i].x);
+      x[4 * i + 1] = __uint_as_float(r.q[i].y);
+      x[4 * i + 2] = __uint_as_float(r.q[i].z);
+      x[4 * i + 3] = __uint_as_float(r.q[i].w);
+    }
+  } else {
+    const uint32_t w[4] = {r.q[0].x, r.q[0].y, r.q[0].z, r.q[0].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+}
+
+// t_r = W[r, :] . v and z += t_r W[r, :] for one row held (packed) in registers.
+template <bool F32, int NV>
+__device__ __forceinline__ float power_row(const Raw8w<F32> (&w)[NV], const float* vs, int C, int lane,
+                                           float (&z)[NV][8]) {
+  float dot = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = 8 * lane + 256 * i;
+    if (c < C) {
+      float x[8];
+      unpack_raw<F32>(w[i], x);
+      // 16-byte reads of v: a lane's 8 values are contiguous, so scalar reads would be 8-way
+      // bank conflicts across the warp
+      const float4 va = *reinterpret_cast<const float4*>(vs + c);
+      const float4 vb = *reinterpret_cast<const float4*>(vs + c + 4);
+      const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+      for (int t = 0; t < 8; ++t) dot = fmaf(x[t], vv[t], dot);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = 8 * lane + 256 * i;
+    if (c < C) {
+      float x[8];
+      unpack_raw<F32>(w[i], x);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) z[i][t] = fmaf(dot, x[t], z[i][t]);
+    }
+  }
+  return dot;
+}
+
+// One pass over the rows of W for a whole power iteration.  With t = W v, the
+// next iterate's W^T u is W^T t / |t|, and W^T t = sum_r t_r W[r, :]: each warp
+// loads its rows once (two rows in flight, NV packed 16-byte vectors per lane
+// each), forms t_r against v (staged in shared memory) and adds t_r W[r, :] to its
+// running sum z.  t goes to u (un-normalised), a fixed-order tree over the warps
+// gives one partial z per block, and each block writes its partial sum of t_r^2.
+// Requires cols % 8 == 0, 16-byte aligned rows and cols <= 256 * NV.
+template <bool F32, int NV>
+__global__ void __launch_bounds__(kThreads) power_pass_kernel(const __grid_constant__ GemvParams p,
+                                                              int rows_per_block, float* tsq_partial) {
+  extern __shared__ float sm[];
+  float* vs = sm;                         // [cols]
+  float* zs = sm + p.cols;                // [warps][cols]
+  constexpr int kWarps = kThreads / 32;
+  const int l = blockIdx.y;
+  const float* x = p.x[l];
+  const int C = p.cols;
+  for (int c = threadIdx.x; c < C; c += kThreads) vs[c] = x[c];
+  __syncthreads();
+  const void* W = p.w[l];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r_beg = blockIdx.x * rows_per_block;
+  const int r_end = min(p.rows, r_beg + rows_per_block);
+  float z[NV][8];
+#pragma unroll
+  for (int i = 0; i < NV; ++i)
+#pragma unroll
+    for (int t = 0; t < 8; ++t) z[i][t] = 0.f;
+  float tsq = 0.f;
+  for (int r0 = r_beg + warp; r0 < r_end; r0 += 2 * kWarps) {
+    const int r1 = r0 + kWarps;
+    const bool two = r1 < r_end;
+    Raw8w<F32> w0[NV], w1[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = 8 * lane + 256 * i;
+      if (c < C) {
+        load_raw<F32>(W, static_cast<long long>(r0) * C + c, w0[i]);
+        if (two) load_raw<F32>(W, static_cast<long long>(r1) * C + c, w1[i]);
+      }
+    }
+    const float t0 = power_row<F32, NV>(w0, vs, C, lane, z);
+    if (lane == 0) p.y[l][r0] = t0;
+    tsq = fmaf(t0, t0, tsq);
+    if (two) {
+      const float t1 = power_row<F32, NV>(w1, vs, C, lane, z);
+      if (lane == 0) p.y[l][r1] = t1;
+      tsq = fmaf(t1, t1, tsq);
+    }
+  }
+  // warps' z into shared memory, then a fixed-order sum over the warps
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = 8 * lane + 256 * i;
+    if (c < C) {
+      float4* d = reinterpret_cast<float4*>(zs + warp * C + c);
+      d[0] = make_float4(z[i][0], z[i][1], z[i][2], z[i][3]);
+      d[1] = make_float4(z[i][4], z[i][5], z[i][6], z[i][7]);
+    }
+  }
+  __syncthreads();
+  float* out = p.partial + (static_cast<long long>(l) * gridDim.x + blockIdx.x) * C;
+  for (int c = threadIdx.x; c < C; c += kThreads) {
+    float a = 0.f;
+#pragma unroll
+    for (int k = 0; k < kWarps; ++k) a += zs[k * C + c];
+    out[c] = a;
+  }
+  // the warps' sums of t_r^2 (every lane holds its warp's), in warp order
+  __shared__ float tq[kWarps];
+  if (lane == 0) tq[warp] = tsq;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float a = 0.f;
+#pragma unroll
+    for (int k = 0; k < kWarps; ++k) a += tq[k];
+    tsq_partial[static_cast<long long>(l) * gridDim.x + blockIdx.x] = a;
+  }
+}
+
 template <typename T>
 __device__ __forceinline__ T block_sum(T v, T* scratch) {
 #pragma unroll
@@ -141,6 +290,59 @@ __device__ __forceinline__ T block_sum(T v, T* scratch) {
     for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
   }
   return r;
+}
+
+// z = the pass's block partials summed in block order (one thread per column, the loads
+// eight blocks ahead of the additions); z goes to v un-normalised and each block writes
+// its partial sum of z^2.  grid (column blocks, batch).
+__global__ void __launch_bounds__(kThreads) power_reduce_kernel(const __grid_constant__ GemvParams p, int nblk,
+                                                                float* zsq_partial) {
+  __shared__ double scratch[kThreads / 32];
+  const int l = blockIdx.y;
+  const int C = p.cols;
+  const int c = blockIdx.x * kThreads + threadIdx.x;
+  double zz = 0.0;
+  if (c < C) {
+    const float* part = p.partial + static_cast<long long>(l) * nblk * C + c;
+    float a = 0.f;
+    int b = 0;
+    for (; b + 8 <= nblk; b += 8) {
+      float q[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) q[k] = part[static_cast<long long>(b + k) * C];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) a += q[k];
+    }
+    for (; b < nblk; ++b) a += part[static_cast<long long>(b) * C];
+    const_cast<float*>(p.x[l])[c] = a;
+    zz = static_cast<double>(a) * a;
+  }
+  const double tot = block_sum<double>(zz, scratch);
+  if (threadIdx.x == 0) zsq_partial[static_cast<long long>(l) * gridDim.x + blockIdx.x] = static_cast<float>(tot);
+}
+
+// u = t / |t|, v = z / |z|, sigma = |z| / |t| (= |W^T u|), from the partial sums of t^2 and z^2
+// (summed in order by every block).  A zero t leaves u, v at zero and sigma 0.
+// grid (element blocks over max(rows, cols), batch).
+__global__ void __launch_bounds__(kThreads) power_scale_kernel(const __grid_constant__ GemvParams p, int nblk,
+                                                               const float* tsq_partial, int zblk,
+                                                               const float* zsq_partial, float* sigma) {
+  __shared__ float s_inv_t, s_inv_z;
+  const int l = blockIdx.y;
+  if (threadIdx.x == 0) {
+    double tt = 0.0, zz = 0.0;
+    for (int b = 0; b < nblk; ++b) tt += tsq_partial[static_cast<long long>(l) * nblk + b];
+    for (int b = 0; b < zblk; ++b) zz += zsq_partial[static_cast<long long>(l) * zblk + b];
+    const float nt = static_cast<float>(sqrt(tt));
+    const float nz = static_cast<float>(sqrt(zz));
+    s_inv_t = nt > 0.f ? 1.0f / nt : 0.f;
+    s_inv_z = nz > 0.f ? 1.0f / nz : 0.f;
+    if (blockIdx.x == 0) sigma[l] = nt > 0.f ? nz / nt : 0.f;
+  }
+  __syncthreads();
+  const int i = blockIdx.x * kThreads + threadIdx.x;
+  if (i < p.cols) const_cast<float*>(p.x[l])[i] *= s_inv_z;
+  if (i < p.rows) p.y[l][i] *= s_inv_t;
 }
 
 struct VecParams {
@@ -301,6 +503,48 @@ cudaError_t launch_gemv_cols(const GemvParams& p, int batch, bool f32, cudaStrea
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   gemv_cols_reduce_kernel<<<dim3((p.cols + kThreads - 1) / kThreads, batch), kThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+int power_pass_max_cols() { return 256 * 8; }
+
+cudaError_t launch_power_iteration_fused(GemvParams& p, int batch, bool f32, float* tsq_partial, int nblk,
+                                         int rows_per_block, float* sigma, cudaStream_t s) {
+  const int nv = (p.cols + 255) / 256;
+  if (p.cols % 8 != 0 || nv < 1 || nv > 8) return cudaErrorInvalidValue;
+  const size_t smem = sizeof(float) * p.cols * (1 + kThreads / 32);
+  const dim3 grid(nblk, batch);
+  cudaError_t e = cudaSuccess;
+#define MUON_POWER_CASE(NVV)                                                                          \
+  case NVV: {                                                                                        \
+    auto kern = f32 ? power_pass_kernel<true, NVV> : power_pass_kernel<false, NVV>;                 \
+    if (smem > 48 * 1024) {                                                                          \
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)); \
+      if (e != cudaSuccess) return e;                                                                \
+    }                                                                                                \
+    kern<<<grid, kThreads, smem, s>>>(p, rows_per_block, tsq_partial);                               \
+    break;                                                                                           \
+  }
+  switch (nv) {
+    MUON_POWER_CASE(1)
+    MUON_POWER_CASE(2)
+    MUON_POWER_CASE(3)
+    MUON_POWER_CASE(4)
+    MUON_POWER_CASE(5)
+    MUON_POWER_CASE(6)
+    MUON_POWER_CASE(7)
+    MUON_POWER_CASE(8)
+  }
+#undef MUON_POWER_CASE
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int zblk = (p.cols + kThreads - 1) / kThreads;
+  float* zsq_partial = tsq_partial + static_cast<long long>(batch) * nblk;
+  power_reduce_kernel<<<dim3(zblk, batch), kThreads, 0, s>>>(p, nblk, zsq_partial);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int eblk = (std::max(p.rows, p.cols) + kThreads - 1) / kThreads;
+  power_scale_kernel<<<dim3(eblk, batch), kThreads, 0, s>>>(p, nblk, tsq_partial, zblk, zsq_partial, sigma);
   return cudaGetLastError();
 }
 

@@ -8,8 +8,9 @@ from tests.gpu_common import BF16_TOL, F32_TOL, rel_f, to_device, to_numpy
 
 pytestmark = pytest.mark.gpu
 
-# wide, tall, ragged (scalar paths: cols % 8 != 0), and one past the 48 KB shared-memory default
-SHAPES = [(96, 200, 3), (200, 96, 2), (77, 45, 2), (45, 77, 1), (64, 13000, 1)]
+# wide, tall, ragged (scalar paths: cols % 8 != 0), one past the 48 KB shared-memory default, and
+# the single-pass kernel at 6 and 8 vectors per lane (the out_proj width and its 2048 limit)
+SHAPES = [(96, 200, 3), (200, 96, 2), (77, 45, 2), (45, 77, 1), (64, 13000, 1), (768, 1536, 2), (300, 2048, 2)]
 
 
 def _spiked(rows, cols, batch, seed, dtype):
