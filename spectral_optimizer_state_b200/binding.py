@@ -329,6 +329,18 @@ class Muon:
                                        ctypes.byref(h), ctypes.c_void_p(alpha.data_ptr()), _stream_handle(stream))
         self._check(st, "muon_step_capped")
 
+    # -------------------------------------------------------------- plans (checked and marshalled once)
+    def step_plan(self, groups, **hp):
+        """A StepPlan for a fixed set of groups [(W list, G list, M list), ...]: the tensors are
+        checked and their pointers marshalled once, so each step is one C call (the tensors must
+        stay alive and in place; G is read afresh every step)."""
+        return StepPlan(self, groups, **hp)
+
+    def spectral_plan(self, W, u, v, sigma, y=None, sigma_min=None):
+        """A SpectralPlan for fixed tensors: power_iteration(iters) and min_singular(iters) as one
+        C call each (same arguments as the methods of the same names)."""
+        return SpectralPlan(self, W, u, v, sigma, y, sigma_min)
+
     # -------------------------------------------------------------- status
     def status(self):
         """(status code, per-matrix flags) of the last call; synchronises its stream."""
@@ -358,6 +370,66 @@ class Muon:
         p = Profile()
         self._check(self.lib.muon_profile_read(self.handle, ctypes.byref(p), int(bool(reset))), "muon_profile_read")
         return {k: (p.launches[i], p.ms[i]) for i, k in enumerate(KERNEL_KINDS)}
+
+
+class StepPlan:
+    """muon_step_groups over a fixed list of groups, validated and marshalled once."""
+
+    def __init__(self, muon: "Muon", groups, **hp):
+        self.muon = muon
+        gs, self._keep = [], []
+        for (W, G, M) in groups:
+            g, k = muon._group(W, G, M)
+            gs.append(g)
+            self._keep.append((k, list(W), list(G), list(M)))  # pointer arrays and the tensors
+        self._arr = (Group * len(gs))(*gs)
+        self._n = len(gs)
+        self._hp = Muon.hparams(**hp)
+
+    def __call__(self, stream=None):
+        st = self.muon.lib.muon_step_groups(self.muon.handle, self._arr, self._n, ctypes.byref(self._hp),
+                                            _stream_handle(stream))
+        self.muon._check(st, "muon_step_groups")
+
+
+class SpectralPlan:
+    """muon_power_iteration / muon_min_singular over fixed tensors, validated and marshalled once."""
+
+    def __init__(self, muon: "Muon", W, u, v, sigma, y=None, sigma_min=None):
+        import torch
+        self.muon = muon
+        shape, dt = tuple(W[0].shape), W[0].dtype
+        _check_same(W, shape, dt, "cuda", "W")
+        _check_same(u, (shape[0],), torch.float32, "cuda", "u")
+        _check_same(v, (shape[1],), torch.float32, "cuda", "v")
+        if not (len(W) == len(u) == len(v)) or sigma.numel() < len(W) or sigma.dtype != torch.float32:
+            raise ValueError("W, u, v need one entry per matrix and sigma len(W) fp32 slots")
+        if y is not None:
+            _check_same(y, (min(shape),), torch.float32, "cuda", "y")
+            if len(y) != len(W) or sigma_min is None or sigma_min.numel() < len(W) \
+                    or sigma_min.dtype != torch.float32:
+                raise ValueError("y needs one entry per matrix and sigma_min len(W) fp32 slots")
+        self._tensors = (list(W), list(u), list(v), sigma, None if y is None else list(y), sigma_min)
+        self._pw, self._pu, self._pv = _ptrs(W), _ptrs(u), _ptrs(v)
+        self._py = _ptrs(y) if y is not None else None
+        self._args = (len(W), shape[0], shape[1], _dtype_code(W[0]))
+
+    def power_iteration(self, iters=8, stream=None):
+        n, r, c, dt = self._args
+        st = self.muon.lib.muon_power_iteration(self.muon.handle, self._pw, self._pu, self._pv,
+                                                ctypes.c_void_p(self._tensors[3].data_ptr()), n, r, c, dt,
+                                                int(iters), _stream_handle(stream))
+        self.muon._check(st, "muon_power_iteration")
+
+    def min_singular(self, iters=32, stream=None):
+        if self._py is None:
+            raise ValueError("plan built without y / sigma_min")
+        n, r, c, dt = self._args
+        st = self.muon.lib.muon_min_singular(self.muon.handle, self._pw, self._py,
+                                             ctypes.c_void_p(self._tensors[3].data_ptr()),
+                                             ctypes.c_void_p(self._tensors[5].data_ptr()), n, r, c, dt, int(iters),
+                                             _stream_handle(stream))
+        self.muon._check(st, "muon_min_singular")
 
 
 def momentum_norm_noalloc(G, M, nu, beta=0.95, nesterov=True, stream=None):

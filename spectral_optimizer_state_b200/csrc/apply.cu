@@ -102,63 +102,9 @@ __device__ __forceinline__ void rmw1(void* dst, long long e, float v, bool apply
   }
 }
 
-// 16-byte raw vectors of one wide-path step: O and W.  A bf16 W has a one-plane iterate (one
-// vector of each); an fp32 W has three planes and two vectors of W.
-template <bool F32>
-struct Raw8 {
-  static constexpr int kPlanes = F32 ? 3 : 1;
-  uint4 o[kPlanes];
-  uint4 w[F32 ? 2 : 1];
-};
-
-template <bool F32>
-__device__ __forceinline__ void load_raw8(Raw8<F32>& r, const uint16_t* o, long long ps, const void* w, int apply) {
-#pragma unroll
-  for (int p = 0; p < Raw8<F32>::kPlanes; ++p) r.o[p] = __ldcs(reinterpret_cast<const uint4*>(o + p * ps));
-  if (apply) {
-#pragma unroll
-    for (int i = 0; i < (F32 ? 2 : 1); ++i) r.w[i] = reinterpret_cast<const uint4*>(w)[i];
-  }
-}
-
-// Unpack a raw step: ov = sum of the O planes, cw = the current W (zeros when not applying).
-template <bool F32>
-__device__ __forceinline__ void unpack_raw8(const Raw8<F32>& r, int apply, float (&ov)[8], float (&cw)[8]) {
-#pragma unroll
-  for (int t = 0; t < 8; ++t) ov[t] = 0.f;
-#pragma unroll
-  for (int p = 0; p < Raw8<F32>::kPlanes; ++p) {
-    const uint32_t w[4] = {r.o[p].x, r.o[p].y, r.o[p].z, r.o[p].w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      ov[2 * i] += __uint_as_float(w[i] << 16);
-      ov[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  }
-  if (!apply) {
-#pragma unroll
-    for (int t = 0; t < 8; ++t) cw[t] = 0.f;
-  } else if (F32) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      cw[4 * i + 0] = __uint_as_float(r.w[i].x);
-      cw[4 * i + 1] = __uint_as_float(r.w[i].y);
-      cw[4 * i + 2] = __uint_as_float(r.w[i].z);
-      cw[4 * i + 3] = __uint_as_float(r.w[i].w);
-    }
-  } else {
-    const uint32_t w[4] = {r.w[0].x, r.w[0].y, r.w[0].z, r.w[0].w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      cw[2 * i] = __uint_as_float(w[i] << 16);
-      cw[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  }
-}
-
 // Wide W (rows <= cols): W(i, j) with O(i, j).  CAP: O - alpha u v^T (spectral cap).
-// Vector path: 8 elements per thread step, two steps in flight (both steps' loads are
-// issued, as packed 16-byte vectors, before either is used).
+// One 8-element vector per thread step: a short loop body keeps the register count (and so
+// the occupancy that keeps enough bytes in flight) of a plain streaming pass.
 template <bool F32, bool CAP>
 __device__ __forceinline__ void wide_body(const ApplyParams& p, const ApplyGroup& q, int l, int b) {
   void* w = p.w[q.mat0 + l];
@@ -171,34 +117,19 @@ __device__ __forceinline__ void wide_body(const ApplyParams& p, const ApplyGroup
     const long long chunk = (total + q.nblk - 1) / q.nblk;
     const long long beg = chunk * b;
     const long long end = min(total, beg + chunk);
-    for (long long v0 = beg + threadIdx.x; v0 < end; v0 += 2 * kThreads) {
-      const long long v1 = v0 + kThreads;
-      const bool two = v1 < end;
-      long long iv[2];
-      int jv[2];
-      Raw8<F32> raw[2];
+    for (long long v = beg + threadIdx.x; v < end; v += kThreads) {
+      const long long i = v / per_row;
+      const int j = static_cast<int>(v - i * per_row) * 8;
+      char* dst = static_cast<char*>(w) + (i * C + j) * (F32 ? 4 : 2);
+      float ov[8], cw[8];
+      load8_planes(o + i * q.pitch + j, q.o_plane, p.planes, ov);
+      load8_w<F32>(dst, p.apply, cw);
+      if (cap) {
+        const float au = q.alpha[l] * p.cu[q.mat0 + l][i];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const long long v = h ? v1 : v0;
-        iv[h] = v / per_row;
-        jv[h] = static_cast<int>(v - iv[h] * per_row) * 8;
-        if (h == 0 || two)
-          load_raw8<F32>(raw[h], o + iv[h] * q.pitch + jv[h], q.o_plane,
-                         static_cast<char*>(w) + (iv[h] * C + jv[h]) * (F32 ? 4 : 2), p.apply);
+        for (int t = 0; t < 8; ++t) ov[t] = fmaf(-au, p.cv[q.mat0 + l][j + t], ov[t]);
       }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (h == 1 && !two) break;
-        float ov[8], cw[8];
-        unpack_raw8<F32>(raw[h], p.apply, ov, cw);
-        if (cap) {
-          const float au = q.alpha[l] * p.cu[q.mat0 + l][iv[h]];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) ov[t] = fmaf(-au, p.cv[q.mat0 + l][jv[h] + t], ov[t]);
-        }
-        store8_w<F32>(static_cast<char*>(w) + (iv[h] * C + jv[h]) * (F32 ? 4 : 2), ov, cw, p.apply, p.decay,
-                      q.lrs);
-      }
+      store8_w<F32>(dst, ov, cw, p.apply, p.decay, q.lrs);
     }
   } else {
     const long long total = static_cast<long long>(q.rows) * C;
@@ -243,19 +174,7 @@ __device__ __forceinline__ void tall_body(const ApplyParams& p, const ApplyGroup
         for (int t = 0; t < 8; ++t) ov[pass][t] = 0.f;
       }
     }
-    // this thread's W rows for the write-back, read (packed) before the tile exchange
-    uint4 cw_raw[2][F32 ? 2 : 1];
     const bool wvec = q.vec && c0 + cc < C;
-#pragma unroll
-    for (int pass = 0; pass < 2; ++pass) {
-      const int r = r0 + rr + 32 * pass;
-      if (wvec && r < R && p.apply) {
-        const uint4* src = reinterpret_cast<const uint4*>(static_cast<char*>(w) +
-                                                          (static_cast<long long>(r) * C + c0 + cc) * (F32 ? 4 : 2));
-#pragma unroll
-        for (int i = 0; i < (F32 ? 2 : 1); ++i) cw_raw[pass][i] = src[i];
-      }
-    }
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
 #pragma unroll
@@ -278,10 +197,10 @@ __device__ __forceinline__ void tall_body(const ApplyParams& p, const ApplyGroup
             if (c + t < C) v[t] = fmaf(-au, p.cv[q.mat0 + l][c + t], v[t]);
         }
         if (wvec) {
+          char* dst = static_cast<char*>(w) + (static_cast<long long>(r) * C + c) * (F32 ? 4 : 2);
           float cw[8];
-          load8_w<F32>(cw_raw[pass], p.apply, cw);
-          store8_w<F32>(static_cast<char*>(w) + (static_cast<long long>(r) * C + c) * (F32 ? 4 : 2), v, cw,
-                        p.apply, p.decay, q.lrs);
+          load8_w<F32>(dst, p.apply, cw);
+          store8_w<F32>(dst, v, cw, p.apply, p.decay, q.lrs);
         } else {
 #pragma unroll
           for (int t = 0; t < 8; ++t)
@@ -294,7 +213,7 @@ __device__ __forceinline__ void tall_body(const ApplyParams& p, const ApplyGroup
 }
 
 template <bool F32, bool CAP>
-__global__ void __launch_bounds__(kThreads) apply_kernel(const __grid_constant__ ApplyParams p) {
+__global__ void __launch_bounds__(kThreads, 6) apply_kernel(const __grid_constant__ ApplyParams p) {
   int gi = 0;
   while (gi + 1 < p.ngroups && static_cast<int>(blockIdx.x) >= p.grp[gi + 1].block0) ++gi;
   const ApplyGroup& q = p.grp[gi];

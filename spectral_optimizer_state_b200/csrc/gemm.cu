@@ -239,13 +239,38 @@ __device__ __forceinline__ void stage_packed_col(uint32_t buf, int lane, const u
   }
 }
 
+// A chunk and its mirror: both staging buffers filled, one proxy fence, two TMA stores.
+// Lane 0 first makes sure every earlier store of this warp has finished reading its buffer.
+template <typename StageA, typename StageB>
+__device__ __forceinline__ void store_chunk_pair(const CUtensorMap* map, uint32_t stage_base, int& sb, int lane,
+                                                 StageA&& sa, StageB&& sbf, int x, int y, int l, int p) {
+  sb = 2;
+  if (lane == 0) bulk_wait_group_read<0>();
+  __syncwarp();
+  sa(stage_base);
+  sbf(stage_base + 2048u);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_4d(map, stage_base, x, y, l, p);
+    tma_store_4d(map, stage_base + 2048u, y, x, l, p);
+    bulk_commit_group();
+  }
+}
+
 // One 32 x 32 TMA store from the warp's next staging buffer.  Lane 0 first
 // makes sure the store that last read this buffer has finished reading it.
+// `sb` is the next buffer (0 or 1), or 2 after a chunk pair, whose one store group reads both
+// buffers: then the next store waits for every earlier group and starts again at buffer 0.
 template <typename Stage>
 __device__ __forceinline__ void store_chunk(const CUtensorMap* map, uint32_t stage_base, int& sb, int lane,
                                             Stage&& stage, int x, int y, int l, int p) {
+  if (lane == 0) {
+    if (sb == 2) bulk_wait_group_read<0>();
+    else bulk_wait_group_read<1>();
+  }
+  if (sb == 2) sb = 0;
   const uint32_t buf = stage_base + static_cast<uint32_t>(sb) * 2048u;
-  if (lane == 0) bulk_wait_group_read<1>();
   __syncwarp();
   stage(buf);
   fence_proxy_async_smem();
@@ -304,11 +329,14 @@ __device__ __forceinline__ void epilogue_warp_tile(const GemmProblem& q, const T
         const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
         w[i] = *reinterpret_cast<const uint32_t*>(&h);
       }
-      store_chunk(&q.tmOut, my_stage, sb, lane, [&](uint32_t buf) { stage_packed_row(buf, lane, w); }, j0, row0,
-                  ti.l, 0);
-      if (mirror)
-        store_chunk(&q.tmOut, my_stage, sb, lane, [&](uint32_t buf) { stage_packed_col(buf, lane, w); }, row0, j0,
+      if (mirror) {
+        store_chunk_pair(
+            &q.tmOut, my_stage, sb, lane, [&](uint32_t buf) { stage_packed_row(buf, lane, w); },
+            [&](uint32_t buf) { stage_packed_col(buf, lane, w); }, j0, row0, ti.l, 0);
+      } else {
+        store_chunk(&q.tmOut, my_stage, sb, lane, [&](uint32_t buf) { stage_packed_row(buf, lane, w); }, j0, row0,
                     ti.l, 0);
+      }
     } else {
       for (int p = 0; p < q.planes; ++p) {
         uint16_t b[32];
@@ -542,288 +570,31 @@ __global__ void __launch_bounds__(THREADS, 1) ns_gemm_kernel(const __grid_consta
 }
 
 
-// ------------------------------------------------------------------ CTA-pair kernel
-// cta_group::2: a cluster of two CTAs computes a 256 x 256 tile.  CTA r holds
-// rows [128 r, 128 r + 128) of the A tile and columns [r N/2, (r+1) N/2) of
-// the B tile in its own shared memory; the leader (rank 0) issues the MMAs,
-// which read both CTAs' halves and write each CTA's 128 accumulator rows to
-// its own TMEM.  Every CTA needs only 32 KB per 64-deep stage (six stages in
-// flight) instead of 48 KB, for the same MMA time per stage.
-//   full[s]   leader only: its producer posts the bytes of both CTAs; the
-//             follower's loads complete their bytes on the leader's barrier.
-//   empty[s]  both CTAs: the leader's commit arrives on both (multicast).
-//   tfull[a]  both CTAs: likewise, when a tile's MMAs are done.
-//   tempty[a] leader only: one arrival per epilogue warp of either CTA.
-constexpr int PBM = 256;                       // pair tile rows
-constexpr int PSTAGES = 6;
-constexpr uint32_t PA_BYTES = 128 * BK * 2;    // 16 KB: this CTA's A rows
-constexpr uint32_t PB_BYTES = 128 * BK * 2;    // 16 KB: this CTA's half of B
-constexpr uint32_t PSTAGE_BYTES = PA_BYTES + PB_BYTES;
-constexpr uint32_t PBOX_BYTES = 64 * BK * 2;   // any B box {64, 64}
-constexpr int PNUM_BARS = 2 * PSTAGES + 5;
-constexpr uint32_t PBAR_BYTES = 8 * PNUM_BARS + 16;
-
-__global__ void __launch_bounds__(THREADS, 1) ns_gemm_pair_kernel(const __grid_constant__ GemmParams P) {
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_addr(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t stage_area = base + PSTAGES * PSTAGE_BYTES;
-  const uint32_t bar0 = stage_area + EPI_WARPS * STAGING_BYTES_PER_WARP;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + (bar0 - base) + 8 * PNUM_BARS);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  TileMeta* meta = reinterpret_cast<TileMeta*>(gbase + (bar0 - base) + PBAR_BYTES);
-  load_meta(P, meta);
-
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (PSTAGES + s); };
-  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * PSTAGES + a); };
-  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * PSTAGES + 2 + a); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * PSTAGES + 4);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_cta_rank();
-  const bool leader = rank == 0;
-  const int pair = blockIdx.x >> 1;
-  const int npairs = gridDim.x >> 1;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < PSTAGES; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 2 * EPI_WARPS);
-    }
-    mbar_init(drain_bar, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-    fence_proxy_async_smem();
-  }
-  if (warp == 0 && lane == 0) {
-    for (int i = 0; i < P.nprob; ++i) {
-      tma_prefetch_map(&P.prob[i].tmA);
-      tma_prefetch_map(&P.prob[i].tmB);
-      tma_prefetch_map(&P.prob[i].tmOut);
-    }
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(smem_addr(tmem_holder), TMEM_COLS);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  cluster_sync_all();  // barriers of both CTAs initialised, TMEM address written
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_holder;
-
-  if (warp == 0) {
-    // ------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
-      uint32_t it = 0;
-      bool ok = true;
-      unsigned dep_seen = 0;  // next tile's dependency counter, read a tile ahead
-      if (pair < P.total_tiles) {
-        const Tile t0 = decode_tile<PBM, 128>(meta, P.nprob, pair);
-        if (P.prob[t0.pi].done_dep != nullptr) dep_seen = ld_relaxed_gpu(P.prob[t0.pi].done_dep + t0.l);
-      }
-      for (int t = pair; ok && t < P.total_tiles; t += npairs) {
-        const Tile ti = decode_tile<PBM, 128>(meta, P.nprob, t);
-        const GemmProblem& q = P.prob[ti.pi];
-        if (q.done_dep != nullptr) {
-          // both CTAs load, so both acquire the previous phase of this matrix
-          if (dep_seen >= q.dep_target) {
-            __threadfence();
-          } else if (!wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status)) {
-            ok = false;
-            break;
-          }
-          fence_proxy_async_global();
-        }
-        const int tn = t + npairs;
-        if (tn < P.total_tiles) {
-          const Tile tin = decode_tile<PBM, 128>(meta, P.nprob, tn);
-          dep_seen = P.prob[tin.pi].done_dep != nullptr ? ld_relaxed_gpu(P.prob[tin.pi].done_dep + tin.l) : 0u;
-        }
-        const int nk = q.k_tiles * q.nseg;
-        const int half_n = ti.nw >> 1;                 // this CTA's B columns (64 or 128)
-        const bool narrow = half_n <= 64;
-        const int n_mine = ti.n0 + static_cast<int>(rank) * half_n;
-        const uint32_t pair_bytes = 2u * (PA_BYTES + (narrow ? PBOX_BYTES : 2u * PBOX_BYTES));
-        for (int kk = 0; kk < nk; ++kk, ++it) {
-          const int s = it % PSTAGES;
-          const uint32_t ph = (it / PSTAGES) & 1u;
-          if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, abort_flag, P.status)) {
-            ok = false;
-            break;
-          }
-          const int seg = kk / q.k_tiles;
-          const int kb = kk - seg * q.k_tiles;
-          int pa, pb;
-          segment_planes(q.nseg, seg, pa, pb);
-          const uint32_t sa = base + s * PSTAGE_BYTES;
-          const uint32_t sb = sa + PA_BYTES;
-          const uint32_t fb = map_shared_rank(full_bar(s), 0);  // the leader's full barrier
-          if (leader) mbar_arrive_expect_tx(full_bar(s), pair_bytes);
-          tma_load_4d_pair(sa, &q.tmA, fb, kb * BK, ti.m0 + 128 * static_cast<int>(rank), ti.l, pa);
-          const CUtensorMap* mb = narrow ? &q.tmB2 : &q.tmB;
-          if (q.b_mn_major)
-            tma_load_5d_pair(sb, mb, fb, 0, kb * BK, n_mine / 64, ti.l, pb);
-          else
-            tma_load_4d_pair(sb, mb, fb, kb * BK, n_mine, ti.l, pb);
-        }
-      }
-      if (!ok) {
-        // The copies this thread started complete on the leader's barriers; give
-        // them a bounded time to land before the CTA may leave.
-        if (leader) {
-          const uint32_t n = it < PSTAGES ? it : PSTAGES;
-          for (uint32_t j = it - n; j < it; ++j) wait_drain(full_bar(j % PSTAGES), (j / PSTAGES) & 1u);
-        } else {
-          const uint64_t t0 = global_timer_ns();
-          while (global_timer_ns() - t0 < 2000000ull) __nanosleep(1000);
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------ UMMA issuer (leader only)
-    if (lane == 0 && leader) {
-      uint32_t it = 0;
-      int local = 0;
-      bool ok = true;
-      for (int t = pair; ok && t < P.total_tiles; t += npairs, ++local) {
-        const Tile ti = decode_tile<PBM, 128>(meta, P.nprob, t);
-        const GemmProblem& q = P.prob[ti.pi];
-        const int acc = local & 1;
-        const uint32_t aph = (local >> 1) & 1;
-        if (!mbar_wait_bounded(tempty_bar(acc), aph ^ 1u, abort_flag, P.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
-        const uint32_t idesc = instr_desc_bf16(PBM, ti.nw, q.b_mn_major != 0);
-        const int nk = q.k_tiles * q.nseg;
-        for (int kk = 0; kk < nk; ++kk, ++it) {
-          const int s = it % PSTAGES;
-          const uint32_t ph = (it / PSTAGES) & 1u;
-          if (!mbar_wait_bounded(full_bar(s), ph, abort_flag, P.status)) {
-            ok = false;
-            break;
-          }
-          const uint32_t sa = base + s * PSTAGE_BYTES;
-          const uint32_t sb = sa + PA_BYTES;
-#pragma unroll
-          for (int k4 = 0; k4 < BK / 16; ++k4) {
-            const uint64_t ad = smem_desc_sw128(sa + 32u * k4, 16u, 1024u);
-            const uint64_t bd = q.b_mn_major ? smem_desc_sw128(sb + 2048u * k4, PBOX_BYTES, 1024u)
-                                             : smem_desc_sw128(sb + 32u * k4, 16u, 1024u);
-            tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kk | k4) != 0 ? 1u : 0u);
-          }
-          tc_commit_pair(empty_bar(s), 0x3);
-        }
-        if (ok) tc_commit_pair(tfull_bar(acc), 0x3);
-      }
-      if (!ok) {
-        tc_commit_pair(drain_bar, 0x1);
-        wait_drain(drain_bar, 0);
-      }
-    }
-  } else {
-    // ------------------------------------------------ epilogue (both CTAs)
-    const int e = warp - 2;
-    const int quarter = warp & 3;
-    const int half = e >> 2;
-    const uint32_t my_stage = stage_area + static_cast<uint32_t>(e) * STAGING_BYTES_PER_WARP;
-    int sb = 0;
-    int local = 0;
-    for (int t = pair; t < P.total_tiles; t += npairs, ++local) {
-      const Tile ti = decode_tile<PBM, 128>(meta, P.nprob, t);
-      const GemmProblem& q = P.prob[ti.pi];
-      const int acc = local & 1;
-      const uint32_t aph = (local >> 1) & 1;
-      if (!mbar_wait_bounded(tfull_bar(acc), aph, abort_flag, P.status)) break;
-      tc_fence_after();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16) + acc * ACC_COLS;
-      if (q.cin != nullptr && q.done_dep != nullptr) {
-        if (!wait_counter_bounded(q.done_dep + ti.l, q.dep_target, abort_flag, P.status)) break;
-      }
-      epilogue_warp_tile(q, ti, tbase, ti.m0 + 128 * static_cast<int>(rank) + 32 * quarter, lane,
-                         32 * half, ti.m0 + PBM, my_stage, sb, [&] {
-                           tc_fence_before();
-                           __syncwarp();
-                           if (lane == 0) mbar_arrive_remote(map_shared_rank(tempty_bar(acc), 0));
-                         });
-      if (q.done_self != nullptr) {
-        if (lane == 0) {
-          bulk_wait_group_all();
-          fence_proxy_async_global();
-          red_release_gpu_add(q.done_self + ti.l, 1u);
-        }
-        __syncwarp();
-      }
-    }
-    if (lane == 0) bulk_wait_group_all();
-  }
-
-  __syncthreads();
-  cluster_sync_all();  // no MMA, load or arrival still targets the other CTA
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc_pair(tmem_base, TMEM_COLS);
-  }
-}
-
 }  // namespace
 
-size_t gemm_smem_bytes(int kind) {
-  if (kind == GEMM_PAIR)
-    return PSTAGES * PSTAGE_BYTES + EPI_WARPS * STAGING_BYTES_PER_WARP + PBAR_BYTES + META_BYTES + 1024;
-  return STAGES * STAGE_BYTES + EPI_WARPS * STAGING_BYTES_PER_WARP + BAR_BYTES + META_BYTES + 1024;
-}
+size_t gemm_smem_bytes() { return STAGES * STAGE_BYTES + EPI_WARPS * STAGING_BYTES_PER_WARP + BAR_BYTES + META_BYTES + 1024; }
 
-int gemm_tiles_per_matrix(int kind, int M, int N, int sym) {
-  const int tm = kind == GEMM_PAIR ? PBM : BM;
+int gemm_tiles_per_matrix(int M, int N, int sym) {
   if (sym) {
     int n = 0;
-    for (int mb = 0; mb * tm < M; ++mb) n += (M - tm * mb + BN - 1) / BN;
+    for (int mb = 0; mb * BM < M; ++mb) n += (M - BM * mb + BN - 1) / BN;
     return n;
   }
-  return ((M + tm - 1) / tm) * ((N + BN - 1) / BN);
+  return ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
 }
 
-cudaError_t launch_gemm(const GemmParams& p, int kind, int units, cudaStream_t stream) {
-  static int configured_device[2] = {-1, -1};
+cudaError_t launch_gemm(const GemmParams& p, int ctas, cudaStream_t stream) {
+  static int configured_device = -1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const void* fn = kind == GEMM_PAIR ? reinterpret_cast<const void*>(ns_gemm_pair_kernel)
-                                     : reinterpret_cast<const void*>(ns_gemm_kernel);
-  const int smem = static_cast<int>(gemm_smem_bytes(kind));
-  if (configured_device[kind] != dev) {
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = static_cast<int>(gemm_smem_bytes());
+  if (configured_device != dev) {
+    e = cudaFuncSetAttribute(ns_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    configured_device[kind] = dev;
+    configured_device = dev;
   }
-  if (kind == GEMM_PAIR) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * units, 1, 1);
-    cfg.blockDim = dim3(THREADS, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, ns_gemm_pair_kernel, p);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
-  }
-  ns_gemm_kernel<<<units, THREADS, smem, stream>>>(p);
+  ns_gemm_kernel<<<ctas, THREADS, smem, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -122,11 +122,10 @@ constexpr int kMaxProblems = 30;
 
 struct alignas(64) GemmProblem {
   CUtensorMap tmA;   // A operand [planes][L][M][K], K contiguous, box {64, 128}
-  CUtensorMap tmB;   // B operand.  Single-CTA kernel: K-major [planes][L][N][K] box
-                     // {64, 256}; MN-major as the 5-D chunked view {64 n, K, N/64,
-                     // L, planes} with box {64, 64, 4, 1, 1} (one load per stage).
-                     // CTA-pair kernel: 4-D box {64, 64} in either layout.
-  CUtensorMap tmB2;  // single-CTA kernel, K-major B: box {64, 128} for tiles <= 128 wide
+  CUtensorMap tmB;   // B operand: K-major [planes][L][N][K] box {64, 256}; MN-major as the
+                     // 5-D chunked view {64 n, K, N/64, L, planes} with box {64, 64, 4, 1, 1}
+                     // (one load per stage).
+  CUtensorMap tmB2;  // K-major B: box {64, 128} for tiles <= 128 wide
   CUtensorMap tmOut;  // output [planes][L][M][N], box {32, 32}, 64-byte swizzle
   int M, N, K, L;
   int nseg;          // 1 (bf16) or 6 (three-plane split)
@@ -161,17 +160,12 @@ struct GemmParams {
   int drop_signal;
 };
 
-// Two kernels share the problem description:
-//   single CTA: 128 x 256 tiles; B operand boxes {64, 128} (K-major) or {64, 64}.
-//   CTA pair (cta_group::2): 256 x 256 tiles, each CTA holds 128 rows of A and
-//   half of the tile's N columns of B; B operand boxes {64, 64}.
-enum GemmKind : int { GEMM_SINGLE = 0, GEMM_PAIR = 1 };
-
-size_t gemm_smem_bytes(int kind);
-// `units`: CTAs (single) or CTA pairs (pair) to launch.
-cudaError_t launch_gemm(const GemmParams& p, int kind, int units, cudaStream_t stream);
+// 128 x 256 tiles, B operand boxes {64, 128}/{64, 256} (K-major) or {64, 64, 4} (MN-major).
+size_t gemm_smem_bytes();
+// `ctas`: persistent CTAs to launch (one per SM at most).
+cudaError_t launch_gemm(const GemmParams& p, int ctas, cudaStream_t stream);
 
 // Tiles one matrix of this problem shape contributes.
-int gemm_tiles_per_matrix(int kind, int M, int N, int sym);
+int gemm_tiles_per_matrix(int M, int N, int sym);
 
 }  // namespace muon

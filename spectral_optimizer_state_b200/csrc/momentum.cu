@@ -315,7 +315,7 @@ __device__ __forceinline__ void tall_body(const MomentumParams& p, const Momentu
 
 // Every group of the launch: the block range of group g starts at grp[g].block0.
 template <typename TG, bool MOM, int PLANES>
-__global__ void __launch_bounds__(kThreads) momentum_kernel(const __grid_constant__ MomentumParams p) {
+__global__ void __launch_bounds__(kThreads, 4) momentum_kernel(const __grid_constant__ MomentumParams p) {
   int gi = 0;
   while (gi + 1 < p.ngroups && static_cast<int>(blockIdx.x) >= p.grp[gi + 1].block0) ++gi;
   const MomentumGroup& q = p.grp[gi];

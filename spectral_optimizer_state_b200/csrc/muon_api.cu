@@ -145,7 +145,6 @@ struct muon_ctx {
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
   cudaEvent_t ev_k1[MUON_MAX_GROUPS] = {};
   cudaEvent_t ev_gemm[MUON_MAX_GROUPS] = {};
-  int gemm_kind = GEMM_SINGLE;  // MUON_GEMM=pair selects the CTA-pair kernel
   bool per_phase = false;       // MUON_LAUNCH=phase: one launch per phase (same work; per-phase timing)
   int last_count = 0;
   cudaStream_t last_stream = nullptr;
@@ -338,10 +337,8 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
   q.planes = p.planes;
   const bool have_poly = cc != 0.f;
   const CUtensorMapSwizzle sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
-  // K-major B operand box height: the tile's N (256, or 128 for narrow tiles) on a
-  // single CTA; half of it (128, or 64) on each CTA of a pair.
-  const bool pair = c->gemm_kind == GEMM_PAIR;
-  const int kb_rows = pair ? 128 : 256;
+  // K-major B operand box height: the tile's N (256, or 128 for narrow tiles)
+  const int kb_rows = 256;
   switch (ph) {
     case PH_GRAM:
       // A = s2 * X X^T; with c = 0 the polynomial is linear and the Gram
@@ -372,10 +369,8 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
     case PH_UPDATE: {
       // X' = s1 * B' X   (s1 = 1/(nu+eps) on the first iteration, X = U unnormalised)
       if (!encode_map(&q.tmA, B, m, m, p.batch, p.planes, p.pitch_m, 64, 128)) return false;
-      // chunked MN-major view: 4 chunks per load (single CTA) or 2 (each CTA of a pair);
-      // the narrow variant (pair, half-width tiles) loads one chunk
-      if (!encode_chunked_map(&q.tmB, X, m, p.batch, p.planes, p.pitch_n, pair ? 2 : 4)) return false;
-      if (pair && !encode_chunked_map(&q.tmB2, X, m, p.batch, p.planes, p.pitch_n, 1)) return false;
+      // chunked MN-major view: 4 chunks of 64 columns per load
+      if (!encode_chunked_map(&q.tmB, X, m, p.batch, p.planes, p.pitch_n, 4)) return false;
       q.M = m; q.N = n; q.K = m;
       q.b_mn_major = 1; q.sym = 0;
       q.alpha = 1.f; q.beta = 0.f; q.diag = 0.f;
@@ -384,7 +379,7 @@ bool fill_problem(muon_ctx* c, const GroupPlan& p, Phase ph, int it, GemmProblem
       break;
     }
   }
-  q.tiles_per_matrix = gemm_tiles_per_matrix(c->gemm_kind, q.M, q.N, q.sym);
+  q.tiles_per_matrix = gemm_tiles_per_matrix(q.M, q.N, q.sym);
   q.k_tiles = (q.K + 63) / 64;
   return true;
 }
@@ -465,11 +460,10 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
   };
   std::vector<int> all_groups;
   for (int g = 0; g < static_cast<int>(plans.size()); ++g) all_groups.push_back(g);
-  // k Newton-Schulz iterations.  The single-CTA kernel runs every phase of
-  // every group in one persistent launch (as many as fit in one parameter
-  // block), ordered phase by phase; per-(phase, matrix) counters let a tile
-  // start as soon as the previous phase of its own matrix has landed.  The
-  // CTA-pair kernel runs one launch per phase.
+  // k Newton-Schulz iterations.  One persistent launch runs every phase of
+  // every group (as many as fit in one parameter block), ordered phase by phase;
+  // per-(phase, matrix) counters let a tile start as soon as the previous phase
+  // of its own matrix has landed.  MUON_LAUNCH=phase runs one launch per phase.
   std::vector<Phase> seq_ph;
   std::vector<int> seq_it;
   for (int it = 0; it < c->k; ++it) {
@@ -480,8 +474,7 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
     }
   }
   const bool persistent = !c->per_phase;
-  const bool pair = c->gemm_kind == GEMM_PAIR;
-  const int signals_per_tile = kEpilogueWarps * (pair ? 2 : 1);
+  const int signals_per_tile = kEpilogueWarps;
   const int ng = static_cast<int>(plans.size());
   const int nph = static_cast<int>(seq_ph.size());
   // Launch order of (group, phase) problems.  Persistent launches go group by
@@ -489,8 +482,8 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
   // next group starts while the last phases of the previous one drain.  (Each
   // phase keeps the matrix order of the previous one, so a matrix's next phase
   // is dispatched a whole phase after its previous one; reversing the order for
-  // L2 reuse measured slower because of those dependency waits.)  The CTA-pair
-  // kernel runs one launch per phase covering every group.
+  // L2 reuse measured slower because of those dependency waits.)  The per-phase
+  // mode runs one launch per phase covering every group.
   struct Item { int g, pi; };
   std::vector<std::vector<Item>> launches;
   // Pipelined schedule (two or more groups, persistent kernel): one launch per group on the
@@ -554,18 +547,18 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
       ++gp.nprob;
     }
     gp.total_tiles = tiles;
-    if (persistent && c->drop_signal_once && c->gemm_kind == GEMM_SINGLE && gp.nprob > 1) {
+    if (persistent && c->drop_signal_once && gp.nprob > 1) {
       gp.drop_signal = 1;
       c->drop_signal_once = false;
     }
     if (persistent)
       MUON_CUDA(cudaMemsetAsync(c->d_done, 0, sizeof(unsigned) * gp.nprob * MUON_MAX_BATCH, strm), "clear counters");
-    const int units = std::min(tiles, pair ? c->sm_count / 2 : c->sm_count);
+    const int units = std::min(tiles, c->sm_count);
     const int kind = items.size() > static_cast<size_t>(ng) || persistent
                          ? MUON_KERNEL_NS_FUSED
                          : MUON_KERNEL_GRAM + (seq_ph[items[0].pi] - PH_GRAM);
     const int slot = prof_begin(c, kind, strm);
-    MUON_CUDA(launch_gemm(gp, c->gemm_kind, units, strm), "newton-schulz gemm");
+    MUON_CUDA(launch_gemm(gp, units, strm), "newton-schulz gemm");
     prof_end(c, slot, strm);
     return MUON_OK;
   };
@@ -737,9 +730,7 @@ muon_status muon_create(muon_ctx** out, int device) {
   c->sm_count = prop.multiProcessorCount;
   for (int i = 0; i < 5; ++i) std::memcpy(&c->coeffs[3 * i], kQuintic, sizeof(kQuintic));
   c->k = 5;
-  if (const char* g = std::getenv("MUON_GEMM")) {
-    if (std::strcmp(g, "pair") == 0) c->gemm_kind = GEMM_PAIR;
-  }
+
   if (const char* l = std::getenv("MUON_LAUNCH")) {
     if (std::strcmp(l, "phase") == 0) c->per_phase = true;
   }

@@ -425,34 +425,6 @@ def test_ill_conditioned_variant(ctx, dtype):
             assert full < 0.15  # reported; single-pass bf16 cannot resolve sigma ~1e-6 directions
 
 
-def test_single_cta_and_pair_kernels_agree():
-    """The single-CTA (128 x 256) and CTA-pair (256 x 256) kernels compute the same products."""
-    import os
-    import torch
-    from spectral_optimizer_state_b200 import Muon
-    outs = {}
-    shapes = [(200, 328), (768, 1536), (3352, 768)]
-    for kind in ("single", "pair"):
-        os.environ["MUON_GEMM"] = kind
-        try:
-            m = Muon(0)
-        finally:
-            del os.environ["MUON_GEMM"]
-        m.set_coeffs(QUINTIC5)
-        res = []
-        for i, shape in enumerate(shapes):
-            X = [to_device(g, "bf16") for g in _inputs(shape, 2, seed=300 + i, kind="spike")]
-            Out = [torch.empty_like(x) for x in X]
-            m.ns_orthogonalize(X, Out, eps=1e-7)
-            assert m.status()[0] == 0
-            res.append([to_numpy(o) for o in Out])
-        m.close()
-        outs[kind] = res
-    for a_list, b_list in zip(outs["single"], outs["pair"]):
-        for a, b in zip(a_list, b_list):
-            assert rel_f(a, b) <= 5e-3
-
-
 @pytest.mark.parametrize("env", [{"MUON_OVERLAP": "1"}, {"MUON_LAUNCH": "phase"}])
 def test_alternative_schedules_are_bitwise_equal_to_the_default(env):
     """The two-stream schedule (momentum and apply passes of other groups on a side stream)
@@ -524,3 +496,23 @@ def test_scaled_2k_model_full_size_sampled():
         err = rel_f(update_from_zero_weights(W[g][l], HP["lr"], oracle.shape_scale(*shapes[g])), r["O"])
         assert err <= BF16_UPDATE_TOL, (g, err)
     mu.close()
+
+
+def test_step_plan_equals_step_groups_bitwise(ctx):
+    """A StepPlan (tensors checked and marshalled once) performs exactly the step step_groups does."""
+    import torch
+    shapes = [(200, 328), (328, 200)]
+    W0 = [[to_device(w, "bf16") for w in group_weights(8, i, 2, *sh)] for i, sh in enumerate(shapes)]
+    Wa = [[w.clone() for w in ws] for ws in W0]
+    Wb = [[w.clone() for w in ws] for ws in W0]
+    Ma = [[torch.zeros(sh, device="cuda") for _ in range(2)] for sh in shapes]
+    Mb = [[torch.zeros(sh, device="cuda") for _ in range(2)] for sh in shapes]
+    G = [[to_device(g, "bf16") for g in _inputs(sh, 2, seed=810 + i)] for i, sh in enumerate(shapes)]
+    ctx.set_coeffs(QUINTIC5)
+    plan = ctx.step_plan([(Wb[i], G[i], Mb[i]) for i in range(2)], **HP)
+    for _ in range(2):
+        ctx.step_groups([(Wa[i], G[i], Ma[i]) for i in range(2)], **HP)
+        plan()
+    assert ctx.status()[0] == 0
+    for a, b in zip([w for ws in Wa + Ma for w in ws], [w for ws in Wb + Mb for w in ws]):
+        assert torch.equal(a, b)

@@ -192,3 +192,30 @@ def test_min_singular_of_semi_orthogonal_is_one():
         _, smin_tall = _min_singular(muon, Ws[:1], [np.ones(128, np.float32)], [1.0], 5, "f32")
         _, smin_wide = _min_singular(muon, Ws[1:], [np.ones(128, np.float32)], [1.0], 5, "f32")
     assert abs(smin_tall[0] - 1.0) <= 1e-5 and abs(smin_wide[0] - 1.0) <= 1e-5
+
+
+def test_spectral_plan_equals_the_methods():
+    """SpectralPlan (tensors checked and marshalled once) gives what power_iteration and
+    min_singular give."""
+    import torch
+    from spectral_optimizer_state_b200 import Muon
+    Ws = [to_device(w, "bf16") for w in _spiked(160, 96, 3, 91, "bf16")]
+    out = []
+    with Muon() as muon:
+        for use_plan in (False, True):
+            u = [torch.zeros(160, device="cuda") for _ in Ws]
+            v = [torch.ones(96, device="cuda") for _ in Ws]
+            y = [torch.ones(96, device="cuda") for _ in Ws]
+            smax = torch.zeros(3, device="cuda")
+            smin = torch.zeros(3, device="cuda")
+            if use_plan:
+                plan = muon.spectral_plan(Ws, u, v, smax, y, smin)
+                plan.power_iteration(iters=5)
+                plan.min_singular(iters=7)
+            else:
+                muon.power_iteration(Ws, u, v, smax, iters=5)
+                muon.min_singular(Ws, y, smax, smin, iters=7)
+            torch.cuda.synchronize()
+            out.append([t.clone() for t in u + v + y] + [smax.clone(), smin.clone()])
+    for a, b in zip(*out):
+        assert torch.equal(a, b)

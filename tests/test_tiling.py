@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 
 BN = 256
-KINDS = {"single": (128, 64), "pair": (256, 128)}  # (tile rows, column granularity)
+KINDS = {"single": (128, 64)}  # (tile rows, column granularity)
 
 
 def tiles_per_matrix(M, N, sym, kind="single"):
@@ -101,12 +101,10 @@ def test_tma_coordinates_aligned(m, n, kind):
             m0, n0, nw = decode(m, N, sym, r, kind)
             for kb in range((K + 63) // 64):
                 assert (kb * 64 * 2) % 16 == 0  # A / K-major B: x = k
-            half = nw // 2 if kind == "pair" else nw
-            for rank in ((0, 1) if kind == "pair" else (0,)):
-                for c in range(half // 64):
-                    x = n0 + rank * half + 64 * c
-                    assert (x * 2) % 16 == 0  # MN-major B: x = n
-                    assert half % 64 == 0
+            for c in range(nw // 64):
+                x = n0 + 64 * c
+                assert (x * 2) % 16 == 0  # MN-major B: x = n
+                assert nw % 64 == 0
 
 
 @pytest.mark.parametrize("m,n", SHAPES)
