@@ -103,8 +103,10 @@ __device__ __forceinline__ void rmw1(void* dst, long long e, float v, bool apply
 }
 
 // Wide W (rows <= cols): W(i, j) with O(i, j).  CAP: O - alpha u v^T (spectral cap).
-// One 8-element vector per thread step: a short loop body keeps the register count (and so
-// the occupancy that keeps enough bytes in flight) of a plain streaming pass.
+// A bf16 W takes two 8-element steps per iteration, both steps' loads issued as packed
+// 16-byte vectors before either is unpacked (within the 40-register budget that keeps six
+// blocks per SM); an fp32 W (three-plane iterate) or the capped pass, which would not fit
+// that budget, one step.
 template <bool F32, bool CAP>
 __device__ __forceinline__ void wide_body(const ApplyParams& p, const ApplyGroup& q, int l, int b) {
   void* w = p.w[q.mat0 + l];
@@ -117,19 +119,70 @@ __device__ __forceinline__ void wide_body(const ApplyParams& p, const ApplyGroup
     const long long chunk = (total + q.nblk - 1) / q.nblk;
     const long long beg = chunk * b;
     const long long end = min(total, beg + chunk);
-    for (long long v = beg + threadIdx.x; v < end; v += kThreads) {
-      const long long i = v / per_row;
-      const int j = static_cast<int>(v - i * per_row) * 8;
-      char* dst = static_cast<char*>(w) + (i * C + j) * (F32 ? 4 : 2);
-      float ov[8], cw[8];
-      load8_planes(o + i * q.pitch + j, q.o_plane, p.planes, ov);
-      load8_w<F32>(dst, p.apply, cw);
-      if (cap) {
-        const float au = q.alpha[l] * p.cu[q.mat0 + l][i];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) ov[t] = fmaf(-au, p.cv[q.mat0 + l][j + t], ov[t]);
+    if (F32 || CAP) {
+      for (long long v = beg + threadIdx.x; v < end; v += kThreads) {
+        const long long i = v / per_row;
+        const int j = static_cast<int>(v - i * per_row) * 8;
+        char* dst = static_cast<char*>(w) + (i * C + j) * (F32 ? 4 : 2);
+        float ov[8], cw[8];
+        load8_planes(o + i * q.pitch + j, q.o_plane, p.planes, ov);
+        load8_w<F32>(dst, p.apply, cw);
+        if (cap) {
+          const float au = q.alpha[l] * p.cu[q.mat0 + l][i];
+  #pragma unroll
+          for (int t = 0; t < 8; ++t) ov[t] = fmaf(-au, p.cv[q.mat0 + l][j + t], ov[t]);
+        }
+        store8_w<F32>(dst, ov, cw, p.apply, p.decay, q.lrs);
       }
-      store8_w<F32>(dst, ov, cw, p.apply, p.decay, q.lrs);
+    } else {
+      for (long long v0 = beg + threadIdx.x; v0 < end; v0 += 2 * kThreads) {
+        const long long v1 = v0 + kThreads;
+        const bool two = v1 < end;
+        const long long i0 = v0 / per_row, i1 = v1 / per_row;
+        const int j0 = static_cast<int>(v0 - i0 * per_row) * 8, j1 = static_cast<int>(v1 - i1 * per_row) * 8;
+        char* d0 = static_cast<char*>(w) + (i0 * C + j0) * (F32 ? 4 : 2);
+        char* d1 = static_cast<char*>(w) + (i1 * C + j1) * (F32 ? 4 : 2);
+        // both steps' loads as packed 16-byte vectors before either is unpacked
+        uint4 oa[F32 ? 3 : 1], ob[F32 ? 3 : 1], wa[F32 ? 2 : 1], wb[F32 ? 2 : 1];
+  #pragma unroll
+        for (int pl = 0; pl < (F32 ? 3 : 1); ++pl) {
+          oa[pl] = __ldcs(reinterpret_cast<const uint4*>(o + pl * q.o_plane + i0 * q.pitch + j0));
+          if (two) ob[pl] = __ldcs(reinterpret_cast<const uint4*>(o + pl * q.o_plane + i1 * q.pitch + j1));
+        }
+        if (p.apply) {
+  #pragma unroll
+          for (int k = 0; k < (F32 ? 2 : 1); ++k) {
+            wa[k] = reinterpret_cast<const uint4*>(d0)[k];
+            if (two) wb[k] = reinterpret_cast<const uint4*>(d1)[k];
+          }
+        }
+  #pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (h == 1 && !two) break;
+          const uint4* ov4 = h ? ob : oa;
+          float ov[8], cw[8];
+  #pragma unroll
+          for (int t = 0; t < 8; ++t) ov[t] = 0.f;
+  #pragma unroll
+          for (int pl = 0; pl < (F32 ? 3 : 1); ++pl) {
+            const uint32_t u[4] = {ov4[pl].x, ov4[pl].y, ov4[pl].z, ov4[pl].w};
+  #pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              ov[2 * k] += __uint_as_float(u[k] << 16);
+              ov[2 * k + 1] += __uint_as_float(u[k] & 0xFFFF0000u);
+            }
+          }
+          load8_w<F32>(h ? wb : wa, p.apply, cw);
+          const long long ii = h ? i1 : i0;
+          const int jj = h ? j1 : j0;
+          if (cap) {
+            const float au = q.alpha[l] * p.cu[q.mat0 + l][ii];
+  #pragma unroll
+            for (int t = 0; t < 8; ++t) ov[t] = fmaf(-au, p.cv[q.mat0 + l][jj + t], ov[t]);
+          }
+          store8_w<F32>(h ? d1 : d0, ov, cw, p.apply, p.decay, q.lrs);
+        }
+      }
     }
   } else {
     const long long total = static_cast<long long>(q.rows) * C;
@@ -218,8 +271,10 @@ __global__ void __launch_bounds__(kThreads, 6) apply_kernel(const __grid_constan
   while (gi + 1 < p.ngroups && static_cast<int>(blockIdx.x) >= p.grp[gi + 1].block0) ++gi;
   const ApplyGroup& q = p.grp[gi];
   const int local = static_cast<int>(blockIdx.x) - q.block0;
-  const int l = local / q.nblk;
-  const int b = local - l * q.nblk;
+  const int lr = local / q.nblk;
+  const int b = local - lr * q.nblk;
+  // matrices last to first: the Newton-Schulz launch wrote the last matrix last
+  const int l = q.batch - 1 - lr;
   if (q.flags != nullptr && q.flags[l] != 0) return;
   if (p.status != nullptr && (*p.status & kStatusTimeout)) return;  // the iterate is incomplete
   if (q.rows > q.cols) tall_body<F32, CAP>(p, q, l, b);

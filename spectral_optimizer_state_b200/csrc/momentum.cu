@@ -320,8 +320,10 @@ __global__ void __launch_bounds__(kThreads, 4) momentum_kernel(const __grid_cons
   while (gi + 1 < p.ngroups && static_cast<int>(blockIdx.x) >= p.grp[gi + 1].block0) ++gi;
   const MomentumGroup& q = p.grp[gi];
   const int local = static_cast<int>(blockIdx.x) - q.block0;
-  const int l = local / q.nblk;
-  const int b = local - l * q.nblk;
+  const int lr = local / q.nblk;
+  const int b = local - lr * q.nblk;
+  // matrices last to first: the Newton-Schulz launch reads matrix 0 first, so its U is written last
+  const int l = q.batch - 1 - lr;
   if (q.rows > q.cols) tall_body<TG, MOM, PLANES>(p, q, l, b);
   else wide_body<TG, MOM, PLANES>(p, q, l, b);
 }

@@ -458,8 +458,12 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
     }
     return MUON_OK;
   };
+  // Both elementwise launches take the groups last to first (and, inside each launch, the
+  // matrices last to first): the momentum pass then writes last the U the Newton-Schulz launch
+  // reads first (group 0, matrix 0), and the apply reads first the iterates that launch wrote
+  // last, while they are still in L2.
   std::vector<int> all_groups;
-  for (int g = 0; g < static_cast<int>(plans.size()); ++g) all_groups.push_back(g);
+  for (int g = static_cast<int>(plans.size()) - 1; g >= 0; --g) all_groups.push_back(g);
   // k Newton-Schulz iterations.  One persistent launch runs every phase of
   // every group (as many as fit in one parameter block), ordered phase by phase;
   // per-(phase, matrix) counters let a tile start as soon as the previous phase
