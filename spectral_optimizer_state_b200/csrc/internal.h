@@ -96,13 +96,13 @@ struct CapParams {
   double* partial;                 // [batch][blocks]
 };
 
-// One power iteration in one pass over W (u <- W v / |W v|, v <- W^T u / |W^T u|, sigma = |W^T u|):
-// p.x = v (read, then overwritten), p.y = u, p.partial [batch][nblk][cols] and tsq_partial
-// [batch][nblk + ceil(cols / 256)] scratch; nblk blocks of rows_per_block rows per matrix.
-// cols % 8 == 0, 16-byte aligned W, cols <= power_pass_max_cols().
+// `iters` power iterations, one pass over W each (u <- W v / |W v|, v <- W^T u / |W^T u|,
+// sigma = |W^T u|): p.x = v (read, then overwritten), p.y = u, p.partial [batch][nblk][cols]
+// and tsq_partial [batch][nblk + ceil(cols / 256)] scratch; nblk blocks of rows_per_block rows
+// per matrix.  cols % 8 == 0, 16-byte aligned W, cols <= power_pass_max_cols().
 int power_pass_max_cols();
 cudaError_t launch_power_iteration_fused(GemvParams& p, int batch, bool f32, float* tsq_partial, int nblk,
-                                         int rows_per_block, float* sigma, cudaStream_t s);
+                                         int rows_per_block, int iters, float* sigma, cudaStream_t s);
 cudaError_t launch_gemv_rows(const GemvParams& p, int batch, bool f32, cudaStream_t s);
 cudaError_t launch_gemv_cols(const GemvParams& p, int batch, bool f32, cudaStream_t s);
 cudaError_t launch_normalize(float* const* vecs_dev, int batch, int n, float* norm, cudaStream_t s);

@@ -1069,8 +1069,7 @@ muon_status muon_power_iteration(muon_ctx* c, const void* const* W, float* const
       gp.x[l] = v[l];
       gp.y[l] = u[l];
     }
-    for (int i = 0; i < iters; ++i)
-      MUON_CUDA(launch_power_iteration_fused(gp, batch, f32, tsq, nblk, rpb, sigma, s), "power iteration");
+    MUON_CUDA(launch_power_iteration_fused(gp, batch, f32, tsq, nblk, rpb, iters, sigma, s), "power iteration");
     return MUON_OK;
   }
   gp.rows_per_chunk = 64;

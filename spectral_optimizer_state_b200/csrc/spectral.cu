@@ -126,6 +126,16 @@ __global__ void __launch_bounds__(kThreads) gemv_cols_reduce_kernel(const __grid
   p.y[l][c] = s;
 }
 
+// Sum of n partial sums, by one warp: lane k adds partials k, k + 32, ... in order, then a fixed
+// xor-shuffle tree combines the lanes (the same order on every call); every lane gets the total.
+__device__ __forceinline__ double warp_sum_partials(const float* part, int n, int lane) {
+  double a = 0.0;
+  for (int k = lane; k < n; k += 32) a += static_cast<double>(part[k]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+  return a;
+}
+
 // 8 consecutive elements of W as packed 16-byte vectors (bf16: one, fp32: two) and their values.
 template <bool F32>
 struct Raw8w {
@@ -202,17 +212,34 @@ __device__ __forceinline__ float power_row(const Raw8w<F32> (&w)[NV], const floa
 // running sum z.  t goes to u (un-normalised), a fixed-order tree over the warps
 // gives one partial z per block, and each block writes its partial sum of t_r^2.
 // Requires cols % 8 == 0, 16-byte aligned rows and cols <= 256 * NV.
+//
+// v is read as v / |v| when zsq_prev is set (the un-normalised W^T t of the previous
+// iteration, whose squared norm is the sum of zsq_prev's zblk partials); the first
+// iteration takes the caller's vector as it is (u and the next v do not depend on its scale).
 template <bool F32, int NV>
 __global__ void __launch_bounds__(kThreads) power_pass_kernel(const __grid_constant__ GemvParams p,
-                                                              int rows_per_block, float* tsq_partial) {
+                                                              int rows_per_block, float* tsq_partial,
+                                                              const float* zsq_prev, int zblk) {
   extern __shared__ float sm[];
   float* vs = sm;                         // [cols]
   float* zs = sm + p.cols;                // [warps][cols]
   constexpr int kWarps = kThreads / 32;
+  __shared__ float s_inv;
   const int l = blockIdx.y;
   const float* x = p.x[l];
   const int C = p.cols;
-  for (int c = threadIdx.x; c < C; c += kThreads) vs[c] = x[c];
+  if (threadIdx.x < 32) {
+    float inv = 1.0f;
+    if (zsq_prev != nullptr) {
+      const float nz = static_cast<float>(sqrt(warp_sum_partials(zsq_prev + static_cast<long long>(l) * zblk, zblk,
+                                                                 threadIdx.x)));
+      inv = nz > 0.f ? 1.0f / nz : 0.f;
+    }
+    if (threadIdx.x == 0) s_inv = inv;
+  }
+  __syncthreads();
+  const float inv = s_inv;
+  for (int c = threadIdx.x; c < C; c += kThreads) vs[c] = x[c] * inv;
   __syncthreads();
   const void* W = p.w[l];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -329,15 +356,16 @@ __global__ void __launch_bounds__(kThreads) power_scale_kernel(const __grid_cons
                                                                const float* zsq_partial, float* sigma) {
   __shared__ float s_inv_t, s_inv_z;
   const int l = blockIdx.y;
-  if (threadIdx.x == 0) {
-    double tt = 0.0, zz = 0.0;
-    for (int b = 0; b < nblk; ++b) tt += tsq_partial[static_cast<long long>(l) * nblk + b];
-    for (int b = 0; b < zblk; ++b) zz += zsq_partial[static_cast<long long>(l) * zblk + b];
-    const float nt = static_cast<float>(sqrt(tt));
-    const float nz = static_cast<float>(sqrt(zz));
-    s_inv_t = nt > 0.f ? 1.0f / nt : 0.f;
-    s_inv_z = nz > 0.f ? 1.0f / nz : 0.f;
-    if (blockIdx.x == 0) sigma[l] = nt > 0.f ? nz / nt : 0.f;
+  if (threadIdx.x < 32) {
+    const double tt = warp_sum_partials(tsq_partial + static_cast<long long>(l) * nblk, nblk, threadIdx.x);
+    const double zz = warp_sum_partials(zsq_partial + static_cast<long long>(l) * zblk, zblk, threadIdx.x);
+    if (threadIdx.x == 0) {
+      const float nt = static_cast<float>(sqrt(tt));
+      const float nz = static_cast<float>(sqrt(zz));
+      s_inv_t = nt > 0.f ? 1.0f / nt : 0.f;
+      s_inv_z = nz > 0.f ? 1.0f / nz : 0.f;
+      if (blockIdx.x == 0) sigma[l] = nt > 0.f ? nz / nt : 0.f;
+    }
   }
   __syncthreads();
   const int i = blockIdx.x * kThreads + threadIdx.x;
@@ -509,12 +537,16 @@ cudaError_t launch_gemv_cols(const GemvParams& p, int batch, bool f32, cudaStrea
 int power_pass_max_cols() { return 256 * 8; }
 
 cudaError_t launch_power_iteration_fused(GemvParams& p, int batch, bool f32, float* tsq_partial, int nblk,
-                                         int rows_per_block, float* sigma, cudaStream_t s) {
+                                         int rows_per_block, int iters, float* sigma, cudaStream_t s) {
   const int nv = (p.cols + 255) / 256;
-  if (p.cols % 8 != 0 || nv < 1 || nv > 8) return cudaErrorInvalidValue;
+  if (p.cols % 8 != 0 || nv < 1 || nv > 8 || iters < 1) return cudaErrorInvalidValue;
   const size_t smem = sizeof(float) * p.cols * (1 + kThreads / 32);
   const dim3 grid(nblk, batch);
+  const int zblk = (p.cols + kThreads - 1) / kThreads;
+  float* zsq_partial = tsq_partial + static_cast<long long>(batch) * nblk;
   cudaError_t e = cudaSuccess;
+  for (int it = 0; it < iters; ++it) {
+    const float* zprev = it == 0 ? nullptr : zsq_partial;
 #define MUON_POWER_CASE(NVV)                                                                          \
   case NVV: {                                                                                        \
     auto kern = f32 ? power_pass_kernel<true, NVV> : power_pass_kernel<false, NVV>;                 \
@@ -522,27 +554,26 @@ cudaError_t launch_power_iteration_fused(GemvParams& p, int batch, bool f32, flo
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)); \
       if (e != cudaSuccess) return e;                                                                \
     }                                                                                                \
-    kern<<<grid, kThreads, smem, s>>>(p, rows_per_block, tsq_partial);                               \
+    kern<<<grid, kThreads, smem, s>>>(p, rows_per_block, tsq_partial, zprev, zblk);                 \
     break;                                                                                           \
   }
-  switch (nv) {
-    MUON_POWER_CASE(1)
-    MUON_POWER_CASE(2)
-    MUON_POWER_CASE(3)
-    MUON_POWER_CASE(4)
-    MUON_POWER_CASE(5)
-    MUON_POWER_CASE(6)
-    MUON_POWER_CASE(7)
-    MUON_POWER_CASE(8)
-  }
+    switch (nv) {
+      MUON_POWER_CASE(1)
+      MUON_POWER_CASE(2)
+      MUON_POWER_CASE(3)
+      MUON_POWER_CASE(4)
+      MUON_POWER_CASE(5)
+      MUON_POWER_CASE(6)
+      MUON_POWER_CASE(7)
+      MUON_POWER_CASE(8)
+    }
 #undef MUON_POWER_CASE
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const int zblk = (p.cols + kThreads - 1) / kThreads;
-  float* zsq_partial = tsq_partial + static_cast<long long>(batch) * nblk;
-  power_reduce_kernel<<<dim3(zblk, batch), kThreads, 0, s>>>(p, nblk, zsq_partial);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    power_reduce_kernel<<<dim3(zblk, batch), kThreads, 0, s>>>(p, nblk, zsq_partial);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   const int eblk = (std::max(p.rows, p.cols) + kThreads - 1) / kThreads;
   power_scale_kernel<<<dim3(eblk, batch), kThreads, 0, s>>>(p, nblk, tsq_partial, zblk, zsq_partial, sigma);
   return cudaGetLastError();
