@@ -97,12 +97,16 @@ struct CapParams {
 };
 
 // `iters` power iterations, one pass over W each (u <- W v / |W v|, v <- W^T u / |W^T u|,
-// sigma = |W^T u|): p.x = v (read, then overwritten), p.y = u, p.partial [batch][nblk][cols]
-// and tsq_partial [batch][nblk + ceil(cols / 256)] scratch; nblk blocks of rows_per_block rows
-// per matrix.  cols % 8 == 0, 16-byte aligned W, cols <= power_pass_max_cols().
+// sigma = |W^T u|), in one cooperative launch when the blocks fit on the GPU at once, else one
+// launch per iteration: p.x = v (read, then overwritten), p.y = u; p.partial
+// 2 x [batch][nblk][cols] (two iterations' partials), tsq_partial [batch][nblk] and
+// counters [2 * batch] scratch (zeroed here).  nblk from power_pass_blocks; cols % 8 == 0,
+// 16-byte aligned W, cols <= power_pass_max_cols().  Wait timeouts set `status`.
 int power_pass_max_cols();
-cudaError_t launch_power_iteration_fused(GemvParams& p, int batch, bool f32, float* tsq_partial, int nblk,
-                                         int rows_per_block, int iters, float* sigma, cudaStream_t s);
+int power_pass_blocks(int rows, int cols, int batch, bool f32, int sm_count);
+cudaError_t launch_power_iteration_stream(GemvParams& p, int batch, bool f32, int nblk, int iters,
+                                          float* tsq_partial, unsigned* counters, float* sigma, int* status,
+                                          int sm_count, cudaStream_t s);
 cudaError_t launch_gemv_rows(const GemvParams& p, int batch, bool f32, cudaStream_t s);
 cudaError_t launch_gemv_cols(const GemvParams& p, int batch, bool f32, cudaStream_t s);
 cudaError_t launch_normalize(float* const* vecs_dev, int batch, int n, float* norm, cudaStream_t s);

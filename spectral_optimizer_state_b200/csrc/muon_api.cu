@@ -1057,19 +1057,22 @@ muon_status muon_power_iteration(muon_ctx* c, const void* const* W, float* const
   for (int l = 0; l < batch && fused; ++l)
     if (reinterpret_cast<uintptr_t>(W[l]) % 16) fused = false;
   if (fused) {
-    // one pass over W per iteration (power_pass_kernel); 64 rows per block
-    const int rpb = 64;
-    const int nblk = (rows + rpb - 1) / rpb;
-    const size_t part_bytes = align_up(sizeof(float) * batch * nblk * cols, 256);
-    muon_status st = ensure_aux(c, part_bytes + sizeof(float) * batch * (nblk + (cols + 255) / 256));
+    // one pass over W and one launch per iteration (power_stream_kernel)
+    const int nblk = power_pass_blocks(rows, cols, batch, f32, c->sm_count);
+    const size_t part_bytes = align_up(2 * sizeof(float) * batch * nblk * cols, 256);
+    const size_t tsq_bytes = align_up(sizeof(float) * batch * nblk, 256);
+    muon_status st = ensure_aux(c, part_bytes + tsq_bytes + 2 * sizeof(unsigned) * batch);
     if (st != MUON_OK) return st;
     gp.partial = static_cast<float*>(c->d_aux);
     float* tsq = reinterpret_cast<float*>(static_cast<char*>(c->d_aux) + part_bytes);
+    unsigned* done = reinterpret_cast<unsigned*>(static_cast<char*>(c->d_aux) + part_bytes + tsq_bytes);
     for (int l = 0; l < batch; ++l) {
       gp.x[l] = v[l];
       gp.y[l] = u[l];
     }
-    MUON_CUDA(launch_power_iteration_fused(gp, batch, f32, tsq, nblk, rpb, iters, sigma, s), "power iteration");
+    MUON_CUDA(launch_power_iteration_stream(gp, batch, f32, nblk, iters, tsq, done, sigma, c->d_status,
+                                            c->sm_count, s),
+              "power iteration");
     return MUON_OK;
   }
   gp.rows_per_chunk = 64;

@@ -143,163 +143,414 @@ struct Raw8w {
 };
 
 template <bool F32>
-__device__ __forceinline__ void load_raw(const void* base, long long e, Raw8w<F32>& r) {
-  const uint4* p = F32 ? reinterpret_cast<const uint4*>(static_cast<const float*>(base) + e)
-                       : reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + e);
+__device__ __forceinline__ void load_raw_smem(const uint8_t* row, int c, Raw8w<F32>& r) {
+  const uint4* q = reinterpret_cast<const uint4*>(row + static_cast<size_t>(c) * (F32 ? 4 : 2));
 #pragma unroll
-  for (int i = 0; i < (F32 ? 2 : 1); ++i) r.q[i] = p[i];
+  for (int i = 0; i < (F32 ? 2 : 1); ++i) r.q[i] = q[i];
 }
 
+// Where column c of v sits in the streaming pass's shared copy: within each 256-column chunk,
+// the first four of every eight columns come first (128 values), the last four after them.
+// Lane k's columns 8k..8k+7 of a chunk are then two 16-byte reads at 4k and 128 + 4k, which
+// fall in distinct banks across each quarter warp.  The copy holds cols rounded up to 256.
+__device__ __forceinline__ int vs_index(int c) {
+  return (c & ~255) | ((c & 4) << 5) | (((c & 255) >> 3) << 2) | (c & 3);
+}
+
+// Packed pairs of fp32 values and the sm_100a two-lane FMA (each lane an ordinary fp32 fma,
+// rounded to nearest): the streaming pass's dot products and z updates issue half the FMAs.
+__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void unpack_f2(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+
+__device__ __forceinline__ uint64_t fma_f2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// The 8 values of a packed 16-byte load as four (even, odd) column pairs.
 template <bool F32>
-__device__ __forceinline__ void unpack_raw(const Raw8w<F32>& r, float (&x)[8]) {
+__device__ __forceinline__ void raw_to_pairs(const Raw8w<F32>& r, uint64_t (&x)[4]) {
   if (F32) {
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      x[4 * i] = __uint_as_float(r.q[i].x);
-      x[4 * i + 1] = __uint_as_float(r.q[i].y);
-      x[4 * i + 2] = __uint_as_float(r.q[i].z);
-      x[4 * i + 3] = __uint_as_float(r.q[i].w);
+      x[2 * i] = pack_f2(__uint_as_float(r.q[i].x), __uint_as_float(r.q[i].y));
+      x[2 * i + 1] = pack_f2(__uint_as_float(r.q[i].z), __uint_as_float(r.q[i].w));
     }
   } else {
     const uint32_t w[4] = {r.q[0].x, r.q[0].y, r.q[0].z, r.q[0].w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      x[2 * i] = __uint_as_float(w[i] << 16);
-      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
+    for (int i = 0; i < 4; ++i) x[i] = pack_f2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
   }
 }
 
-// t_r = W[r, :] . v and z += t_r W[r, :] for one row held (packed) in registers.
+// Two rows at once (the second when has1), both read from their shared-memory stage:
+// t = W[r, :] . v for each, then z += t W[r, :], on (even, odd) column pairs.  Each dot product
+// runs as two pair chains (the first and last four columns of every eight); the two rows' chains
+// and shuffle trees interleave.  Rows of up to 512 columns keep their pairs in registers for the
+// z update; longer ones read the stage again rather than hold them across the trees.
 template <bool F32, int NV>
-__device__ __forceinline__ float power_row(const Raw8w<F32> (&w)[NV], const float* vs, int C, int lane,
-                                           float (&z)[NV][8]) {
-  float dot = 0.f;
+__device__ __forceinline__ void power_rows2(const uint8_t* row0, const uint8_t* row1, bool has1, const float* vs,
+                                            int C, int lane, uint64_t (&z)[NV][4], float& t0, float& t1) {
+  constexpr bool kKeep = NV <= 2;
+  uint64_t x0[kKeep ? NV : 1][4], x1[kKeep ? NV : 1][4];
+  uint64_t a0 = 0, b0 = 0, a1 = 0, b1 = 0;  // (+0.0f, +0.0f) pairs
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int c = 8 * lane + 256 * i;
     if (c < C) {
-      float x[8];
-      unpack_raw<F32>(w[i], x);
-      // 16-byte reads of v: a lane's 8 values are contiguous, so scalar reads would be 8-way
-      // bank conflicts across the warp
-      const float4 va = *reinterpret_cast<const float4*>(vs + c);
-      const float4 vb = *reinterpret_cast<const float4*>(vs + c + 4);
-      const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+      const ulonglong2 lo = *reinterpret_cast<const ulonglong2*>(vs + 256 * i + 4 * lane);
+      const ulonglong2 hi = *reinterpret_cast<const ulonglong2*>(vs + 256 * i + 128 + 4 * lane);
+      Raw8w<F32> w;
+      uint64_t x[4];
+      load_raw_smem<F32>(row0, c, w);
+      raw_to_pairs<F32>(w, x);
+      a0 = fma_f2(x[0], lo.x, a0);
+      a0 = fma_f2(x[1], lo.y, a0);
+      b0 = fma_f2(x[2], hi.x, b0);
+      b0 = fma_f2(x[3], hi.y, b0);
+      if (kKeep)
 #pragma unroll
-      for (int t = 0; t < 8; ++t) dot = fmaf(x[t], vv[t], dot);
-    }
-  }
+        for (int k = 0; k < 4; ++k) x0[kKeep ? i : 0][k] = x[k];
+      if (has1) {
+        load_raw_smem<F32>(row1, c, w);
+        raw_to_pairs<F32>(w, x);
+        a1 = fma_f2(x[0], lo.x, a1);
+        a1 = fma_f2(x[1], lo.y, a1);
+        b1 = fma_f2(x[2], hi.x, b1);
+        b1 = fma_f2(x[3], hi.y, b1);
+        if (kKeep)
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c = 8 * lane + 256 * i;
-    if (c < C) {
-      float x[8];
-      unpack_raw<F32>(w[i], x);
-#pragma unroll
-      for (int t = 0; t < 8; ++t) z[i][t] = fmaf(dot, x[t], z[i][t]);
-    }
-  }
-  return dot;
-}
-
-// One pass over the rows of W for a whole power iteration.  With t = W v, the
-// next iterate's W^T u is W^T t / |t|, and W^T t = sum_r t_r W[r, :]: each warp
-// loads its rows once (two rows in flight, NV packed 16-byte vectors per lane
-// each), forms t_r against v (staged in shared memory) and adds t_r W[r, :] to its
-// running sum z.  t goes to u (un-normalised), a fixed-order tree over the warps
-// gives one partial z per block, and each block writes its partial sum of t_r^2.
-// Requires cols % 8 == 0, 16-byte aligned rows and cols <= 256 * NV.
-//
-// v is read as v / |v| when zsq_prev is set (the un-normalised W^T t of the previous
-// iteration, whose squared norm is the sum of zsq_prev's zblk partials); the first
-// iteration takes the caller's vector as it is (u and the next v do not depend on its scale).
-template <bool F32, int NV>
-__global__ void __launch_bounds__(kThreads) power_pass_kernel(const __grid_constant__ GemvParams p,
-                                                              int rows_per_block, float* tsq_partial,
-                                                              const float* zsq_prev, int zblk) {
-  extern __shared__ float sm[];
-  float* vs = sm;                         // [cols]
-  float* zs = sm + p.cols;                // [warps][cols]
-  constexpr int kWarps = kThreads / 32;
-  __shared__ float s_inv;
-  const int l = blockIdx.y;
-  const float* x = p.x[l];
-  const int C = p.cols;
-  if (threadIdx.x < 32) {
-    float inv = 1.0f;
-    if (zsq_prev != nullptr) {
-      const float nz = static_cast<float>(sqrt(warp_sum_partials(zsq_prev + static_cast<long long>(l) * zblk, zblk,
-                                                                 threadIdx.x)));
-      inv = nz > 0.f ? 1.0f / nz : 0.f;
-    }
-    if (threadIdx.x == 0) s_inv = inv;
-  }
-  __syncthreads();
-  const float inv = s_inv;
-  for (int c = threadIdx.x; c < C; c += kThreads) vs[c] = x[c] * inv;
-  __syncthreads();
-  const void* W = p.w[l];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r_beg = blockIdx.x * rows_per_block;
-  const int r_end = min(p.rows, r_beg + rows_per_block);
-  float z[NV][8];
-#pragma unroll
-  for (int i = 0; i < NV; ++i)
-#pragma unroll
-    for (int t = 0; t < 8; ++t) z[i][t] = 0.f;
-  float tsq = 0.f;
-  for (int r0 = r_beg + warp; r0 < r_end; r0 += 2 * kWarps) {
-    const int r1 = r0 + kWarps;
-    const bool two = r1 < r_end;
-    Raw8w<F32> w0[NV], w1[NV];
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const int c = 8 * lane + 256 * i;
-      if (c < C) {
-        load_raw<F32>(W, static_cast<long long>(r0) * C + c, w0[i]);
-        if (two) load_raw<F32>(W, static_cast<long long>(r1) * C + c, w1[i]);
+          for (int k = 0; k < 4; ++k) x1[kKeep ? i : 0][k] = x[k];
       }
     }
-    const float t0 = power_row<F32, NV>(w0, vs, C, lane, z);
-    if (lane == 0) p.y[l][r0] = t0;
-    tsq = fmaf(t0, t0, tsq);
-    if (two) {
-      const float t1 = power_row<F32, NV>(w1, vs, C, lane, z);
-      if (lane == 0) p.y[l][r1] = t1;
-      tsq = fmaf(t1, t1, tsq);
-    }
   }
-  // warps' z into shared memory, then a fixed-order sum over the warps
+  float p, q, r, s;
+  unpack_f2(a0, p, q);
+  unpack_f2(b0, r, s);
+  float d0 = (p + q) + (r + s);
+  unpack_f2(a1, p, q);
+  unpack_f2(b1, r, s);
+  float d1 = (p + q) + (r + s);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    d0 += __shfl_xor_sync(0xffffffffu, d0, o);
+    d1 += __shfl_xor_sync(0xffffffffu, d1, o);
+  }
+  const uint64_t dd0 = pack_f2(d0, d0), dd1 = pack_f2(d1, d1);
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int c = 8 * lane + 256 * i;
     if (c < C) {
-      float4* d = reinterpret_cast<float4*>(zs + warp * C + c);
-      d[0] = make_float4(z[i][0], z[i][1], z[i][2], z[i][3]);
-      d[1] = make_float4(z[i][4], z[i][5], z[i][6], z[i][7]);
+      uint64_t x[4];
+      if (kKeep) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x[k] = x0[kKeep ? i : 0][k];
+      } else {
+        Raw8w<F32> w;
+        load_raw_smem<F32>(row0, c, w);
+        raw_to_pairs<F32>(w, x);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) z[i][k] = fma_f2(dd0, x[k], z[i][k]);
+      if (has1) {
+        if (kKeep) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) x[k] = x1[kKeep ? i : 0][k];
+        } else {
+          Raw8w<F32> w;
+          load_raw_smem<F32>(row1, c, w);
+          raw_to_pairs<F32>(w, x);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) z[i][k] = fma_f2(dd1, x[k], z[i][k]);
+      }
     }
   }
-  __syncthreads();
-  float* out = p.partial + (static_cast<long long>(l) * gridDim.x + blockIdx.x) * C;
-  for (int c = threadIdx.x; c < C; c += kThreads) {
-    float a = 0.f;
+  t0 = d0;
+  t1 = d1;
+}
+
+// z[k] = sum over b = 0, 1, ... (in that order) of part[b][c_k], c_k = tid + k * nthr (zero past
+// cols; at most 8 columns per thread): every column of this thread at once, four partials ahead,
+// so the loads overlap.
+__device__ __forceinline__ void sum_partials(const float* part, int nblk, int C, int tid, int nthr, float (&z)[8]) {
 #pragma unroll
-    for (int k = 0; k < kWarps; ++k) a += zs[k * C + c];
-    out[c] = a;
+  for (int k = 0; k < 8; ++k) z[k] = 0.f;
+  int b = 0;
+  for (; b + 4 <= nblk; b += 4) {
+    float q[8][4];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int c = tid + k * nthr;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) q[k][j] = c < C ? __ldcg(part + static_cast<long long>(b + j) * C + c) : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) z[k] += q[k][j];
   }
-  // the warps' sums of t_r^2 (every lane holds its warp's), in warp order
-  __shared__ float tq[kWarps];
-  if (lane == 0) tq[warp] = tsq;
-  __syncthreads();
+  for (; b < nblk; ++b)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int c = tid + k * nthr;
+      if (c < C) z[k] += __ldcg(part + static_cast<long long>(b) * C + c);
+    }
+}
+
+// Sum of squares of this thread's columns over the first nwarps warps, in a fixed order;
+// every participating thread gets it.  `bar` synchronises exactly those warps.
+template <typename Bar>
+__device__ __forceinline__ double sum_squares(const float (&z)[8], double* scratch, int nwarps, Bar&& bar) {
+  double ss = 0.0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) ss += static_cast<double>(z[k]) * z[k];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = ss;
+  bar();
+  double tot = 0.0;
+  for (int k = 0; k < nwarps; ++k) tot += scratch[k];
+  return tot;
+}
+
+// One pass over the rows of W per power iteration.  With t = W v, the next W^T u is
+// W^T t / |t|, and W^T t = sum_r t_r W[r, :], so a row read once gives both its t_r and its
+// share of z = W^T t.  A block owns rows_per_block consecutive rows of one matrix: a producer
+// warp streams them through a ring of shared-memory stages (eight consecutive rows, one 1-D
+// bulk copy, per stage), and each of the eight consumer warps takes one row of each of two
+// stages at a time, forms t_r against v (staged in shared memory) and adds t_r W[r, :] to its
+// running z.  The warps' z are summed in warp order into one partial per block, which also
+// records its sum of t_r^2.
+//
+// One launch runs iterations it0 .. it1-1.  Iteration it > 0 starts from the previous
+// iteration's partials, which every block sums in block order (z, then v = z / |z|); within a
+// launch a block first waits (bounded) until all blocks of its matrix have written them (a
+// per-matrix counter), which needs the launch's blocks co-resident (a cooperative launch).
+// The producer does not wait: W does not change, so it streams the next iteration's rows while
+// the consumers wait.  Iteration 0 takes the caller's v as it is (u and the next v do not depend
+// on its scale).  After the last iteration, the last block of a matrix to finish writes
+// v = z / |z|, u = t / |t| and sigma = |z| / |t| = |W^T u|.  A zero t leaves u, v at zero and
+// sigma 0.  Requires cols % 8 == 0, 16-byte aligned W and cols <= 256 * NV <= 2048.
+constexpr int kPowerWarps = 8;                         // consumer warps: a stage holds a row for each
+constexpr int kPowerThreads = 32 * (kPowerWarps + 1);  // and one producer warp
+constexpr int kPowerMaxBlocks = 64;                    // block partials per matrix
+constexpr int kPowerCols = 8;                          // columns per thread in the partial sums
+constexpr uint64_t kPowerDrainNs = 200000000ull;
+
+struct PowerArgs {
+  int rows_per_block, stages, nblk, iters;  // iters: of the whole call
+  int it0, it1;                             // the iterations this launch runs
+  float* part[2];      // [batch][nblk][cols] each: z partials of even / odd iterations
+  float* tsq_partial;  // [batch][nblk]: each block's sum of t_r^2 (last iteration written)
+  unsigned* sync;      // [batch]: partial sets written in this call (blocks x iterations)
+  unsigned* done;      // [batch]: blocks through the final iteration
+  float* sigma;        // [batch], written after the final iteration
+  int* status;         // device status word (wait timeouts)
+};
+
+// Two blocks per SM where z's registers allow it (rows up to 1280 columns, bf16 up to 1536).
+template <bool F32, int NV>
+__global__ void __launch_bounds__(kPowerThreads, (NV <= 5 || (!F32 && NV <= 6)) ? 2 : 1) power_stream_kernel(
+    const __grid_constant__ GemvParams p, const PowerArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float tq[kPowerWarps];
+  __shared__ double sq[kPowerWarps + 1];
+  __shared__ float s_tt;
+  __shared__ int s_last;
+  __shared__ volatile int abort_flag;
+  constexpr int kConsumers = 32 * kPowerWarps;
+  const int C = p.cols;
+  const int Cr = (C + 255) & ~255;
+  const uint32_t row_bytes = static_cast<uint32_t>(C) * (F32 ? 4u : 2u);
+  const uint32_t stage_bytes = kPowerWarps * row_bytes;
+  uint8_t* ring = smem;
+  float* vs = reinterpret_cast<float*>(smem + static_cast<size_t>(a.stages) * stage_bytes);  // [Cr], permuted
+  float* zs = vs + Cr;                                                                         // [C]
+  const uint32_t bar0 = smem_addr(zs + C);  // full[stages], then empty[stages]
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (a.stages + s); };
+  const int l = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r_beg = blockIdx.x * a.rows_per_block;
+  const int r_end = min(p.rows, r_beg + a.rows_per_block);
+  const int nst = (r_end - r_beg + kPowerWarps - 1) / kPowerWarps;
   if (threadIdx.x == 0) {
-    float a = 0.f;
-#pragma unroll
-    for (int k = 0; k < kWarps; ++k) a += tq[k];
-    tsq_partial[static_cast<long long>(l) * gridDim.x + blockIdx.x] = a;
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), kPowerWarps);
+    }
+    abort_flag = 0;
+    fence_barrier_init();
   }
+  __syncthreads();
+  const int niter = a.it1 - a.it0;
+  if (warp == kPowerWarps) {
+    // ------------------------------------------------ producer (one thread): every iteration's rows
+    if (lane == 0) {
+      const uint8_t* src = static_cast<const uint8_t*>(p.w[l]) + static_cast<size_t>(r_beg) * row_bytes;
+      const int total = niter * nst;
+      int g = 0;
+      for (; g < total; ++g) {
+        const int s = g % a.stages;
+        const int j = g % nst;
+        if (g >= a.stages &&
+            !mbar_wait_bounded(empty_bar(s), static_cast<uint32_t>((g / a.stages) - 1) & 1u, &abort_flag, a.status))
+          break;
+        const int nr = min(kPowerWarps, r_end - (r_beg + kPowerWarps * j));
+        const uint32_t bytes = static_cast<uint32_t>(nr) * row_bytes;
+        mbar_arrive_expect_tx(full_bar(s), bytes);
+        bulk_load_1d(smem_addr(ring + static_cast<size_t>(s) * stage_bytes), src + static_cast<size_t>(j) * stage_bytes,
+                     bytes, full_bar(s));
+      }
+      if (g < total) {
+        // gave up: let the copies in flight land before the block exits
+        const int n = min(g, a.stages);
+        for (int k = g - n; k < g; ++k) {
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(full_bar(k % a.stages), static_cast<uint32_t>(k / a.stages) & 1u))
+            if (global_timer_ns() - t0 > kPowerDrainNs) break;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------ consumers
+    for (int it = a.it0; it < a.it1; ++it) {
+      // v for this iteration
+      if (it == 0) {
+        const float* x = p.x[l];
+        for (int c = threadIdx.x; c < C; c += kConsumers) vs[vs_index(c)] = x[c];
+      } else {
+        if (it > a.it0) {
+          // the previous iteration's partials of this matrix, written by this launch's blocks
+          if (threadIdx.x == 0 && !abort_flag &&
+              !wait_counter_bounded(a.sync + l, static_cast<unsigned>(a.nblk * (it - a.it0)), &abort_flag, a.status))
+            abort_flag = 1;
+          named_barrier_sync(1, kConsumers);
+        }
+        float zc[kPowerCols];
+        sum_partials(a.part[(it - 1) & 1] + static_cast<long long>(l) * a.nblk * C, a.nblk, C, threadIdx.x,
+                     kConsumers, zc);
+        const double ss = sum_squares(zc, sq, kPowerWarps, [] { named_barrier_sync(1, kConsumers); });
+        const float nz = static_cast<float>(sqrt(ss));
+        const float inv = nz > 0.f ? 1.0f / nz : 0.f;
+#pragma unroll
+        for (int k = 0; k < kPowerCols; ++k) {
+          const int c = threadIdx.x + k * kConsumers;
+          if (c < C) vs[vs_index(c)] = zc[k] * inv;
+        }
+      }
+      named_barrier_sync(1, kConsumers);
+      uint64_t z[NV][4];  // (even, odd) column pairs of this lane's running W^T t
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) z[i][k] = 0;
+      float tsq = 0.f;
+      const int gbase = (it - a.it0) * nst;
+      // After a failed wait (the status word says so) a warp skips the rest of its rows, but every
+      // consumer warp still takes the same named barriers below, so none of them is left waiting.
+      for (int j = 0; j < nst && !abort_flag; j += 2) {
+        const bool two = j + 1 < nst;
+        const int g0 = gbase + j, g1 = g0 + 1;
+        const int s0 = g0 % a.stages, s1 = g1 % a.stages;
+        if (!mbar_wait_bounded(full_bar(s0), static_cast<uint32_t>(g0 / a.stages) & 1u, &abort_flag, a.status) ||
+            (two && !mbar_wait_bounded(full_bar(s1), static_cast<uint32_t>(g1 / a.stages) & 1u, &abort_flag,
+                                       a.status)))
+          break;
+        const int r0 = r_beg + kPowerWarps * j + warp, r1 = r0 + kPowerWarps;
+        const bool has1 = two && r1 < r_end;
+        if (r0 < r_end) {
+          const uint8_t* row0 = ring + static_cast<size_t>(s0) * stage_bytes + static_cast<size_t>(warp) * row_bytes;
+          const uint8_t* row1 = ring + static_cast<size_t>(s1) * stage_bytes + static_cast<size_t>(warp) * row_bytes;
+          float t0, t1;
+          power_rows2<F32, NV>(row0, row1, has1, vs, C, lane, z, t0, t1);
+          if (lane == 0) {
+            p.y[l][r0] = t0;
+            if (has1) p.y[l][r1] = t1;
+          }
+          tsq = fmaf(t0, t0, tsq);
+          if (has1) tsq = fmaf(t1, t1, tsq);
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(empty_bar(s0));
+          if (two) mbar_arrive(empty_bar(s1));
+        }
+      }
+      // the block's partial: the warps' z added into zs one warp after another
+      for (int w = 0; w < kPowerWarps; ++w) {
+        if (warp == w) {
+#pragma unroll
+          for (int i = 0; i < NV; ++i) {
+            const int c = 8 * lane + 256 * i;
+            if (c < C) {
+              ulonglong2* d = reinterpret_cast<ulonglong2*>(zs + c);
+              if (w == 0) {
+                d[0] = make_ulonglong2(z[i][0], z[i][1]);
+                d[1] = make_ulonglong2(z[i][2], z[i][3]);
+              } else {
+                const ulonglong2 e0 = d[0], e1 = d[1];
+                const uint64_t one = pack_f2(1.0f, 1.0f);
+                d[0] = make_ulonglong2(fma_f2(e0.x, one, z[i][0]), fma_f2(e0.y, one, z[i][1]));
+                d[1] = make_ulonglong2(fma_f2(e1.x, one, z[i][2]), fma_f2(e1.y, one, z[i][3]));
+              }
+            }
+          }
+          if (lane == 0) tq[w] = tsq;
+        }
+        named_barrier_sync(1, kConsumers);
+      }
+      float* part = a.part[it & 1] + (static_cast<long long>(l) * a.nblk + blockIdx.x) * C;
+      for (int c = threadIdx.x; c < C; c += kConsumers) part[c] = zs[c];
+      if (threadIdx.x == 0) {
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < kPowerWarps; ++k) acc += tq[k];
+        a.tsq_partial[static_cast<long long>(l) * a.nblk + blockIdx.x] = acc;
+      }
+      __threadfence();
+      named_barrier_sync(1, kConsumers);  // zs is free again, and every store of the set is fenced
+      if (threadIdx.x == 0) red_release_gpu_add(a.sync + l, 1u);
+    }
+  }
+  if (a.it1 < a.iters) return;
+  // after the final iteration: the last block of this matrix to get here writes u, v and sigma
+  __syncthreads();
+  if (abort_flag) return;
+  if (threadIdx.x == 0) s_last = atomicAdd(a.done + l, 1u) == static_cast<unsigned>(a.nblk - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  float zc[kPowerCols];
+  sum_partials(a.part[(a.iters - 1) & 1] + static_cast<long long>(l) * a.nblk * C, a.nblk, C, threadIdx.x,
+               kPowerThreads, zc);
+  if (warp == 0) {
+    const double tt = warp_sum_partials(a.tsq_partial + static_cast<long long>(l) * a.nblk, a.nblk, lane);
+    if (lane == 0) s_tt = static_cast<float>(sqrt(tt));
+  }
+  const double zz = sum_squares(zc, sq, kPowerWarps + 1, [] { __syncthreads(); });
+  const float nz = static_cast<float>(sqrt(zz));
+  const float inv_z = nz > 0.f ? 1.0f / nz : 0.f;
+  float* v = const_cast<float*>(p.x[l]);
+#pragma unroll
+  for (int k = 0; k < kPowerCols; ++k) {
+    const int c = threadIdx.x + k * kPowerThreads;
+    if (c < C) v[c] = zc[k] * inv_z;
+  }
+  const float nt = s_tt;
+  const float inv_t = nt > 0.f ? 1.0f / nt : 0.f;
+  float* u = p.y[l];
+  for (int r = threadIdx.x; r < p.rows; r += kPowerThreads) u[r] = __ldcg(u + r) * inv_t;
+  if (threadIdx.x == 0) a.sigma[l] = nt > 0.f ? nz / nt : 0.f;
 }
 
 template <typename T>
@@ -317,60 +568,6 @@ __device__ __forceinline__ T block_sum(T v, T* scratch) {
     for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
   }
   return r;
-}
-
-// z = the pass's block partials summed in block order (one thread per column, the loads
-// eight blocks ahead of the additions); z goes to v un-normalised and each block writes
-// its partial sum of z^2.  grid (column blocks, batch).
-__global__ void __launch_bounds__(kThreads) power_reduce_kernel(const __grid_constant__ GemvParams p, int nblk,
-                                                                float* zsq_partial) {
-  __shared__ double scratch[kThreads / 32];
-  const int l = blockIdx.y;
-  const int C = p.cols;
-  const int c = blockIdx.x * kThreads + threadIdx.x;
-  double zz = 0.0;
-  if (c < C) {
-    const float* part = p.partial + static_cast<long long>(l) * nblk * C + c;
-    float a = 0.f;
-    int b = 0;
-    for (; b + 8 <= nblk; b += 8) {
-      float q[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) q[k] = part[static_cast<long long>(b + k) * C];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) a += q[k];
-    }
-    for (; b < nblk; ++b) a += part[static_cast<long long>(b) * C];
-    const_cast<float*>(p.x[l])[c] = a;
-    zz = static_cast<double>(a) * a;
-  }
-  const double tot = block_sum<double>(zz, scratch);
-  if (threadIdx.x == 0) zsq_partial[static_cast<long long>(l) * gridDim.x + blockIdx.x] = static_cast<float>(tot);
-}
-
-// u = t / |t|, v = z / |z|, sigma = |z| / |t| (= |W^T u|), from the partial sums of t^2 and z^2
-// (summed in order by every block).  A zero t leaves u, v at zero and sigma 0.
-// grid (element blocks over max(rows, cols), batch).
-__global__ void __launch_bounds__(kThreads) power_scale_kernel(const __grid_constant__ GemvParams p, int nblk,
-                                                               const float* tsq_partial, int zblk,
-                                                               const float* zsq_partial, float* sigma) {
-  __shared__ float s_inv_t, s_inv_z;
-  const int l = blockIdx.y;
-  if (threadIdx.x < 32) {
-    const double tt = warp_sum_partials(tsq_partial + static_cast<long long>(l) * nblk, nblk, threadIdx.x);
-    const double zz = warp_sum_partials(zsq_partial + static_cast<long long>(l) * zblk, zblk, threadIdx.x);
-    if (threadIdx.x == 0) {
-      const float nt = static_cast<float>(sqrt(tt));
-      const float nz = static_cast<float>(sqrt(zz));
-      s_inv_t = nt > 0.f ? 1.0f / nt : 0.f;
-      s_inv_z = nz > 0.f ? 1.0f / nz : 0.f;
-      if (blockIdx.x == 0) sigma[l] = nt > 0.f ? nz / nt : 0.f;
-    }
-  }
-  __syncthreads();
-  const int i = blockIdx.x * kThreads + threadIdx.x;
-  if (i < p.cols) const_cast<float*>(p.x[l])[i] *= s_inv_z;
-  if (i < p.rows) p.y[l][i] *= s_inv_t;
 }
 
 struct VecParams {
@@ -536,28 +733,111 @@ cudaError_t launch_gemv_cols(const GemvParams& p, int batch, bool f32, cudaStrea
 
 int power_pass_max_cols() { return 256 * 8; }
 
-cudaError_t launch_power_iteration_fused(GemvParams& p, int batch, bool f32, float* tsq_partial, int nblk,
-                                         int rows_per_block, int iters, float* sigma, cudaStream_t s) {
-  const int nv = (p.cols + 255) / 256;
-  if (p.cols % 8 != 0 || nv < 1 || nv > 8 || iters < 1) return cudaErrorInvalidValue;
-  const size_t smem = sizeof(float) * p.cols * (1 + kThreads / 32);
-  const dim3 grid(nblk, batch);
-  const int zblk = (p.cols + kThreads - 1) / kThreads;
-  float* zsq_partial = tsq_partial + static_cast<long long>(batch) * nblk;
-  cudaError_t e = cudaSuccess;
-  for (int it = 0; it < iters; ++it) {
-    const float* zprev = it == 0 ? nullptr : zsq_partial;
-#define MUON_POWER_CASE(NVV)                                                                          \
-  case NVV: {                                                                                        \
-    auto kern = f32 ? power_pass_kernel<true, NVV> : power_pass_kernel<false, NVV>;                 \
-    if (smem > 48 * 1024) {                                                                          \
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)); \
-      if (e != cudaSuccess) return e;                                                                \
-    }                                                                                                \
-    kern<<<grid, kThreads, smem, s>>>(p, rows_per_block, tsq_partial, zprev, zblk);                 \
-    break;                                                                                           \
+namespace {
+
+template <bool F32, int NV>
+cudaError_t power_launch(const GemvParams& p, const PowerArgs& a, dim3 grid, size_t smem, bool cooperative,
+                         cudaStream_t s) {
+  auto kern = power_stream_kernel<F32, NV>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
   }
+  if (!cooperative) {
+    kern<<<grid, kPowerThreads, smem, s>>>(p, a);
+    return cudaGetLastError();
+  }
+  void* args[] = {const_cast<GemvParams*>(&p), const_cast<PowerArgs*>(&a)};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), grid, dim3(kPowerThreads), args, smem, s);
+}
+
+template <bool F32, int NV>
+int power_blocks_per_sm(size_t smem) {
+  auto kern = power_stream_kernel<F32, NV>;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    return 0;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kPowerThreads, smem) != cudaSuccess) return 0;
+  return n;
+}
+
+size_t power_smem_bytes(int cols, bool f32, int& stages) {
+  const size_t stage_bytes = kPowerWarps * static_cast<size_t>(cols) * (f32 ? 4 : 2);
+  // ~96 KB of rows in flight per block (two blocks per SM), two to eight stages (the consumers
+  // work on two at a time)
+  stages = static_cast<int>(std::max<size_t>(2, std::min<size_t>(8, (96 * 1024) / stage_bytes)));
+  return stages * stage_bytes + sizeof(float) * (((cols + 255) & ~255) + cols) + 16 * stages;
+}
+
+int power_occupancy(int cols, bool f32) {
+  int stages = 0;
+  const size_t smem = power_smem_bytes(cols, f32, stages);
+  switch ((cols + 255) / 256) {
+#define MUON_POWER_OCC(NVV) \
+  case NVV:                 \
+    return f32 ? power_blocks_per_sm<true, NVV>(smem) : power_blocks_per_sm<false, NVV>(smem);
+    MUON_POWER_OCC(1)
+    MUON_POWER_OCC(2)
+    MUON_POWER_OCC(3)
+    MUON_POWER_OCC(4)
+    MUON_POWER_OCC(5)
+    MUON_POWER_OCC(6)
+    MUON_POWER_OCC(7)
+    MUON_POWER_OCC(8)
+#undef MUON_POWER_OCC
+  }
+  return 0;
+}
+
+}  // namespace
+
+int power_pass_blocks(int rows, int cols, int batch, bool f32, int sm_count) {
+  // as many blocks as fit on the GPU at once (all of them resident, for the cooperative launch),
+  // at most 64 per matrix and one stage of rows each
+  const int per_sm = std::max(1, power_occupancy(cols, f32));
+  const int want = std::max(1, std::min(kPowerMaxBlocks, per_sm * sm_count / batch));
+  const int rpb = ((rows + want - 1) / want + kPowerWarps - 1) / kPowerWarps * kPowerWarps;
+  return (rows + rpb - 1) / rpb;
+}
+
+cudaError_t launch_power_iteration_stream(GemvParams& p, int batch, bool f32, int nblk, int iters,
+                                          float* tsq_partial, unsigned* counters, float* sigma, int* status,
+                                          int sm_count, cudaStream_t s) {
+  const int nv = (p.cols + 255) / 256;
+  if (p.cols % 8 != 0 || nv < 1 || nv > 8 || iters < 1 || nblk < 1 || nblk > kPowerMaxBlocks)
+    return cudaErrorInvalidValue;
+  const int rpb = ((p.rows + nblk - 1) / nblk + kPowerWarps - 1) / kPowerWarps * kPowerWarps;
+  if ((p.rows + rpb - 1) / rpb != nblk) return cudaErrorInvalidValue;
+  int stages = 0;
+  const size_t smem = power_smem_bytes(p.cols, f32, stages);
+  // all iterations in one cooperative launch when every block fits on the GPU at once
+  const bool together = iters > 1 && static_cast<long long>(nblk) * batch <=
+                                         static_cast<long long>(power_occupancy(p.cols, f32)) * sm_count;
+  cudaError_t e = cudaMemsetAsync(counters, 0, 2 * sizeof(unsigned) * batch, s);
+  if (e != cudaSuccess) return e;
+  PowerArgs a;
+  a.rows_per_block = rpb;
+  a.stages = stages;
+  a.nblk = nblk;
+  a.iters = iters;
+  a.part[0] = p.partial;
+  a.part[1] = p.partial + static_cast<long long>(batch) * nblk * p.cols;
+  a.tsq_partial = tsq_partial;
+  a.sync = counters;
+  a.done = counters + batch;
+  a.sigma = sigma;
+  a.status = status;
+  const dim3 grid(nblk, batch);
+  for (int it = 0; it < iters; it = a.it1) {
+    a.it0 = it;
+    a.it1 = together ? iters : it + 1;
     switch (nv) {
+#define MUON_POWER_CASE(NVV)                                                                               \
+  case NVV:                                                                                               \
+    e = f32 ? power_launch<true, NVV>(p, a, grid, smem, together, s)                                      \
+            : power_launch<false, NVV>(p, a, grid, smem, together, s);                                    \
+    break;
       MUON_POWER_CASE(1)
       MUON_POWER_CASE(2)
       MUON_POWER_CASE(3)
@@ -566,17 +846,11 @@ cudaError_t launch_power_iteration_fused(GemvParams& p, int batch, bool f32, flo
       MUON_POWER_CASE(6)
       MUON_POWER_CASE(7)
       MUON_POWER_CASE(8)
-    }
 #undef MUON_POWER_CASE
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    power_reduce_kernel<<<dim3(zblk, batch), kThreads, 0, s>>>(p, nblk, zsq_partial);
-    e = cudaGetLastError();
+    }
     if (e != cudaSuccess) return e;
   }
-  const int eblk = (std::max(p.rows, p.cols) + kThreads - 1) / kThreads;
-  power_scale_kernel<<<dim3(eblk, batch), kThreads, 0, s>>>(p, nblk, tsq_partial, zblk, zsq_partial, sigma);
-  return cudaGetLastError();
+  return cudaSuccess;
 }
 
 cudaError_t launch_normalize(float* const* vecs, int batch, int n, float* norm, cudaStream_t s) {

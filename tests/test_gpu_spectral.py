@@ -9,8 +9,11 @@ from tests.gpu_common import BF16_TOL, F32_TOL, rel_f, to_device, to_numpy
 pytestmark = pytest.mark.gpu
 
 # wide, tall, ragged (scalar paths: cols % 8 != 0), one past the 48 KB shared-memory default, and
-# the single-pass kernel at 6 and 8 vectors per lane (the out_proj width and its 2048 limit)
-SHAPES = [(96, 200, 3), (200, 96, 2), (77, 45, 2), (45, 77, 1), (64, 13000, 1), (768, 1536, 2), (300, 2048, 2)]
+# the streaming one-pass kernel at 6 and 8 vectors per lane (the out_proj width and its 2048
+# limit), with a last stage of fewer than eight rows, at its 64-block cap (one matrix of 4000
+# rows) and over the full out_proj batch (twelve blocks per matrix)
+SHAPES = [(96, 200, 3), (200, 96, 2), (77, 45, 2), (45, 77, 1), (64, 13000, 1), (768, 1536, 2), (300, 2048, 2),
+          (77, 48, 2), (4000, 512, 1), (768, 1536, 24)]
 
 
 def _spiked(rows, cols, batch, seed, dtype):
@@ -46,6 +49,26 @@ def test_power_iteration_matches_oracle(rows, cols, batch, dtype):
         assert abs(sigma[l] - rs) <= 1e-5 * rs
         assert rel_f(u[l], ru) <= 1e-4
         assert rel_f(v[l], rv) <= 1e-4
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_power_iteration_in_two_calls_continues_from_v(dtype):
+    """One iteration, then two calls of three: each call leaves v normalised and its per-matrix
+    block counters at zero, so 3 + 3 iterations are the oracle's 6 from the same start."""
+    from spectral_optimizer_state_b200 import Muon
+    rows, cols, batch = 200, 256, 3
+    Ws = _spiked(rows, cols, batch, 74, dtype)
+    v0s = [rng_for(75, l).standard_normal(cols).astype(np.float32) for l in range(batch)]
+    with Muon() as muon:
+        u1, v1, s1 = _power(muon, Ws, v0s, 1, dtype)
+        _, vh, _ = _power(muon, Ws, v0s, 3, dtype)
+        u6, v6, s6 = _power(muon, Ws, vh, 3, dtype)
+    for l in range(batch):
+        W = Ws[l].astype(np.float64)
+        ru, rv, rs = oracle.power_iteration(W, v0s[l].astype(np.float64), 1)
+        assert abs(s1[l] - rs) <= 1e-5 * rs and rel_f(u1[l], ru) <= 1e-4 and rel_f(v1[l], rv) <= 1e-4
+        ru, rv, rs = oracle.power_iteration(W, v0s[l].astype(np.float64), 6)
+        assert abs(s6[l] - rs) <= 1e-5 * rs and rel_f(u6[l], ru) <= 1e-4 and rel_f(v6[l], rv) <= 1e-4
 
 
 def test_power_iteration_reaches_the_svd_on_full_size_in_proj():
