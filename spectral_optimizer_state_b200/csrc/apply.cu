@@ -91,6 +91,15 @@ __device__ __forceinline__ void store8_w(void* dst, const float (&v)[8], const f
   }
 }
 
+// 16 bytes global -> this thread's shared memory, asynchronously (no registers held).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 template <bool F32>
 __device__ __forceinline__ void rmw1(void* dst, long long e, float v, bool apply, float decay, float lrs) {
   if (F32) {
@@ -199,10 +208,13 @@ __device__ __forceinline__ void wide_body(const ApplyParams& p, const ApplyGroup
   }
 }
 
-// Tall W (rows > cols): W(r, c) with O(c, r), through a 64 x 64 tile.
+// Tall W (rows > cols): W(r, c) with O(c, r), through a 64 x 64 tile.  Each thread's share of
+// the tile's W is copied into shared memory (cp.async) while O is read and transposed, so the two
+// reads' latencies overlap; the thread reads back only what it copied itself.
 template <bool F32, bool CAP>
 __device__ __forceinline__ void tall_body(const ApplyParams& p, const ApplyGroup& q, int l, int b) {
   __shared__ float tile[64][65];
+  __shared__ __align__(16) uint8_t wtile[64][64 * (F32 ? 4 : 2)];
   void* w = p.w[q.mat0 + l];
   const uint16_t* o = q.o + static_cast<long long>(l) * q.o_mat;
   const int R = q.rows, C = q.cols;
@@ -213,6 +225,18 @@ __device__ __forceinline__ void tall_body(const ApplyParams& p, const ApplyGroup
   const int cc = (threadIdx.x & 7) * 8;  // 0..56
   for (int tt = b; tt < ntiles; tt += q.nblk) {
     const int r0 = (tt / tiles_c) * 64, c0 = (tt % tiles_c) * 64;
+    const bool wvec = q.vec && c0 + cc < C;
+    if (wvec && p.apply) {
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        const int r = r0 + rr + 32 * pass;
+        if (r < R) {
+          const char* src = static_cast<const char*>(w) + (static_cast<long long>(r) * C + c0 + cc) * (F32 ? 4 : 2);
+#pragma unroll
+          for (int k = 0; k < (F32 ? 2 : 1); ++k) cp_async16(&wtile[rr + 32 * pass][cc * (F32 ? 4 : 2) + 16 * k], src + 16 * k);
+        }
+      }
+    }
     // O rows c (= W columns), 8 consecutive W rows r per thread: O(c, r..r+7)
     float ov[2][8];
 #pragma unroll
@@ -227,12 +251,12 @@ __device__ __forceinline__ void tall_body(const ApplyParams& p, const ApplyGroup
         for (int t = 0; t < 8; ++t) ov[pass][t] = 0.f;
       }
     }
-    const bool wvec = q.vec && c0 + cc < C;
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
 #pragma unroll
       for (int t = 0; t < 8; ++t) tile[cc + t][rr + 32 * pass] = ov[pass][t];
     }
+    if (wvec && p.apply) cp_async_wait_all();
     __syncthreads();
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
@@ -252,7 +276,7 @@ __device__ __forceinline__ void tall_body(const ApplyParams& p, const ApplyGroup
         if (wvec) {
           char* dst = static_cast<char*>(w) + (static_cast<long long>(r) * C + c) * (F32 ? 4 : 2);
           float cw[8];
-          load8_w<F32>(dst, p.apply, cw);
+          load8_w<F32>(&wtile[rl][cc * (F32 ? 4 : 2)], p.apply, cw);
           store8_w<F32>(dst, v, cw, p.apply, p.decay, q.lrs);
         } else {
 #pragma unroll
