@@ -20,6 +20,7 @@
 
 #include "device_utils.cuh"
 #include "internal.h"
+#include "rowpos.cuh"
 
 namespace muon {
 
@@ -123,15 +124,17 @@ __device__ __forceinline__ void wide_body(const ApplyParams& p, const ApplyGroup
   const int C = q.cols;
   const bool cap = CAP && q.alpha != nullptr;
   if (q.vec) {
-    const long long per_row = C / 8;
+    const int per_row = C / 8;
     const long long total = static_cast<long long>(q.rows) * per_row;
     const long long chunk = (total + q.nblk - 1) / q.nblk;
     const long long beg = chunk * b;
     const long long end = min(total, beg + chunk);
+    const RowStep one = rowstep_of(kThreads, per_row), two_steps = rowstep_of(2 * kThreads, per_row);
     if (F32 || CAP) {
-      for (long long v = beg + threadIdx.x; v < end; v += kThreads) {
-        const long long i = v / per_row;
-        const int j = static_cast<int>(v - i * per_row) * 8;
+      RowPos pos = rowpos_at(beg + threadIdx.x, per_row);
+      for (long long v = beg + threadIdx.x; v < end; v += kThreads, pos = rowpos_add(pos, one, per_row)) {
+        const long long i = pos.i;
+        const int j = pos.j * 8;
         char* dst = static_cast<char*>(w) + (i * C + j) * (F32 ? 4 : 2);
         float ov[8], cw[8];
         load8_planes(o + i * q.pitch + j, q.o_plane, p.planes, ov);
@@ -144,11 +147,13 @@ __device__ __forceinline__ void wide_body(const ApplyParams& p, const ApplyGroup
         store8_w<F32>(dst, ov, cw, p.apply, p.decay, q.lrs);
       }
     } else {
-      for (long long v0 = beg + threadIdx.x; v0 < end; v0 += 2 * kThreads) {
+      RowPos pa = rowpos_at(beg + threadIdx.x, per_row);
+      for (long long v0 = beg + threadIdx.x; v0 < end; v0 += 2 * kThreads, pa = rowpos_add(pa, two_steps, per_row)) {
         const long long v1 = v0 + kThreads;
         const bool two = v1 < end;
-        const long long i0 = v0 / per_row, i1 = v1 / per_row;
-        const int j0 = static_cast<int>(v0 - i0 * per_row) * 8, j1 = static_cast<int>(v1 - i1 * per_row) * 8;
+        const RowPos pb = rowpos_add(pa, one, per_row);
+        const long long i0 = pa.i, i1 = pb.i;
+        const int j0 = pa.j * 8, j1 = pb.j * 8;
         char* d0 = static_cast<char*>(w) + (i0 * C + j0) * (F32 ? 4 : 2);
         char* d1 = static_cast<char*>(w) + (i1 * C + j1) * (F32 ? 4 : 2);
         // both steps' loads as packed 16-byte vectors before either is unpacked

@@ -23,6 +23,7 @@
 
 #include "device_utils.cuh"
 #include "internal.h"
+#include "rowpos.cuh"
 
 namespace muon {
 
@@ -178,16 +179,19 @@ __device__ __forceinline__ void wide_body(const MomentumParams& p, const Momentu
   const int C = q.cols;
   float ss = 0.f;
   if (q.vec) {
-    const long long per_row = C / 8;
+    const int per_row = C / 8;
     const long long total = static_cast<long long>(q.rows) * per_row;
     const long long chunk = (total + q.nblk - 1) / q.nblk;
     const long long beg = chunk * b;
     const long long end = min(total, beg + chunk);
-    for (long long v0 = beg + threadIdx.x; v0 < end; v0 += 2 * kThreads) {
+    const RowStep one = rowstep_of(kThreads, per_row), two_steps = rowstep_of(2 * kThreads, per_row);
+    RowPos pa = rowpos_at(beg + threadIdx.x, per_row);
+    for (long long v0 = beg + threadIdx.x; v0 < end; v0 += 2 * kThreads, pa = rowpos_add(pa, two_steps, per_row)) {
       const long long v1 = v0 + kThreads;
       const bool two = v1 < end;
-      const long long i0 = v0 / per_row, i1 = v1 / per_row;
-      const int j0 = static_cast<int>(v0 - i0 * per_row) * 8, j1 = static_cast<int>(v1 - i1 * per_row) * 8;
+      const RowPos pb = rowpos_add(pa, one, per_row);
+      const long long i0 = pa.i, i1 = pb.i;
+      const int j0 = pa.j * 8, j1 = pb.j * 8;
       const long long e0 = i0 * C + j0, e1 = i1 * C + j1;
       float ga[8], gb[8], ma[8], mb[8], ua[8], ub[8];
       load8<TG>(g + e0, ga);
