@@ -102,11 +102,16 @@ struct CapParams {
 // 2 x [batch][nblk][cols] (two iterations' partials), tsq_partial [batch][nblk] and
 // counters [2 * batch] scratch (zeroed here).  nblk from power_pass_blocks; cols % 8 == 0,
 // 16-byte aligned W, cols <= power_pass_max_cols().  Wait timeouts set `status`.
+// With `shift` ([batch] sigma_max, device) the passes run the shifted iteration for the smallest
+// singular value of a tall W instead (iters = shifted steps + 1; p.x = y, read then overwritten;
+// p.y scratch of `rows` floats; sigma receives |W y|); it needs every pass in one launch
+// (power_pass_together, or iters == 1).
 int power_pass_max_cols();
 int power_pass_blocks(int rows, int cols, int batch, bool f32, int sm_count);
+bool power_pass_together(int cols, bool f32, int nblk, int batch, int sm_count);
 cudaError_t launch_power_iteration_stream(GemvParams& p, int batch, bool f32, int nblk, int iters,
                                           float* tsq_partial, unsigned* counters, float* sigma, int* status,
-                                          int sm_count, cudaStream_t s);
+                                          int sm_count, cudaStream_t s, const float* shift = nullptr);
 cudaError_t launch_gemv_rows(const GemvParams& p, int batch, bool f32, cudaStream_t s);
 cudaError_t launch_gemv_cols(const GemvParams& p, int batch, bool f32, cudaStream_t s);
 cudaError_t launch_normalize(float* const* vecs_dev, int batch, int n, float* norm, cudaStream_t s);

@@ -1114,6 +1114,40 @@ muon_status muon_min_singular(muon_ctx* c, const void* const* W, float* const* y
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool tall = rows > cols;
   const int m = tall ? cols : rows, n = tall ? rows : cols;  // wide view X is m x n
+  const bool f32 = dtype == MUON_F32;
+  if (tall) {
+    // X X^T y = W^T W y: one streaming pass over W per shifted step (power_stream_kernel with a
+    // shift), all passes in one launch when its blocks fit on the GPU at once
+    bool stream_ok = cols % 8 == 0 && cols <= power_pass_max_cols();
+    for (int l = 0; l < batch && stream_ok; ++l)
+      if (reinterpret_cast<uintptr_t>(W[l]) % 16) stream_ok = false;
+    const int nblk = stream_ok ? power_pass_blocks(rows, cols, batch, f32, c->sm_count) : 0;
+    if (stream_ok && (iters == 0 || power_pass_together(cols, f32, nblk, batch, c->sm_count))) {
+      const size_t part_bytes = align_up(2 * sizeof(float) * batch * nblk * cols, 256);
+      const size_t tsq_bytes = align_up(sizeof(float) * batch * nblk, 256);
+      const size_t cnt_bytes = align_up(2 * sizeof(unsigned) * batch, 256);
+      const size_t t_bytes = align_up(sizeof(float) * rows, 256);
+      muon_status st = ensure_aux(c, part_bytes + tsq_bytes + cnt_bytes + batch * t_bytes);
+      if (st != MUON_OK) return st;
+      char* base = static_cast<char*>(c->d_aux);
+      GemvParams sp;
+      std::memset(static_cast<void*>(&sp), 0, sizeof(sp));
+      sp.rows = rows;
+      sp.cols = cols;
+      sp.partial = reinterpret_cast<float*>(base);
+      float* tsq = reinterpret_cast<float*>(base + part_bytes);
+      unsigned* counters = reinterpret_cast<unsigned*>(base + part_bytes + tsq_bytes);
+      for (int l = 0; l < batch; ++l) {
+        sp.w[l] = W[l];
+        sp.x[l] = y[l];
+        sp.y[l] = reinterpret_cast<float*>(base + part_bytes + tsq_bytes + cnt_bytes + l * t_bytes);
+      }
+      MUON_CUDA(launch_power_iteration_stream(sp, batch, f32, nblk, iters + 1, tsq, counters, sigma_min,
+                                              c->d_status, c->sm_count, s, sigma_max),
+                "shifted iteration");
+      return MUON_OK;
+    }
+  }
   GemvParams gp;
   std::memset(static_cast<void*>(&gp), 0, sizeof(gp));
   gp.rows = rows;
@@ -1133,7 +1167,6 @@ muon_status muon_min_singular(muon_ctx* c, const void* const* W, float* const* y
     wv[l] = reinterpret_cast<float*>(base + part_bytes + l * w_bytes);
     zv[l] = reinterpret_cast<float*>(base + part_bytes + batch * w_bytes + l * z_bytes);
   }
-  const bool f32 = dtype == MUON_F32;
   // out <- X^T in (length n) and out <- X in (length m), X the wide view of W
   auto apply_xt = [&](float* const* in, float* const* out) {
     for (int l = 0; l < batch; ++l) {

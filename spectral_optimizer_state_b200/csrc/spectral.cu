@@ -340,6 +340,13 @@ __device__ __forceinline__ double sum_squares(const float (&z)[8], double* scrat
 // on its scale).  After the last iteration, the last block of a matrix to finish writes
 // v = z / |z|, u = t / |t| and sigma = |z| / |t| = |W^T u|.  A zero t leaves u, v at zero and
 // sigma 0.  Requires cols % 8 == 0, 16-byte aligned W and cols <= 256 * NV <= 2048.
+//
+// With `shift` set (the smallest singular value of a tall W, whose wide view is X = W^T, so
+// X X^T y = W^T W y = z), the same passes run the shifted iteration: pass 0 takes y = v / |v|,
+// pass k > 0 takes y <- (s y - z) / |s y - z| with s = shift[l]^2 and z from pass k-1 (y, the
+// previous pass's v, is still in every block's shared memory), and after the last pass the
+// last block writes y to v and sigma[l] = |X^T y| = |W y| = |t|.  All passes of such a call run
+// in one launch.
 constexpr int kPowerWarps = 8;                         // consumer warps: a stage holds a row for each
 constexpr int kPowerThreads = 32 * (kPowerWarps + 1);  // and one producer warp
 constexpr int kPowerMaxBlocks = 64;                    // block partials per matrix
@@ -349,6 +356,7 @@ constexpr uint64_t kPowerDrainNs = 200000000ull;
 struct PowerArgs {
   int rows_per_block, stages, nblk, iters;  // iters: of the whole call
   int it0, it1;                             // the iterations this launch runs
+  const float* shift;  // [batch] sigma_max for the shifted iteration, or null for the power iteration
   float* part[2];      // [batch][nblk][cols] each: z partials of even / odd iterations
   float* tsq_partial;  // [batch][nblk]: each block's sum of t_r^2 (last iteration written)
   unsigned* sync;      // [batch]: partial sets written in this call (blocks x iterations)
@@ -425,7 +433,7 @@ __global__ void __launch_bounds__(kPowerThreads, (NV <= 5 || (!F32 && NV <= 6)) 
     // ------------------------------------------------ consumers
     for (int it = a.it0; it < a.it1; ++it) {
       // v for this iteration
-      if (it == 0) {
+      if (it == 0 && a.shift == nullptr) {
         const float* x = p.x[l];
         for (int c = threadIdx.x; c < C; c += kConsumers) vs[vs_index(c)] = x[c];
       } else {
@@ -437,8 +445,27 @@ __global__ void __launch_bounds__(kPowerThreads, (NV <= 5 || (!F32 && NV <= 6)) 
           named_barrier_sync(1, kConsumers);
         }
         float zc[kPowerCols];
-        sum_partials(a.part[(it - 1) & 1] + static_cast<long long>(l) * a.nblk * C, a.nblk, C, threadIdx.x,
-                     kConsumers, zc);
+        if (it == 0) {
+          // the shifted iteration starts from the caller's vector, normalised
+          const float* x = p.x[l];
+#pragma unroll
+          for (int k = 0; k < kPowerCols; ++k) {
+            const int c = threadIdx.x + k * kConsumers;
+            zc[k] = c < C ? x[c] : 0.f;
+          }
+        } else {
+          sum_partials(a.part[(it - 1) & 1] + static_cast<long long>(l) * a.nblk * C, a.nblk, C, threadIdx.x,
+                       kConsumers, zc);
+          if (a.shift != nullptr) {
+            // s y - z, y the previous pass's v (each thread reads and rewrites only its columns)
+            const float s2 = a.shift[l] * a.shift[l];
+#pragma unroll
+            for (int k = 0; k < kPowerCols; ++k) {
+              const int c = threadIdx.x + k * kConsumers;
+              if (c < C) zc[k] = fmaf(s2, vs[vs_index(c)], -zc[k]);
+            }
+          }
+        }
         const double ss = sum_squares(zc, sq, kPowerWarps, [] { named_barrier_sync(1, kConsumers); });
         const float nz = static_cast<float>(sqrt(ss));
         const float inv = nz > 0.f ? 1.0f / nz : 0.f;
@@ -530,6 +557,16 @@ __global__ void __launch_bounds__(kPowerThreads, (NV <= 5 || (!F32 && NV <= 6)) 
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  if (a.shift != nullptr) {
+    // y is this block's v of the last pass (every block holds the same); sigma_min = |W y|
+    float* y = const_cast<float*>(p.x[l]);
+    for (int c = threadIdx.x; c < C; c += kPowerThreads) y[c] = vs[vs_index(c)];
+    if (warp == 0) {
+      const double tt = warp_sum_partials(a.tsq_partial + static_cast<long long>(l) * a.nblk, a.nblk, lane);
+      if (lane == 0) a.sigma[l] = static_cast<float>(sqrt(tt));
+    }
+    return;
+  }
   float zc[kPowerCols];
   sum_partials(a.part[(a.iters - 1) & 1] + static_cast<long long>(l) * a.nblk * C, a.nblk, C, threadIdx.x,
                kPowerThreads, zc);
@@ -801,9 +838,13 @@ int power_pass_blocks(int rows, int cols, int batch, bool f32, int sm_count) {
   return (rows + rpb - 1) / rpb;
 }
 
+bool power_pass_together(int cols, bool f32, int nblk, int batch, int sm_count) {
+  return static_cast<long long>(nblk) * batch <= static_cast<long long>(power_occupancy(cols, f32)) * sm_count;
+}
+
 cudaError_t launch_power_iteration_stream(GemvParams& p, int batch, bool f32, int nblk, int iters,
                                           float* tsq_partial, unsigned* counters, float* sigma, int* status,
-                                          int sm_count, cudaStream_t s) {
+                                          int sm_count, cudaStream_t s, const float* shift) {
   const int nv = (p.cols + 255) / 256;
   if (p.cols % 8 != 0 || nv < 1 || nv > 8 || iters < 1 || nblk < 1 || nblk > kPowerMaxBlocks)
     return cudaErrorInvalidValue;
@@ -812,8 +853,9 @@ cudaError_t launch_power_iteration_stream(GemvParams& p, int batch, bool f32, in
   int stages = 0;
   const size_t smem = power_smem_bytes(p.cols, f32, stages);
   // all iterations in one cooperative launch when every block fits on the GPU at once
-  const bool together = iters > 1 && static_cast<long long>(nblk) * batch <=
-                                         static_cast<long long>(power_occupancy(p.cols, f32)) * sm_count;
+  const bool together = iters > 1 && power_pass_together(p.cols, f32, nblk, batch, sm_count);
+  // the shifted iteration keeps y in shared memory from pass to pass: one launch for all passes
+  if (shift != nullptr && iters > 1 && !together) return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(counters, 0, 2 * sizeof(unsigned) * batch, s);
   if (e != cudaSuccess) return e;
   PowerArgs a;
@@ -821,6 +863,7 @@ cudaError_t launch_power_iteration_stream(GemvParams& p, int batch, bool f32, in
   a.stages = stages;
   a.nblk = nblk;
   a.iters = iters;
+  a.shift = shift;
   a.part[0] = p.partial;
   a.part[1] = p.partial + static_cast<long long>(batch) * nblk * p.cols;
   a.tsq_partial = tsq_partial;

@@ -71,6 +71,23 @@ def test_power_iteration_in_two_calls_continues_from_v(dtype):
         assert abs(s6[l] - rs) <= 1e-5 * rs and rel_f(u6[l], ru) <= 1e-4 and rel_f(v6[l], rv) <= 1e-4
 
 
+def test_power_iteration_one_launch_per_iteration_when_blocks_do_not_fit():
+    """fp32 rows of 2048 columns leave one block per SM, so 200 matrices cannot all be resident
+    at once: the iterations then run as one launch each (no block waits on another) and must
+    give the same results as the oracle."""
+    from spectral_optimizer_state_b200 import Muon
+    rows, cols, batch = 16, 2048, 200
+    Ws = _spiked(rows, cols, batch, 76, "f32")
+    v0s = [rng_for(77, l).standard_normal(cols).astype(np.float32) for l in range(batch)]
+    with Muon() as muon:
+        u, v, sigma = _power(muon, Ws, v0s, 3, "f32")
+    for l in (0, 99, 199):
+        ru, rv, rs = oracle.power_iteration(Ws[l].astype(np.float64), v0s[l].astype(np.float64), 3)
+        assert abs(sigma[l] - rs) <= 1e-5 * rs
+        assert rel_f(u[l], ru) <= 1e-4
+        assert rel_f(v[l], rv) <= 1e-4
+
+
 def test_power_iteration_reaches_the_svd_on_full_size_in_proj():
     """in_proj shape of the 130M model: 24 matrices with a planted top direction, 30 iterations."""
     from spectral_optimizer_state_b200 import Muon
@@ -205,6 +222,23 @@ def test_min_singular_matches_oracle(rows, cols, batch, dtype, iters):
         assert abs(smin[l] - rs) <= 1e-4 * rs
         assert rel_f(y[l], ry) <= 1e-4
         assert smin[l] >= np.linalg.svd(Ws[l].astype(np.float64), compute_uv=False)[-1] * (1 - 1e-4)
+
+
+def test_min_singular_full_size_in_proj_streams_in_one_launch():
+    """The in_proj group of the 130M model (24 tall 3352 x 768 bf16 matrices, the one-pass
+    streaming path: X X^T y = W^T W y) against the oracle's shifted iteration."""
+    from spectral_optimizer_state_b200 import Muon
+    rows, cols = MAMBA2_130M_IN_PROJ
+    Ws = [round_bf16(weights(rng_for(78, l), rows, cols)) for l in range(24)]
+    y0s = [rng_for(79, l).standard_normal(cols).astype(np.float32) for l in range(24)]
+    smax = [float(np.float32(np.linalg.svd(Ws[l].astype(np.float64), compute_uv=False)[0])) if l in (0, 23)
+            else 1.0 for l in range(24)]
+    with Muon() as muon:
+        y, smin = _min_singular(muon, Ws, y0s, smax, 16, "bf16")
+    for l in (0, 23):
+        ry, rs = oracle.min_singular_shifted(Ws[l].astype(np.float64), y0s[l].astype(np.float64), smax[l], 16)
+        assert abs(smin[l] - rs) <= 1e-4 * rs
+        assert rel_f(y[l], ry) <= 1e-4
 
 
 def test_min_singular_of_semi_orthogonal_is_one():
