@@ -228,8 +228,11 @@ __device__ __forceinline__ void tall_body(const ApplyParams& p, const ApplyGroup
   const int ntiles = ((R + 63) / 64) * tiles_c;
   const int rr = threadIdx.x >> 3;       // 0..31
   const int cc = (threadIdx.x & 7) * 8;  // 0..56
-  for (int tt = b; tt < ntiles; tt += q.nblk) {
-    const int r0 = (tt / tiles_c) * 64, c0 = (tt % tiles_c) * 64;
+  // tile tt = (row tile, column tile) walked in strides of nblk without a division per tile
+  const RowStep tstep = rowstep_of(q.nblk, tiles_c);
+  RowPos tp = rowpos_at(b, tiles_c);
+  for (int tt = b; tt < ntiles; tt += q.nblk, tp = rowpos_add(tp, tstep, tiles_c)) {
+    const int r0 = tp.i * 64, c0 = tp.j * 64;
     const bool wvec = q.vec && c0 + cc < C;
     if (wvec && p.apply) {
 #pragma unroll
@@ -242,24 +245,42 @@ __device__ __forceinline__ void tall_body(const ApplyParams& p, const ApplyGroup
         }
       }
     }
-    // O rows c (= W columns), 8 consecutive W rows r per thread: O(c, r..r+7)
-    float ov[2][8];
+    // O rows c (= W columns), 8 consecutive W rows r per thread: O(c, r..r+7); the wide pitch is
+    // >= round_up(R, 8) and r % 8 == 0, so the 8-wide read stays in the row.  A bf16 W comes with
+    // a one-plane iterate: both passes' 16-byte vectors are read before either is unpacked.
+    if (!F32) {
+      uint4 oq[2];
 #pragma unroll
-    for (int pass = 0; pass < 2; ++pass) {
-      const int c = c0 + rr + 32 * pass;
-      const int r = r0 + cc;
-      if (c < C && r < R) {
-        // the wide pitch is >= round_up(R, 8) and r % 8 == 0: the 8-wide read stays in the row
-        load8_planes(o + static_cast<long long>(c) * q.pitch + r, q.o_plane, p.planes, ov[pass]);
-      } else {
-#pragma unroll
-        for (int t = 0; t < 8; ++t) ov[pass][t] = 0.f;
+      for (int pass = 0; pass < 2; ++pass) {
+        const int c = c0 + rr + 32 * pass;
+        const int r = r0 + cc;
+        oq[pass] = c < C && r < R ? __ldcs(reinterpret_cast<const uint4*>(o + static_cast<long long>(c) * q.pitch + r))
+                                  : make_uint4(0u, 0u, 0u, 0u);
       }
-    }
 #pragma unroll
-    for (int pass = 0; pass < 2; ++pass) {
+      for (int pass = 0; pass < 2; ++pass) {
+        const uint32_t u[4] = {oq[pass].x, oq[pass].y, oq[pass].z, oq[pass].w};
 #pragma unroll
-      for (int t = 0; t < 8; ++t) tile[cc + t][rr + 32 * pass] = ov[pass][t];
+        for (int k = 0; k < 4; ++k) {
+          tile[cc + 2 * k][rr + 32 * pass] = __uint_as_float(u[k] << 16);
+          tile[cc + 2 * k + 1][rr + 32 * pass] = __uint_as_float(u[k] & 0xFFFF0000u);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        const int c = c0 + rr + 32 * pass;
+        const int r = r0 + cc;
+        float ov[8];
+        if (c < C && r < R) {
+          load8_planes(o + static_cast<long long>(c) * q.pitch + r, q.o_plane, p.planes, ov);
+        } else {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) ov[t] = 0.f;
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) tile[cc + t][rr + 32 * pass] = ov[t];
+      }
     }
     if (wvec && p.apply) cp_async_wait_all();
     __syncthreads();
