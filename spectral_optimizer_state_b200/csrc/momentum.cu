@@ -243,8 +243,11 @@ __device__ __forceinline__ void tall_body(const MomentumParams& p, const Momentu
   const int rr = threadIdx.x >> 3;        // 0..31
   const int cc = (threadIdx.x & 7) * 8;   // 0..56
   float ss = 0.f;
-  for (int tt = b; tt < ntiles; tt += q.nblk) {
-    const int r0 = (tt / tiles_c) * 64, c0 = (tt % tiles_c) * 64;
+  // tile tt = (row tile, column tile) walked in strides of nblk without a division per tile
+  const RowStep tstep = rowstep_of(q.nblk, tiles_c);
+  RowPos tp = rowpos_at(b, tiles_c);
+  for (int tt = b; tt < ntiles; tt += q.nblk, tp = rowpos_add(tp, tstep, tiles_c)) {
+    const int r0 = tp.i * 64, c0 = tp.j * 64;
     float u[2][8];
     if (q.vec) {
       // both passes' loads first: two rows of 8 in flight per thread
