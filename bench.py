@@ -374,12 +374,13 @@ def measure_spectral(mu, Ws, Gs, Ms, groups, stream, peaks, pi_iters=8, min_iter
     assert st == 0, f"device status {st}"
     kappa = [float((vecs[g][3] / vecs[g][4]).max()) for g in range(len(groups))]
     pi_gbs = pi_iters * w_bytes / (pi_ms / 1e3) / 1e9
-    min_gbs = (2 * min_iters + 1) * w_bytes / (min_ms / 1e3) / 1e9
+    min_gbs = (min_iters + 1) * w_bytes / (min_ms / 1e3) / 1e9
     hbm = peaks["hbm_gbs"]
     return {
         "bound": "hbm",
         "note": ("passes over W; algorithmic bytes: one pass over W per power iteration (u and W^T u "
-                 "come from the same pass, since W^T u = W^T (W v) / |W v|), two per shifted iteration + 1; "
+                 "come from the same pass, since W^T u = W^T (W v) / |W v|), one per shifted iteration + 1 "
+                 "(X X^T y formed in one pass: rows of a tall W, column slabs of a wide one); "
                  "one group's W (<= 124 MB at 130M) can stay in the 126 MB L2 between passes"),
         "power_iteration": {"iters": pi_iters, "ms": pi_ms, "achieved_gbs": pi_gbs, "frac": pi_gbs / hbm},
         "min_singular": {"iters": min_iters, "ms": min_ms, "achieved_gbs": min_gbs, "frac": min_gbs / hbm,

@@ -112,6 +112,14 @@ bool power_pass_together(int cols, bool f32, int nblk, int batch, int sm_count);
 cudaError_t launch_power_iteration_stream(GemvParams& p, int batch, bool f32, int nblk, int iters,
                                           float* tsq_partial, unsigned* counters, float* sigma, int* status,
                                           int sm_count, cudaStream_t s, const float* shift = nullptr);
+// Smallest singular value of a wide W (rows <= cols, X = W) by `iters` shifted steps, one pass
+// over W each plus a last one (colslab_kernel, one cooperative launch): slabs of S columns.
+// colslab_width gives S (0: this path does not apply: rows > 4096, cols not a multiple of 64,
+// or the grid does not fit on the GPU at once).  p.x = y (read, then overwritten), p.partial
+// 2 x [batch][cols / S][rows], dsq [batch][cols / S], counters [2 * batch] scratch.
+int colslab_width(int rows, int cols, int batch, bool f32, int sm_count);
+cudaError_t launch_min_singular_slabs(GemvParams& p, int batch, bool f32, int S, int iters, const float* shift,
+                                      float* dsq, unsigned* counters, float* sigma, int* status, cudaStream_t s);
 cudaError_t launch_gemv_rows(const GemvParams& p, int batch, bool f32, cudaStream_t s);
 cudaError_t launch_gemv_cols(const GemvParams& p, int batch, bool f32, cudaStream_t s);
 cudaError_t launch_normalize(float* const* vecs_dev, int batch, int n, float* norm, cudaStream_t s);

@@ -1148,6 +1148,36 @@ muon_status muon_min_singular(muon_ctx* c, const void* const* W, float* const* y
       return MUON_OK;
     }
   }
+  if (!tall) {
+    // X = W: one pass over W per shifted step, column slabs (colslab_kernel), one launch
+    bool aligned = true;
+    for (int l = 0; l < batch && aligned; ++l)
+      if (reinterpret_cast<uintptr_t>(W[l]) % 16) aligned = false;
+    const int S = aligned ? colslab_width(rows, cols, batch, f32, c->sm_count) : 0;
+    if (S > 0) {
+      const int nslab = cols / S;
+      const size_t part_bytes = align_up(2 * sizeof(float) * batch * nslab * rows, 256);
+      const size_t dsq_bytes = align_up(sizeof(float) * batch * nslab, 256);
+      muon_status st = ensure_aux(c, part_bytes + dsq_bytes + 2 * sizeof(unsigned) * batch);
+      if (st != MUON_OK) return st;
+      char* base = static_cast<char*>(c->d_aux);
+      GemvParams sp;
+      std::memset(static_cast<void*>(&sp), 0, sizeof(sp));
+      sp.rows = rows;
+      sp.cols = cols;
+      sp.partial = reinterpret_cast<float*>(base);
+      for (int l = 0; l < batch; ++l) {
+        sp.w[l] = W[l];
+        sp.x[l] = y[l];
+      }
+      MUON_CUDA(launch_min_singular_slabs(sp, batch, f32, S, iters, sigma_max,
+                                          reinterpret_cast<float*>(base + part_bytes),
+                                          reinterpret_cast<unsigned*>(base + part_bytes + dsq_bytes), sigma_min,
+                                          c->d_status, s),
+                "shifted iteration (column slabs)");
+      return MUON_OK;
+    }
+  }
   GemvParams gp;
   std::memset(static_cast<void*>(&gp), 0, sizeof(gp));
   gp.rows = rows;

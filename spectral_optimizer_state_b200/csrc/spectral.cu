@@ -715,6 +715,207 @@ __global__ void cap_alpha_reduce_kernel(const double* partial, int nblk, float* 
   alpha[blockIdx.x] = static_cast<float>(s);
 }
 
+// ------------------------------------------------------------------ shifted iteration, wide W
+// For a wide W (rows <= cols) the wide view is X = W, so X X^T y = W (W^T y): a pass needs
+// W^T y before W (W^T y).  A block owns a slab of S columns of one matrix (every row): phase 1
+// streams the slab from HBM and forms d = W[:, slab]^T y (S values, lanes across the columns,
+// a fixed xor tree over the rows a warp covers, then a warp-ordered sum) and |d|^2; phase 2
+// reads the slab again (just read, so from L2) with a thread per row, adding W[r, slab] d into
+// this slab's partial of z = W d.  The next pass's blocks sum the partials in slab order and take
+// y <- (s y - z) / |s y - z| (s = shift[l]^2), once a per-matrix counter says every slab of the
+// matrix has written them; the blocks wait on one another, so all passes run in one
+// cooperative launch.  Pass 0 takes y = v / |v| from the caller's v.  The last pass skips
+// phase 2, and the last block of a matrix to finish writes y to v and
+// sigma[l] = |X^T y| = sqrt(sum over slabs of |d|^2).  Deterministic: every sum has a fixed order.
+constexpr int kSlabRowsMax = 4096;  // y is kept in shared memory
+constexpr int kSlabUnroll = 8;      // rows in flight per lane in phase 1
+
+struct SlabArgs {
+  int nslab, passes;
+  const float* shift;  // [batch] sigma_max
+  float* part[2];      // [batch][nslab][rows]: z partials of even / odd passes
+  float* dsq;          // [batch][nslab]: |d|^2 of the last pass
+  unsigned* sync;      // [batch]: slabs of this call that have written their partials
+  unsigned* done;      // [batch]: slabs through the last pass
+  float* sigma;        // [batch]
+  int* status;
+};
+
+// Fixed-order sum of one value per thread over the whole block (every thread gets it).
+__device__ __forceinline__ double block_total(double v, double* scratch) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = v;
+  __syncthreads();
+  double t = 0.0;
+  for (int k = 0; k < kThreads / 32; ++k) t += scratch[k];
+  return t;
+}
+
+template <bool F32, int S>
+__global__ void __launch_bounds__(kThreads, 2) colslab_kernel(const __grid_constant__ GemvParams p, const SlabArgs a) {
+  constexpr int LPR = S / 8;            // lanes per row in phase 1 (8 columns each)
+  constexpr int RPW = 32 / LPR;         // rows a warp covers per load
+  constexpr int kWarps = kThreads / 32;
+  __shared__ float ys[kSlabRowsMax];
+  __shared__ float dred[kWarps][S];
+  __shared__ float ds[S];
+  __shared__ double scratch[kWarps];
+  __shared__ int s_last;
+  __shared__ volatile int abort_flag;
+  const int l = blockIdx.y, slab = blockIdx.x;
+  const int R = p.rows, C = p.cols;
+  const int c0 = slab * S;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rg = lane / LPR, k = lane % LPR;
+  const char* W = static_cast<const char*>(p.w[l]);
+  constexpr int ES = F32 ? 4 : 2;
+  if (threadIdx.x == 0) abort_flag = 0;
+  for (int pass = 0; pass < a.passes; ++pass) {
+    // y for this pass
+    {
+      double ss = 0.0;
+      if (pass == 0) {
+        for (int r = threadIdx.x; r < R; r += kThreads) {
+          const float v = p.x[l][r];
+          ys[r] = v;
+          ss += static_cast<double>(v) * v;
+        }
+      } else {
+        if (threadIdx.x == 0 && !abort_flag &&
+            !wait_counter_bounded(a.sync + l, static_cast<unsigned>(a.nslab * pass), &abort_flag, a.status))
+          abort_flag = 1;
+        __syncthreads();
+        const float* pp = a.part[(pass - 1) & 1] + static_cast<long long>(l) * a.nslab * R;
+        const float s2 = a.shift[l] * a.shift[l];
+        for (int r = threadIdx.x; r < R; r += kThreads) {
+          float z = 0.f;
+          for (int b = 0; b < a.nslab; ++b) z += __ldcg(pp + static_cast<long long>(b) * R + r);
+          const float v = fmaf(s2, ys[r], -z);
+          ys[r] = v;
+          ss += static_cast<double>(v) * v;
+        }
+      }
+      const double tot = block_total(ss, scratch);
+      const float nrm = static_cast<float>(sqrt(tot));
+      const float inv = nrm > 0.f ? 1.0f / nrm : 0.f;
+      for (int r = threadIdx.x; r < R; r += kThreads) ys[r] *= inv;
+      __syncthreads();
+    }
+    // phase 1: d = W[:, slab]^T y, rows in strides of (warps x RPW), kSlabUnroll loads in flight
+    float acc[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+    const int rstride = kWarps * RPW;
+    for (int r0 = warp * RPW + rg; r0 < R && !abort_flag; r0 += rstride * kSlabUnroll) {
+      uint4 raw[kSlabUnroll][F32 ? 2 : 1];
+#pragma unroll
+      for (int u = 0; u < kSlabUnroll; ++u) {
+        const int r = r0 + u * rstride;
+        if (r < R) {
+          const uint4* src = reinterpret_cast<const uint4*>(W + (static_cast<long long>(r) * C + c0 + 8 * k) * ES);
+#pragma unroll
+          for (int h = 0; h < (F32 ? 2 : 1); ++h) raw[u][h] = __ldcs(src + h);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kSlabUnroll; ++u) {
+        const int r = r0 + u * rstride;
+        if (r < R) {
+          const float yr = ys[r];
+          float x[8];
+          if (F32) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              x[4 * h] = __uint_as_float(raw[u][h].x);
+              x[4 * h + 1] = __uint_as_float(raw[u][h].y);
+              x[4 * h + 2] = __uint_as_float(raw[u][h].z);
+              x[4 * h + 3] = __uint_as_float(raw[u][h].w);
+            }
+          } else {
+            const uint32_t w4[4] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              x[2 * i] = __uint_as_float(w4[i] << 16);
+              x[2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
+            }
+          }
+#pragma unroll
+          for (int t = 0; t < 8; ++t) acc[t] = fmaf(x[t], yr, acc[t]);
+        }
+      }
+    }
+    // the rows this warp covered: xor tree over the row groups, then warps in order
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+      for (int t = 0; t < 8; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+    if (rg == 0)
+#pragma unroll
+      for (int t = 0; t < 8; ++t) dred[warp][8 * k + t] = acc[t];
+    __syncthreads();
+    double dd = 0.0;
+    for (int j = threadIdx.x; j < S; j += kThreads) {
+      float d = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) d += dred[w][j];
+      ds[j] = d;
+      dd += static_cast<double>(d) * d;
+    }
+    const double dtot = block_total(dd, scratch);  // also orders ds before phase 2
+    if (pass == a.passes - 1) {
+      if (threadIdx.x == 0) a.dsq[static_cast<long long>(l) * a.nslab + slab] = static_cast<float>(dtot);
+      break;
+    }
+    // phase 2: this slab's share of z = W d, a thread per row
+    float* part = a.part[pass & 1] + (static_cast<long long>(l) * a.nslab + slab) * R;
+    for (int r = threadIdx.x; r < R && !abort_flag; r += kThreads) {
+      const uint4* src = reinterpret_cast<const uint4*>(W + (static_cast<long long>(r) * C + c0) * ES);
+      float z = 0.f;
+#pragma unroll
+      for (int m = 0; m < S / 8; ++m) {
+        float x[8];
+        if (F32) {
+          const uint4 q0 = src[2 * m], q1 = src[2 * m + 1];
+          x[0] = __uint_as_float(q0.x); x[1] = __uint_as_float(q0.y); x[2] = __uint_as_float(q0.z);
+          x[3] = __uint_as_float(q0.w); x[4] = __uint_as_float(q1.x); x[5] = __uint_as_float(q1.y);
+          x[6] = __uint_as_float(q1.z); x[7] = __uint_as_float(q1.w);
+        } else {
+          const uint4 q0 = src[m];
+          const uint32_t w4[4] = {q0.x, q0.y, q0.z, q0.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(w4[i] << 16);
+            x[2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
+          }
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) z = fmaf(x[t], ds[8 * m + t], z);
+      }
+      part[r] = z;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) red_release_gpu_add(a.sync + l, 1u);
+  }
+  // after the last pass: the last slab of this matrix to get here writes y and sigma_min
+  __syncthreads();
+  if (abort_flag) return;
+  __threadfence();
+  if (threadIdx.x == 0) s_last = atomicAdd(a.done + l, 1u) == static_cast<unsigned>(a.nslab - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  float* y = const_cast<float*>(p.x[l]);
+  for (int r = threadIdx.x; r < R; r += kThreads) y[r] = ys[r];
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int b = 0; b < a.nslab; ++b) t += __ldcg(a.dsq + static_cast<long long>(l) * a.nslab + b);
+    a.sigma[l] = static_cast<float>(sqrt(t));
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_gemv_rows(const GemvParams& p, int batch, bool f32, cudaStream_t s) {
@@ -894,6 +1095,65 @@ cudaError_t launch_power_iteration_stream(GemvParams& p, int batch, bool f32, in
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+namespace {
+
+template <bool F32, int S>
+int slab_blocks_per_sm() {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, colslab_kernel<F32, S>, kThreads, 0) != cudaSuccess) return 0;
+  return n;
+}
+
+int slab_capacity(bool f32, int S, int sm_count) {
+  int per_sm = 0;
+  if (S == 64) per_sm = f32 ? slab_blocks_per_sm<true, 64>() : slab_blocks_per_sm<false, 64>();
+  if (S == 128) per_sm = f32 ? slab_blocks_per_sm<true, 128>() : slab_blocks_per_sm<false, 128>();
+  if (S == 256) per_sm = f32 ? slab_blocks_per_sm<true, 256>() : slab_blocks_per_sm<false, 256>();
+  return per_sm * sm_count;
+}
+
+}  // namespace
+
+int colslab_width(int rows, int cols, int batch, bool f32, int sm_count) {
+  if (rows > kSlabRowsMax || rows > cols) return 0;
+  // the narrowest slab whose grid still fits on the GPU at once (more blocks, shorter rows)
+  for (int S : {64, 128, 256}) {
+    if (cols % S != 0) continue;
+    const long long blocks = static_cast<long long>(cols / S) * batch;
+    if (cols / S <= 1024 && blocks <= slab_capacity(f32, S, sm_count)) return S;
+  }
+  return 0;
+}
+
+cudaError_t launch_min_singular_slabs(GemvParams& p, int batch, bool f32, int S, int iters, const float* shift,
+                                      float* dsq, unsigned* counters, float* sigma, int* status, cudaStream_t s) {
+  if (S != 64 && S != 128 && S != 256) return cudaErrorInvalidValue;
+  if (p.cols % S != 0 || p.rows > kSlabRowsMax || iters < 0) return cudaErrorInvalidValue;
+  SlabArgs a;
+  a.nslab = p.cols / S;
+  a.passes = iters + 1;
+  a.shift = shift;
+  a.part[0] = p.partial;
+  a.part[1] = p.partial + static_cast<long long>(batch) * a.nslab * p.rows;
+  a.dsq = dsq;
+  a.sync = counters;
+  a.done = counters + batch;
+  a.sigma = sigma;
+  a.status = status;
+  cudaError_t e = cudaMemsetAsync(counters, 0, 2 * sizeof(unsigned) * batch, s);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(a.nslab, batch);
+  void* args[] = {&p, &a};
+  const void* kern = nullptr;
+  if (S == 64) kern = f32 ? reinterpret_cast<const void*>(colslab_kernel<true, 64>)
+                          : reinterpret_cast<const void*>(colslab_kernel<false, 64>);
+  if (S == 128) kern = f32 ? reinterpret_cast<const void*>(colslab_kernel<true, 128>)
+                           : reinterpret_cast<const void*>(colslab_kernel<false, 128>);
+  if (S == 256) kern = f32 ? reinterpret_cast<const void*>(colslab_kernel<true, 256>)
+                           : reinterpret_cast<const void*>(colslab_kernel<false, 256>);
+  return cudaLaunchCooperativeKernel(kern, grid, dim3(kThreads), args, 0, s);
 }
 
 cudaError_t launch_normalize(float* const* vecs, int batch, int n, float* norm, cudaStream_t s) {

@@ -241,6 +241,43 @@ def test_min_singular_full_size_in_proj_streams_in_one_launch():
         assert rel_f(y[l], ry) <= 1e-4
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_min_singular_full_size_out_proj_column_slabs(dtype):
+    """The out_proj group of the 130M model (24 wide 768 x 1536 matrices: X = W, the one-pass
+    column-slab path) against the oracle's shifted iteration, 16 steps."""
+    from spectral_optimizer_state_b200 import Muon
+    rows, cols = 768, 1536
+    Ws = [weights(rng_for(80, l), rows, cols) for l in range(24)]
+    Ws = [round_bf16(w) if dtype == "bf16" else w.astype(np.float32) for w in Ws]
+    y0s = [rng_for(81, l).standard_normal(rows).astype(np.float32) for l in range(24)]
+    smax = [float(np.float32(np.linalg.svd(Ws[l].astype(np.float64), compute_uv=False)[0])) if l in (0, 23)
+            else 1.0 for l in range(24)]
+    with Muon() as muon:
+        y, smin = _min_singular(muon, Ws, y0s, smax, 16, dtype)
+    for l in (0, 23):
+        ry, rs = oracle.min_singular_shifted(Ws[l].astype(np.float64), y0s[l].astype(np.float64), smax[l], 16)
+        assert abs(smin[l] - rs) <= 1e-4 * rs
+        assert rel_f(y[l], ry) <= 1e-4
+
+
+@pytest.mark.parametrize("rows,cols,batch", [(64, 64, 3), (96, 256, 2), (130, 384, 5), (1000, 4096, 1),
+                                             (256, 2048, 24)])
+def test_min_singular_column_slab_shapes(rows, cols, batch):
+    """Slab widths 64 (the first four shapes; a square W is not transposed) and 256 (24 x 2048
+    columns: narrower slabs would not all fit on the GPU at once; 128 is the out_proj case), rows
+    not a multiple of the warps' row stride, against the oracle."""
+    from spectral_optimizer_state_b200 import Muon
+    Ws = [weights(rng_for(82, l), rows, cols).astype(np.float32) for l in range(batch)]
+    y0s = [rng_for(83, l).standard_normal(rows).astype(np.float32) for l in range(batch)]
+    smax = [float(np.float32(np.linalg.svd(w.astype(np.float64), compute_uv=False)[0])) for w in Ws]
+    with Muon() as muon:
+        y, smin = _min_singular(muon, Ws, y0s, smax, 12, "f32")
+    for l in sorted({0, min(1, batch - 1), batch - 1}):
+        ry, rs = oracle.min_singular_shifted(Ws[l].astype(np.float64), y0s[l].astype(np.float64), smax[l], 12)
+        assert abs(smin[l] - rs) <= 1e-4 * rs
+        assert rel_f(y[l], ry) <= 1e-4
+
+
 def test_min_singular_of_semi_orthogonal_is_one():
     from spectral_optimizer_state_b200 import Muon
     Q, _ = np.linalg.qr(rng_for(77, 0).standard_normal((300, 128)))
