@@ -1142,10 +1142,12 @@ muon_status muon_min_singular(muon_ctx* c, const void* const* W, float* const* y
         sp.x[l] = y[l];
         sp.y[l] = reinterpret_cast<float*>(base + part_bytes + tsq_bytes + cnt_bytes + l * t_bytes);
       }
-      MUON_CUDA(launch_power_iteration_stream(sp, batch, f32, nblk, iters + 1, tsq, counters, sigma_min,
-                                              c->d_status, c->sm_count, s, sigma_max),
-                "shifted iteration");
-      return MUON_OK;
+      const cudaError_t e = launch_power_iteration_stream(sp, batch, f32, nblk, iters + 1, tsq, counters,
+                                                          sigma_min, c->d_status, c->sm_count, s, sigma_max);
+      if (e == cudaSuccess) return MUON_OK;
+      // no room for the cooperative launch after all (another client on the device): two GEMVs
+      if (e != cudaErrorCooperativeLaunchTooLarge) return cuda_fail(e, "shifted iteration");
+      (void)cudaGetLastError();
     }
   }
   if (!tall) {
@@ -1170,12 +1172,14 @@ muon_status muon_min_singular(muon_ctx* c, const void* const* W, float* const* y
         sp.w[l] = W[l];
         sp.x[l] = y[l];
       }
-      MUON_CUDA(launch_min_singular_slabs(sp, batch, f32, S, iters, sigma_max,
-                                          reinterpret_cast<float*>(base + part_bytes),
-                                          reinterpret_cast<unsigned*>(base + part_bytes + dsq_bytes), sigma_min,
-                                          c->d_status, s),
-                "shifted iteration (column slabs)");
-      return MUON_OK;
+      const cudaError_t e = launch_min_singular_slabs(sp, batch, f32, S, iters, sigma_max,
+                                                      reinterpret_cast<float*>(base + part_bytes),
+                                                      reinterpret_cast<unsigned*>(base + part_bytes + dsq_bytes),
+                                                      sigma_min, c->d_status, s);
+      if (e == cudaSuccess) return MUON_OK;
+      // no room for the cooperative launch after all (another client on the device): two GEMVs
+      if (e != cudaErrorCooperativeLaunchTooLarge) return cuda_fail(e, "shifted iteration (column slabs)");
+      (void)cudaGetLastError();
     }
   }
   GemvParams gp;

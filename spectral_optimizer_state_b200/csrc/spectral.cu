@@ -1054,7 +1054,7 @@ cudaError_t launch_power_iteration_stream(GemvParams& p, int batch, bool f32, in
   int stages = 0;
   const size_t smem = power_smem_bytes(p.cols, f32, stages);
   // all iterations in one cooperative launch when every block fits on the GPU at once
-  const bool together = iters > 1 && power_pass_together(p.cols, f32, nblk, batch, sm_count);
+  bool together = iters > 1 && power_pass_together(p.cols, f32, nblk, batch, sm_count);
   // the shifted iteration keeps y in shared memory from pass to pass: one launch for all passes
   if (shift != nullptr && iters > 1 && !together) return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(counters, 0, 2 * sizeof(unsigned) * batch, s);
@@ -1091,6 +1091,14 @@ cudaError_t launch_power_iteration_stream(GemvParams& p, int batch, bool f32, in
       MUON_POWER_CASE(7)
       MUON_POWER_CASE(8)
 #undef MUON_POWER_CASE
+    }
+    if (e == cudaErrorCooperativeLaunchTooLarge && together && shift == nullptr) {
+      // the device had less room than its occupancy promised (another client on it): the power
+      // iteration runs as one launch per iteration instead, from the start
+      (void)cudaGetLastError();
+      together = false;
+      a.it1 = 0;
+      continue;
     }
     if (e != cudaSuccess) return e;
   }
