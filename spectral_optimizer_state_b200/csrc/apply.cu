@@ -101,6 +101,22 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
+// O - au v^T on 8 columns c..c+7 (c % 8 == 0): two 16-byte reads of v when the cap's
+// vectors are aligned and the 8 columns exist, else element by element (columns < C).
+__device__ __forceinline__ void cap_term8(float (&ov)[8], float au, const float* v, int c, int C, bool vec) {
+  if (vec && c + 8 <= C) {
+    const float4 x = *reinterpret_cast<const float4*>(v + c);
+    const float4 y = *reinterpret_cast<const float4*>(v + c + 4);
+    const float vv[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int t = 0; t < 8; ++t) ov[t] = fmaf(-au, vv[t], ov[t]);
+  } else {
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      if (c + t < C) ov[t] = fmaf(-au, v[c + t], ov[t]);
+  }
+}
+
 template <bool F32>
 __device__ __forceinline__ void rmw1(void* dst, long long e, float v, bool apply, float decay, float lrs) {
   if (F32) {
@@ -139,11 +155,7 @@ __device__ __forceinline__ void wide_body(const ApplyParams& p, const ApplyGroup
         float ov[8], cw[8];
         load8_planes(o + i * q.pitch + j, q.o_plane, p.planes, ov);
         load8_w<F32>(dst, p.apply, cw);
-        if (cap) {
-          const float au = q.alpha[l] * p.cu[q.mat0 + l][i];
-  #pragma unroll
-          for (int t = 0; t < 8; ++t) ov[t] = fmaf(-au, p.cv[q.mat0 + l][j + t], ov[t]);
-        }
+        if (cap) cap_term8(ov, q.alpha[l] * p.cu[q.mat0 + l][i], p.cv[q.mat0 + l], j, C, q.cvec);
         store8_w<F32>(dst, ov, cw, p.apply, p.decay, q.lrs);
       }
     } else {
@@ -189,11 +201,7 @@ __device__ __forceinline__ void wide_body(const ApplyParams& p, const ApplyGroup
           load8_w<F32>(h ? wb : wa, p.apply, cw);
           const long long ii = h ? i1 : i0;
           const int jj = h ? j1 : j0;
-          if (cap) {
-            const float au = q.alpha[l] * p.cu[q.mat0 + l][ii];
-  #pragma unroll
-            for (int t = 0; t < 8; ++t) ov[t] = fmaf(-au, p.cv[q.mat0 + l][jj + t], ov[t]);
-          }
+          if (cap) cap_term8(ov, q.alpha[l] * p.cu[q.mat0 + l][ii], p.cv[q.mat0 + l], jj, C, q.cvec);
           store8_w<F32>(h ? d1 : d0, ov, cw, p.apply, p.decay, q.lrs);
         }
       }
@@ -293,12 +301,7 @@ __device__ __forceinline__ void tall_body(const ApplyParams& p, const ApplyGroup
         float v[8];
 #pragma unroll
         for (int t = 0; t < 8; ++t) v[t] = tile[rl][cc + t];
-        if (cap) {
-          const float au = q.alpha[l] * p.cu[q.mat0 + l][r];
-#pragma unroll
-          for (int t = 0; t < 8; ++t)
-            if (c + t < C) v[t] = fmaf(-au, p.cv[q.mat0 + l][c + t], v[t]);
-        }
+        if (cap) cap_term8(v, q.alpha[l] * p.cu[q.mat0 + l][r], p.cv[q.mat0 + l], c, C, q.cvec);
         if (wvec) {
           char* dst = static_cast<char*>(w) + (static_cast<long long>(r) * C + c) * (F32 ? 4 : 2);
           float cw[8];
@@ -315,8 +318,10 @@ __device__ __forceinline__ void tall_body(const ApplyParams& p, const ApplyGroup
   }
 }
 
+// Six blocks per SM (40 registers) for the plain pass; the capped instantiation, which also
+// carries the rank-one term, four (64 registers) so that it does not spill.
 template <bool F32, bool CAP>
-__global__ void __launch_bounds__(kThreads, 6) apply_kernel(const __grid_constant__ ApplyParams p) {
+__global__ void __launch_bounds__(kThreads, CAP ? 4 : 6) apply_kernel(const __grid_constant__ ApplyParams p) {
   int gi = 0;
   while (gi + 1 < p.ngroups && static_cast<int>(blockIdx.x) >= p.grp[gi + 1].block0) ++gi;
   const ApplyGroup& q = p.grp[gi];
@@ -343,6 +348,9 @@ cudaError_t launch_apply(ApplyParams& p, bool w_f32, cudaStream_t stream) {
     q.vec = q.cols % 8 == 0;
     for (int l = 0; l < q.batch && q.vec; ++l)
       if (reinterpret_cast<uintptr_t>(p.w[q.mat0 + l]) % 16) q.vec = 0;
+    q.cvec = q.alpha != nullptr;
+    for (int l = 0; l < q.batch && q.cvec; ++l)
+      if (reinterpret_cast<uintptr_t>(p.cv[q.mat0 + l]) % 16) q.cvec = 0;
     cap = cap || q.alpha != nullptr;
     blocks += static_cast<long long>(q.batch) * q.nblk;
   }

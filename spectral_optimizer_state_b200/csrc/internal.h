@@ -52,6 +52,7 @@ int momentum_blocks_per_matrix(int rows, int cols);
 // ------------------------------------------------------------------ K5 apply
 struct ApplyGroup {
   int mat0, batch, rows, cols, nblk, block0, vec;
+  int cvec;                 // the cap's v vectors are 16-byte aligned (read 8 at a time)
   const uint16_t* o;        // final iterate [planes][batch][m][pitch] bf16 bits (wide)
   long long o_plane, o_mat; // elements
   int pitch;
@@ -92,9 +93,11 @@ struct CapParams {
   const float* b[MUON_MAX_BATCH];  // length n (wide columns)
   const uint16_t* o;               // final iterate, wide, [planes][batch][m][pitch]
   long long o_plane, o_mat;
-  int pitch, m, n, planes, rows_per_block;
-  double* partial;                 // [batch][blocks]
+  int pitch, m, n, planes;
+  double* partial;                 // [batch][ceil(m / 32)]: one per block of 32 rows
 };
+// Blocks of the cap coefficient pass per matrix (32 rows each).
+inline int cap_alpha_blocks(int m) { return (m + 31) / 32; }
 
 // `iters` power iterations, one pass over W each (u <- W v / |W v|, v <- W^T u / |W^T u|,
 // sigma = |W^T u|), in one cooperative launch when the blocks fit on the GPU at once, else one

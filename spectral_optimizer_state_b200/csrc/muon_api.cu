@@ -661,8 +661,7 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
       cp.m = p.m_rows;
       cp.n = p.n_cols;
       cp.planes = p.planes;
-      cp.rows_per_block = 8;
-      const size_t need = sizeof(double) * p.batch * ((p.m_rows + 7) / 8);
+      const size_t need = sizeof(double) * p.batch * cap_alpha_blocks(p.m_rows);
       st = ensure_aux(c, need);
       if (st != MUON_OK) return st;
       cp.partial = static_cast<double*>(c->d_aux);

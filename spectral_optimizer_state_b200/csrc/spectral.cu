@@ -664,48 +664,98 @@ __global__ void __launch_bounds__(kThreads) shift_normalize_kernel(const __grid_
 }
 
 // alpha partials: wide O (m x n, planes summed) against a (length m) and b (length n).
-// One warp per row of O (rows_per_block == warps per block); each lane reads
-// 16-byte vectors of every plane (the wide pitch is a multiple of 64 elements,
-// so row starts are 128-byte aligned) and the ragged tail element by element.
+// A block takes kCapRows rows, kCapRowsPerWarp per warp at once; b is staged in shared memory
+// once per block in the layout whose 16-byte reads of a lane's 8 columns are bank-conflict
+// free (vs_index), and each lane reads 16-byte vectors of every plane of its warp's rows
+// (the wide pitch is a multiple of 64 elements, so row starts are 128-byte aligned), two
+// column chunks ahead, and the ragged tail element by element.  The block's partial is
+// sum over its rows (in order) of a_i (O_i . b), the row dots by a fixed xor tree.
+constexpr int kCapRowsPerWarp = 4;
+constexpr int kCapRows = kCapRowsPerWarp * (kThreads / 32);
+
+template <int PLANES>
 __global__ void __launch_bounds__(kThreads) cap_alpha_partial_kernel(const __grid_constant__ CapParams p) {
-  __shared__ double scratch[kThreads / 32];
+  extern __shared__ __align__(16) float bs[];  // [round_up(n, 256)], vs_index layout
+  __shared__ double wsum[kThreads / 32];
   const int l = blockIdx.y;
   const float* a = p.a[l];
   const float* b = p.b[l];
+  const int n = p.n;
+  const int nr = (n + 255) & ~255;
+  for (int c = threadIdx.x; c < nr; c += kThreads) bs[vs_index(c)] = c < n ? b[c] : 0.f;
+  __syncthreads();
   const uint16_t* o = p.o + static_cast<long long>(l) * p.o_mat;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.x * (kThreads / 32) + warp;
-  double acc = 0.0;
-  if (i < p.m) {
-    const uint16_t* row = o + static_cast<long long>(i) * p.pitch;
-    const int nv = p.n & ~7;
-    float s = 0.f;
-    for (int j = lane * 8; j < nv; j += 32 * 8) {
+  const int r0 = blockIdx.x * kCapRows + warp * kCapRowsPerWarp;
+  const int nv = n & ~7;  // whole 8-column chunks
+  float s[kCapRowsPerWarp];
+#pragma unroll
+  for (int k = 0; k < kCapRowsPerWarp; ++k) s[k] = 0.f;
+  auto chunk = [&](int j, float (&acc)[kCapRowsPerWarp]) {
+    // this lane's 8 columns j..j+7 of the warp's rows, every plane summed, against b; all the
+    // rows' and planes' 16-byte loads are issued before any is used
+    uint4 w[kCapRowsPerWarp][PLANES];
+#pragma unroll
+    for (int k = 0; k < kCapRowsPerWarp; ++k)
+#pragma unroll
+      for (int q = 0; q < PLANES; ++q)
+        w[k][q] = r0 + k < p.m ? __ldcs(reinterpret_cast<const uint4*>(o + q * p.o_plane +
+                                                                      static_cast<long long>(r0 + k) * p.pitch + j))
+                               : make_uint4(0u, 0u, 0u, 0u);
+    const int i = j >> 8, ln = (j & 255) >> 3;
+    const float4 lo = *reinterpret_cast<const float4*>(bs + 256 * i + 4 * ln);
+    const float4 hi = *reinterpret_cast<const float4*>(bs + 256 * i + 128 + 4 * ln);
+    const float bb[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+    for (int k = 0; k < kCapRowsPerWarp; ++k) {
       float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      for (int q = 0; q < p.planes; ++q) {
-        const uint4 w = __ldcs(reinterpret_cast<const uint4*>(row + q * p.o_plane + j));
-        const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int q = 0; q < PLANES; ++q) {
+        const uint32_t u[4] = {w[k][q].x, w[k][q].y, w[k][q].z, w[k][q].w};
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           v[2 * t] += __uint_as_float(u[t] << 16);
           v[2 * t + 1] += __uint_as_float(u[t] & 0xFFFF0000u);
         }
       }
-      // b is the caller's vector with no alignment promise: scalar reads (it stays in L1)
 #pragma unroll
-      for (int t = 0; t < 8; ++t) s = fmaf(v[t], __ldg(b + j + t), s);
+      for (int t = 0; t < 8; ++t) acc[k] = fmaf(v[t], bb[t], acc[k]);
     }
-    for (int j = nv + lane; j < p.n; j += 32) {
-      float v = 0.f;
-      for (int q = 0; q < p.planes; ++q) v += bf16_bits_to_float(row[q * p.o_plane + j]);
-      s = fmaf(v, b[j], s);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    acc = static_cast<double>(s) * a[i];
+  };
+  int j = lane * 8;
+  for (; j + 256 < nv; j += 512) {
+    chunk(j, s);
+    chunk(j + 256, s);
   }
-  const double tot = block_sum<double>(lane == 0 ? acc : 0.0, scratch);
-  if (threadIdx.x == 0) p.partial[static_cast<long long>(l) * gridDim.x + blockIdx.x] = tot;
+  for (; j < nv; j += 256) chunk(j, s);
+  for (int jj = nv + lane; jj < n; jj += 32) {
+#pragma unroll
+    for (int k = 0; k < kCapRowsPerWarp; ++k) {
+      const int r = r0 + k;
+      if (r >= p.m) continue;
+      float v = 0.f;
+#pragma unroll
+      for (int q = 0; q < PLANES; ++q)
+        v += bf16_bits_to_float(o[q * p.o_plane + static_cast<long long>(r) * p.pitch + jj]);
+      s[k] = fmaf(v, bs[vs_index(jj)], s[k]);
+    }
+  }
+  double acc = 0.0;
+#pragma unroll
+  for (int k = 0; k < kCapRowsPerWarp; ++k) {
+    float d = s[k];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+    if (r0 + k < p.m) acc += static_cast<double>(d) * a[r0 + k];
+  }
+  if (lane == 0) wsum[warp] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) t += wsum[w];
+    p.partial[static_cast<long long>(l) * gridDim.x + blockIdx.x] = t;
+  }
 }
 
 __global__ void cap_alpha_reduce_kernel(const double* partial, int nblk, float* alpha) {
@@ -1187,10 +1237,16 @@ cudaError_t launch_shift_normalize(float* const* y, const float* const* z, int b
 }
 
 cudaError_t launch_cap_alpha(const CapParams& p, int batch, float* alpha, cudaStream_t s) {
-  // one warp per row: p.rows_per_block must equal the warps of a block
-  if (p.rows_per_block != kThreads / 32) return cudaErrorInvalidValue;
-  const int nblk = (p.m + p.rows_per_block - 1) / p.rows_per_block;
-  cap_alpha_partial_kernel<<<dim3(nblk, batch), kThreads, 0, s>>>(p);
+  const int nblk = (p.m + kCapRows - 1) / kCapRows;
+  const size_t smem = sizeof(float) * ((p.n + 255) & ~255);
+  if (p.planes != 1 && p.planes != 3) return cudaErrorInvalidValue;
+  auto kern = p.planes == 1 ? cap_alpha_partial_kernel<1> : cap_alpha_partial_kernel<3>;
+  if (smem > 48 * 1024) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<dim3(nblk, batch), kThreads, smem, s>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   cap_alpha_reduce_kernel<<<batch, 32, 0, s>>>(p.partial, nblk, alpha);
