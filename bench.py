@@ -125,9 +125,9 @@ def _code_only(text):
 
 
 def gemm_source_hash():
-    """sha256 (16 hex digits) of the NS kernel's code: gemm.cu, device_utils.cuh, internal.h without comments."""
+    """sha256 (16 hex digits) of the NS kernel's code: gemm.cu, gemm.h, device_utils.cuh without comments."""
     h = hashlib.sha256()
-    for f in ("gemm.cu", "device_utils.cuh", "internal.h"):
+    for f in ("gemm.cu", "gemm.h", "device_utils.cuh"):
         with open(os.path.join(ROOT, "spectral_optimizer_state_b200", "csrc", f)) as fh:
             h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]

@@ -36,7 +36,7 @@
 #include <cuda_bf16.h>
 
 #include "device_utils.cuh"
-#include "internal.h"
+#include "gemm.h"
 
 namespace muon {
 
