@@ -261,7 +261,7 @@ def test_min_singular_full_size_out_proj_column_slabs(dtype):
 
 
 @pytest.mark.parametrize("rows,cols,batch", [(64, 64, 3), (96, 256, 2), (130, 384, 5), (1000, 4096, 1),
-                                             (256, 2048, 24)])
+                                             (256, 2048, 24), (1, 64, 2), (3, 192, 2)])
 def test_min_singular_column_slab_shapes(rows, cols, batch):
     """Slab widths 64 (the first four shapes; a square W is not transposed) and 256 (24 x 2048
     columns: narrower slabs would not all fit on the GPU at once; 128 is the out_proj case), rows
@@ -274,6 +274,23 @@ def test_min_singular_column_slab_shapes(rows, cols, batch):
         y, smin = _min_singular(muon, Ws, y0s, smax, 12, "f32")
     for l in sorted({0, min(1, batch - 1), batch - 1}):
         ry, rs = oracle.min_singular_shifted(Ws[l].astype(np.float64), y0s[l].astype(np.float64), smax[l], 12)
+        assert abs(smin[l] - rs) <= 1e-4 * rs
+        assert rel_f(y[l], ry) <= 1e-4
+
+
+@pytest.mark.parametrize("rows,cols", [(9, 8), (17, 16), (40, 8)])
+def test_min_singular_small_tall_streaming(rows, cols):
+    """Tall W with few columns on the streaming shifted path: a stage of fewer than eight rows,
+    one block per matrix."""
+    from spectral_optimizer_state_b200 import Muon
+    batch = 3
+    Ws = [weights(rng_for(84, l), rows, cols).astype(np.float32) for l in range(batch)]
+    y0s = [rng_for(85, l).standard_normal(cols).astype(np.float32) for l in range(batch)]
+    smax = [float(np.float32(np.linalg.svd(w.astype(np.float64), compute_uv=False)[0])) for w in Ws]
+    with Muon() as muon:
+        y, smin = _min_singular(muon, Ws, y0s, smax, 10, "f32")
+    for l in range(batch):
+        ry, rs = oracle.min_singular_shifted(Ws[l].astype(np.float64), y0s[l].astype(np.float64), smax[l], 10)
         assert abs(smin[l] - rs) <= 1e-4 * rs
         assert rel_f(y[l], ry) <= 1e-4
 
