@@ -1,0 +1,114 @@
+"""Host-side checks of the index arithmetic the elementwise and spectral kernels use (mirrors of
+the device code, no GPU): the strided row walk of the momentum and apply passes, the shared-memory
+layout of v in the streaming spectral passes, the row coverage of the column-slab pass and the
+block / stage split of the power pass.  Each mirror is compared with the plain definition
+(division, a dense loop) it replaces."""
+import pytest
+
+
+# ---------------------------------------------------------------- strided row walk (rowpos.cuh)
+def rowpos_at(v, per_row):
+    i = v // per_row
+    return [i, v - i * per_row]
+
+
+def rowstep_of(stride, per_row):
+    return stride // per_row, stride % per_row
+
+
+def rowpos_add(p, step, per_row):
+    i, j = p[0] + step[0], p[1] + step[1]
+    if j >= per_row:
+        j -= per_row
+        i += 1
+    return [i, j]
+
+
+@pytest.mark.parametrize("per_row", [1, 7, 96, 192, 384, 419, 1000, 4096])
+@pytest.mark.parametrize("stride", [1, 7, 256, 512])
+def test_row_walk_matches_division(per_row, stride):
+    """Walking a flattened index in fixed strides by one division at the start and an add with at
+    most one wrap per step gives the same (row, position) as dividing at every step."""
+    step = rowstep_of(stride, per_row)
+    for start in (0, 1, per_row - 1, 3 * per_row + 5, 123457):
+        p = rowpos_at(start, per_row)
+        v = start
+        for _ in range(200):
+            assert p == [v // per_row, v % per_row]
+            v += stride
+            p = rowpos_add(p, step, per_row)
+
+
+# ---------------------------------------------------------------- v in shared memory (vs_index)
+def vs_index(c):
+    return (c & ~255) | ((c & 4) << 5) | (((c & 255) >> 3) << 2) | (c & 3)
+
+
+@pytest.mark.parametrize("cols", [8, 256, 520, 768, 1536, 2048])
+def test_split_layout_is_a_bijection_with_conflict_free_lane_reads(cols):
+    """The split layout maps the columns of every 256-column chunk one to one onto that chunk's
+    256 slots; lane k's 16-byte reads at 4k and 128 + 4k of chunk i hold columns 8k..8k+3 and
+    8k+4..8k+7, and the eight lanes of a quarter warp read eight distinct 16-byte slots of one
+    128-byte row (no bank conflict)."""
+    span = (cols + 255) & ~255
+    pos = [vs_index(c) for c in range(span)]
+    assert sorted(pos) == list(range(span))
+    for i in range(span // 256):
+        for k in range(32):
+            lo = [pos.index(256 * i + 4 * k + t) for t in range(4)]
+            hi = [pos.index(256 * i + 128 + 4 * k + t) for t in range(4)]
+            assert lo == [256 * i + 8 * k + t for t in range(4)]
+            assert hi == [256 * i + 8 * k + 4 + t for t in range(4)]
+        for q in range(4):  # quarter warps
+            for base in (0, 128):
+                # first of the four 4-byte banks each 16-byte read covers
+                slots = {(256 * i + base + 4 * k) % 32 // 4 for k in range(8 * q, 8 * q + 8)}
+                assert len(slots) == 8
+
+
+# ---------------------------------------------------------------- column-slab phase 1 rows
+@pytest.mark.parametrize("S", [64, 128, 256])
+@pytest.mark.parametrize("rows", [1, 3, 31, 64, 130, 768, 1000])
+def test_column_slab_rows_each_read_once(S, rows):
+    """Phase 1 of the column-slab pass: warp w and row group g of its lanes start at row
+    w * RPW + g and step by (warps x RPW) rows, kSlabUnroll rows per pass of the loop; every row
+    of the slab is read by exactly one (warp, row group)."""
+    warps, unroll = 8, 8
+    lpr = S // 8
+    rpw = 32 // lpr
+    rstride = warps * rpw
+    seen = [0] * rows
+    for w in range(warps):
+        for g in range(rpw):
+            r0 = w * rpw + g
+            while r0 < rows:
+                for u in range(unroll):
+                    r = r0 + u * rstride
+                    if r < rows:
+                        seen[r] += 1
+                r0 += rstride * unroll
+    assert seen == [1] * rows
+
+
+# ---------------------------------------------------------------- power pass blocks and stages
+def power_blocks(rows, want):
+    rpb = ((rows + want - 1) // want + 7) // 8 * 8
+    return (rows + rpb - 1) // rpb, rpb
+
+
+@pytest.mark.parametrize("rows", [1, 8, 9, 77, 300, 768, 3352, 4000, 32768])
+@pytest.mark.parametrize("want", [1, 2, 12, 37, 64])
+def test_power_pass_blocks_cover_rows_in_whole_stages(rows, want):
+    """The row split of the streaming power pass: every block but the last holds a multiple of
+    eight rows (whole stages), no block is empty, the blocks cover the rows exactly once, and there
+    are never more blocks than asked for (the per-matrix partial count the launch sizes)."""
+    nblk, rpb = power_blocks(rows, want)
+    assert 1 <= nblk <= max(1, want) and rpb % 8 == 0
+    covered = []
+    for b in range(nblk):
+        beg, end = b * rpb, min(rows, b * rpb + rpb)
+        assert end > beg
+        nst = (end - beg + 7) // 8  # stages of eight rows
+        assert nst * 8 >= end - beg > (nst - 1) * 8
+        covered.extend(range(beg, end))
+    assert covered == list(range(rows))
