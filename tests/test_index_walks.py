@@ -48,8 +48,8 @@ def vs_index(c):
 def test_split_layout_is_a_bijection_with_conflict_free_lane_reads(cols):
     """The split layout maps the columns of every 256-column chunk one to one onto that chunk's
     256 slots; lane k's 16-byte reads at 4k and 128 + 4k of chunk i hold columns 8k..8k+3 and
-    8k+4..8k+7, and the eight lanes of a quarter warp read eight distinct 16-byte slots of one
-    128-byte row (no bank conflict)."""
+    8k+4..8k+7, and the eight lanes of a quarter warp start their 16-byte reads in eight distinct
+    groups of four banks (no bank conflict)."""
     span = (cols + 255) & ~255
     pos = [vs_index(c) for c in range(span)]
     assert sorted(pos) == list(range(span))
