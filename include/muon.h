@@ -39,6 +39,19 @@
  *   - Work a call puts on the context's internal streams (the uploads of
  *     muon_step_groups_host) starts after what is already queued on `stream`
  *     and joins back into `stream` before the call's last kernel.
+ *   - CUDA graphs: muon_step_groups, muon_step_capped, muon_ns_orthogonalize,
+ *     muon_power_iteration and muon_min_singular queue only memsets and
+ *     kernel launches once the context's buffers are large enough, so they
+ *     may be captured on `stream` and the graph replayed, as long as the
+ *     pointers and sizes stay the same.  The first call of a shape grows
+ *     them, which synchronises the device: made while `stream` is capturing,
+ *     such a call returns MUON_ERR_ALLOC before queuing anything and leaves
+ *     the capture intact (muon_last_cuda_error says why).  Make the same
+ *     call once before capture.  A graph keeps the addresses of the
+ *     context's buffers, so once any call of a context has been captured the
+ *     context never grows again: a later call that would need more returns
+ *     MUON_ERR_ALLOC (use another context for it).  muon_step_groups_host
+ *     and muon_get_status synchronise and cannot be captured.
  *   - No C++ exception crosses this interface.
  */
 #ifndef LIBMUON_MUON_H
@@ -69,7 +82,7 @@ typedef enum {
   MUON_ERR_NONFINITE = 5,        /* device: ||U||_F was not finite for >= 1 matrix            */
   MUON_ERR_TIMEOUT = 6,          /* device: a bounded wait inside a kernel ran out            */
   MUON_ERR_NO_DEVICE = 7,        /* no usable CUDA device / device is not sm_100              */
-  MUON_ERR_ALLOC = 8             /* workspace allocation failed                               */
+  MUON_ERR_ALLOC = 8             /* workspace allocation failed, or refused while capturing  */
 } muon_status;
 
 typedef enum { MUON_BF16 = 0, MUON_F32 = 1 } muon_dtype;

@@ -168,7 +168,7 @@ class Muon:
     def _check(self, st: int, what: str):
         if st != MUON_OK:
             detail = ""
-            if st == 4:
+            if st in (4, 8):
                 detail = self.lib.muon_last_cuda_error().decode()
             raise MuonError(st, what, detail)
 

@@ -36,6 +36,29 @@ muon_status cuda_fail(cudaError_t e, const char* what) {
     if (_e != cudaSuccess) return cuda_fail(_e, what); \
   } while (0)
 
+// Capture state of `s`: 0 not capturing, 1 capturing into a CUDA graph, -1 unreadable.
+int capture_state(cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  return cs == cudaStreamCaptureStatusNone ? 0 : 1;
+}
+
+muon_status refuse_growth(const char* what, const char* why) {
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  std::snprintf(g_cuda_error, sizeof(g_cuda_error), "%s must grow, but %s", what, why);
+  return MUON_ERR_ALLOC;
+}
+
+// Records why a device allocation failed (and clears the error) for muon_last_cuda_error.
+void note_alloc_failure() {
+  const cudaError_t e = cudaGetLastError();
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  std::snprintf(g_cuda_error, sizeof(g_cuda_error), "device allocation: %s", cudaGetErrorString(e));
+}
+
 // ------------------------------------------------------------------ tensor maps
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -149,6 +172,7 @@ struct muon_ctx {
   int last_count = 0;
   cudaStream_t last_stream = nullptr;
   bool pending = false;
+  bool captured = false;        // a call was captured into a CUDA graph: the buffers never move again
   // device staging for gradients that arrive from host memory
   void* d_stage = nullptr;
   size_t stage_bytes = 0;
@@ -236,6 +260,26 @@ float shape_scale(int rows, int cols, int mode) {
 }
 
 // Make sure the workspace and the per-matrix arrays can hold `plans`.
+// Growing a context buffer synchronises the device and allocates; neither is allowed while the
+// call's stream is being captured into a CUDA graph, and either would invalidate the capture.  A
+// graph captured earlier keeps the buffers' addresses, so once a call has been captured the
+// buffers never move again.  In both cases the call is refused before anything is queued (a
+// capture in progress stays usable).  A stream whose capture state cannot be read counts as
+// capturing: growth would fail on it too.
+muon_status may_grow(muon_ctx* c, cudaStream_t s, const char* what) {
+  if (capture_state(s) != 0)
+    return refuse_growth(what, "the stream is capturing a CUDA graph: make the same call once before capture");
+  if (c->captured)
+    return refuse_growth(what, "a CUDA graph captured from this context holds its buffers: use another context");
+  return MUON_OK;
+}
+
+// Called before any work of a call is queued on `s`: remembers that the context's buffers now
+// sit in a captured graph.
+void note_capture(muon_ctx* c, cudaStream_t s) {
+  if (capture_state(s) == 1) c->captured = true;
+}
+
 muon_status reserve(muon_ctx* c, std::vector<GroupPlan>& plans, cudaStream_t s) {
   size_t bytes = 0;
   int mats = 0;
@@ -252,18 +296,25 @@ muon_status reserve(muon_ctx* c, std::vector<GroupPlan>& plans, cudaStream_t s) 
     p.part_off = static_cast<int>(parts);
     parts += static_cast<size_t>(p.batch) * p.nblk;
   }
-  if (bytes > c->ws_bytes) {
+  const bool grow_ws = bytes > c->ws_bytes;
+  const bool grow_arrays = mats > c->cap_mats || parts > c->cap_parts;
+  if (grow_ws || grow_arrays) {
+    const muon_status st = may_grow(c, s, "the workspace");
+    if (st != MUON_OK) return st;
+  }
+  note_capture(c, s);
+  if (grow_ws) {
     MUON_CUDA(cudaDeviceSynchronize(), "sync before workspace growth");
     if (c->ws) cudaFree(c->ws);
     c->ws = nullptr;
     c->ws_bytes = 0;
     if (cudaMalloc(&c->ws, bytes) != cudaSuccess) {
-      cudaGetLastError();
+      note_alloc_failure();
       return MUON_ERR_ALLOC;
     }
     c->ws_bytes = bytes;
   }
-  if (mats > c->cap_mats || parts > c->cap_parts) {
+  if (grow_arrays) {
     MUON_CUDA(cudaDeviceSynchronize(), "sync before array growth");
     cudaFree(c->d_nu); cudaFree(c->d_s1); cudaFree(c->d_s2); cudaFree(c->d_flags);
     cudaFree(c->d_counters); cudaFree(c->d_partials);
@@ -279,7 +330,7 @@ muon_status reserve(muon_ctx* c, std::vector<GroupPlan>& plans, cudaStream_t s) 
               cudaMalloc(&c->d_counters, cm * sizeof(unsigned)) == cudaSuccess &&
               cudaMalloc(&c->d_partials, cp * sizeof(float)) == cudaSuccess;
     if (!ok) {
-      cudaGetLastError();
+      note_alloc_failure();
       c->cap_mats = 0;
       c->cap_parts = 0;
       return MUON_ERR_ALLOC;
@@ -392,14 +443,19 @@ struct CapSpec {
   float* alpha;  // device [batch]
 };
 
-muon_status ensure_aux(muon_ctx* c, size_t bytes) {
-  if (bytes <= c->aux_bytes) return MUON_OK;
+muon_status ensure_aux(muon_ctx* c, size_t bytes, cudaStream_t s) {
+  if (bytes <= c->aux_bytes) {
+    note_capture(c, s);
+    return MUON_OK;
+  }
+  const muon_status st = may_grow(c, s, "the scratch");
+  if (st != MUON_OK) return st;
   MUON_CUDA(cudaDeviceSynchronize(), "sync before scratch growth");
   cudaFree(c->d_aux);
   c->d_aux = nullptr;
   c->aux_bytes = 0;
   if (cudaMalloc(&c->d_aux, bytes) != cudaSuccess) {
-    cudaGetLastError();
+    note_alloc_failure();
     return MUON_ERR_ALLOC;
   }
   c->aux_bytes = bytes;
@@ -410,6 +466,10 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
                 float eps, cudaStream_t s, const CapSpec* cap = nullptr, bool clear_status = true) {
   muon_status st = reserve(c, plans, s);
   if (st != MUON_OK) return st;
+  if (cap != nullptr) {  // per-block partials of the cap coefficients, sized before any launch
+    st = ensure_aux(c, sizeof(double) * plans[0].batch * cap_alpha_blocks(plans[0].m_rows), s);
+    if (st != MUON_OK) return st;
+  }
   int total = 0;
   for (auto& p : plans) total += p.batch;
   if (clear_status) MUON_CUDA(cudaMemsetAsync(c->d_status, 0, sizeof(int), s), "clear status");
@@ -661,9 +721,6 @@ muon_status run(muon_ctx* c, std::vector<GroupPlan>& plans, const muon_hparams* 
       cp.m = p.m_rows;
       cp.n = p.n_cols;
       cp.planes = p.planes;
-      const size_t need = sizeof(double) * p.batch * cap_alpha_blocks(p.m_rows);
-      st = ensure_aux(c, need);
-      if (st != MUON_OK) return st;
       cp.partial = static_cast<double*>(c->d_aux);
       MUON_CUDA(launch_cap_alpha(cp, p.batch, cap->alpha, s), "cap coefficient");
     }
@@ -759,13 +816,13 @@ muon_status muon_create(muon_ctx** out, int device) {
     }
   }
   if (cudaMalloc(&c->d_status, sizeof(int)) != cudaSuccess) {
-    cudaGetLastError();
+    note_alloc_failure();
     delete c;
     return MUON_ERR_ALLOC;
   }
   cudaMemset(c->d_status, 0, sizeof(int));
   if (cudaMalloc(&c->d_done, sizeof(unsigned) * kMaxProblems * MUON_MAX_BATCH) != cudaSuccess) {
-    cudaGetLastError();
+    note_alloc_failure();
     cudaFree(c->d_status);
     delete c;
     return MUON_ERR_ALLOC;
@@ -917,7 +974,7 @@ muon_status muon_step_groups_host(muon_ctx* c, const muon_group* groups, int ngr
     c->d_stage = nullptr;
     c->stage_bytes = 0;
     if (cudaMalloc(&c->d_stage, need) != cudaSuccess) {
-      cudaGetLastError();
+      note_alloc_failure();
       return MUON_ERR_ALLOC;
     }
     c->stage_bytes = need;
@@ -980,7 +1037,7 @@ muon_status muon_step_groups_host(muon_ctx* c, const muon_group* groups, int ngr
       c->cap_all = 0;
       if (cudaMalloc(&c->d_nu_all, sizeof(float) * total) != cudaSuccess ||
           cudaMalloc(&c->d_flags_all, sizeof(int) * total) != cudaSuccess) {
-        cudaGetLastError();
+        note_alloc_failure();
         return MUON_ERR_ALLOC;
       }
       c->cap_all = total;
@@ -1060,7 +1117,7 @@ muon_status muon_power_iteration(muon_ctx* c, const void* const* W, float* const
     const int nblk = power_pass_blocks(rows, cols, batch, f32, c->sm_count);
     const size_t part_bytes = align_up(2 * sizeof(float) * batch * nblk * cols, 256);
     const size_t tsq_bytes = align_up(sizeof(float) * batch * nblk, 256);
-    muon_status st = ensure_aux(c, part_bytes + tsq_bytes + 2 * sizeof(unsigned) * batch);
+    muon_status st = ensure_aux(c, part_bytes + tsq_bytes + 2 * sizeof(unsigned) * batch, s);
     if (st != MUON_OK) return st;
     gp.partial = static_cast<float*>(c->d_aux);
     float* tsq = reinterpret_cast<float*>(static_cast<char*>(c->d_aux) + part_bytes);
@@ -1077,7 +1134,7 @@ muon_status muon_power_iteration(muon_ctx* c, const void* const* W, float* const
   gp.rows_per_chunk = 64;
   gp.row_chunks = (rows + 63) / 64;
   const size_t part_bytes = align_up(sizeof(float) * batch * gp.row_chunks * cols, 256);
-  muon_status st = ensure_aux(c, part_bytes + sizeof(float) * MUON_MAX_BATCH);
+  muon_status st = ensure_aux(c, part_bytes + sizeof(float) * MUON_MAX_BATCH, s);
   if (st != MUON_OK) return st;
   gp.partial = static_cast<float*>(c->d_aux);
   float* norms = reinterpret_cast<float*>(static_cast<char*>(c->d_aux) + part_bytes);
@@ -1126,7 +1183,7 @@ muon_status muon_min_singular(muon_ctx* c, const void* const* W, float* const* y
       const size_t tsq_bytes = align_up(sizeof(float) * batch * nblk, 256);
       const size_t cnt_bytes = align_up(2 * sizeof(unsigned) * batch, 256);
       const size_t t_bytes = align_up(sizeof(float) * rows, 256);
-      muon_status st = ensure_aux(c, part_bytes + tsq_bytes + cnt_bytes + batch * t_bytes);
+      muon_status st = ensure_aux(c, part_bytes + tsq_bytes + cnt_bytes + batch * t_bytes, s);
       if (st != MUON_OK) return st;
       char* base = static_cast<char*>(c->d_aux);
       GemvParams sp;
@@ -1159,7 +1216,7 @@ muon_status muon_min_singular(muon_ctx* c, const void* const* W, float* const* y
       const int nslab = cols / S;
       const size_t part_bytes = align_up(2 * sizeof(float) * batch * nslab * rows, 256);
       const size_t dsq_bytes = align_up(sizeof(float) * batch * nslab, 256);
-      muon_status st = ensure_aux(c, part_bytes + dsq_bytes + 2 * sizeof(unsigned) * batch);
+      muon_status st = ensure_aux(c, part_bytes + dsq_bytes + 2 * sizeof(unsigned) * batch, s);
       if (st != MUON_OK) return st;
       char* base = static_cast<char*>(c->d_aux);
       GemvParams sp;
@@ -1189,7 +1246,7 @@ muon_status muon_min_singular(muon_ctx* c, const void* const* W, float* const* y
   gp.row_chunks = (rows + 63) / 64;
   const size_t part_bytes = align_up(sizeof(float) * batch * gp.row_chunks * cols, 256);
   const size_t w_bytes = align_up(sizeof(float) * n, 256), z_bytes = align_up(sizeof(float) * m, 256);
-  muon_status st = ensure_aux(c, part_bytes + batch * (w_bytes + z_bytes));
+  muon_status st = ensure_aux(c, part_bytes + batch * (w_bytes + z_bytes), s);
   if (st != MUON_OK) return st;
   char* base = static_cast<char*>(c->d_aux);
   gp.partial = reinterpret_cast<float*>(base);
