@@ -194,13 +194,11 @@ __device__ __forceinline__ void raw_to_pairs(const Raw8w<F32>& r, uint64_t (&x)[
 // Two rows at once (the second when has1), both read from their shared-memory stage:
 // t = W[r, :] . v for each, then z += t W[r, :], on (even, odd) column pairs.  Each dot product
 // runs as two pair chains (the first and last four columns of every eight); the two rows' chains
-// and shuffle trees interleave.  Rows of up to 512 columns keep their pairs in registers for the
-// z update; longer ones read the stage again rather than hold them across the trees.
+// and shuffle trees interleave.  The z update reads the stage again rather than hold the rows'
+// pairs across the trees (within the 96 registers two blocks per SM leave).
 template <bool F32, int NV>
 __device__ __forceinline__ void power_rows2(const uint8_t* row0, const uint8_t* row1, bool has1, const float* vs,
                                             int C, int lane, uint64_t (&z)[NV][4], float& t0, float& t1) {
-  constexpr bool kKeep = NV <= 2;
-  uint64_t x0[kKeep ? NV : 1][4], x1[kKeep ? NV : 1][4];
   uint64_t a0 = 0, b0 = 0, a1 = 0, b1 = 0;  // (+0.0f, +0.0f) pairs
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
@@ -216,9 +214,6 @@ __device__ __forceinline__ void power_rows2(const uint8_t* row0, const uint8_t* 
       a0 = fma_f2(x[1], lo.y, a0);
       b0 = fma_f2(x[2], hi.x, b0);
       b0 = fma_f2(x[3], hi.y, b0);
-      if (kKeep)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) x0[kKeep ? i : 0][k] = x[k];
       if (has1) {
         load_raw_smem<F32>(row1, c, w);
         raw_to_pairs<F32>(w, x);
@@ -226,9 +221,6 @@ __device__ __forceinline__ void power_rows2(const uint8_t* row0, const uint8_t* 
         a1 = fma_f2(x[1], lo.y, a1);
         b1 = fma_f2(x[2], hi.x, b1);
         b1 = fma_f2(x[3], hi.y, b1);
-        if (kKeep)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) x1[kKeep ? i : 0][k] = x[k];
       }
     }
   }
@@ -250,25 +242,14 @@ __device__ __forceinline__ void power_rows2(const uint8_t* row0, const uint8_t* 
     const int c = 8 * lane + 256 * i;
     if (c < C) {
       uint64_t x[4];
-      if (kKeep) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) x[k] = x0[kKeep ? i : 0][k];
-      } else {
-        Raw8w<F32> w;
-        load_raw_smem<F32>(row0, c, w);
-        raw_to_pairs<F32>(w, x);
-      }
+      Raw8w<F32> w;
+      load_raw_smem<F32>(row0, c, w);
+      raw_to_pairs<F32>(w, x);
 #pragma unroll
       for (int k = 0; k < 4; ++k) z[i][k] = fma_f2(dd0, x[k], z[i][k]);
       if (has1) {
-        if (kKeep) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) x[k] = x1[kKeep ? i : 0][k];
-        } else {
-          Raw8w<F32> w;
-          load_raw_smem<F32>(row1, c, w);
-          raw_to_pairs<F32>(w, x);
-        }
+        load_raw_smem<F32>(row1, c, w);
+        raw_to_pairs<F32>(w, x);
 #pragma unroll
         for (int k = 0; k < 4; ++k) z[i][k] = fma_f2(dd1, x[k], z[i][k]);
       }
@@ -284,26 +265,23 @@ __device__ __forceinline__ void power_rows2(const uint8_t* row0, const uint8_t* 
 __device__ __forceinline__ void sum_partials(const float* part, int nblk, int C, int tid, int nthr, float (&z)[8]) {
 #pragma unroll
   for (int k = 0; k < 8; ++k) z[k] = 0.f;
-  int b = 0;
-  for (; b + 4 <= nblk; b += 4) {
-    float q[8][4];
+  // partials in rounds of six (the loads of a round in flight together), added in block order
+  constexpr int kRound = 6;
+  for (int b = 0; b < nblk; b += kRound) {
+    float q[8][kRound];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int c = tid + k * nthr;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) q[k][j] = c < C ? __ldcg(part + static_cast<long long>(b + j) * C + c) : 0.f;
+      for (int j = 0; j < kRound; ++j)
+        q[k][j] = c < C && b + j < nblk ? __ldcg(part + static_cast<long long>(b + j) * C + c) : 0.f;
     }
 #pragma unroll
     for (int k = 0; k < 8; ++k)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) z[k] += q[k][j];
+      for (int j = 0; j < kRound; ++j)
+        if (b + j < nblk) z[k] += q[k][j];
   }
-  for (; b < nblk; ++b)
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int c = tid + k * nthr;
-      if (c < C) z[k] += __ldcg(part + static_cast<long long>(b) * C + c);
-    }
 }
 
 // Sum of squares of this thread's columns over the first nwarps warps, in a fixed order;
@@ -329,7 +307,10 @@ __device__ __forceinline__ double sum_squares(const float (&z)[8], double* scrat
 // bulk copy, per stage), and each of the eight consumer warps takes one row of each of two
 // stages at a time, forms t_r against v (staged in shared memory) and adds t_r W[r, :] to its
 // running z.  The warps' z are summed in warp order into one partial per block, which also
-// records its sum of t_r^2.
+// records its sum of t_r^2: where the final step's stages can hold all eight warps' z (two
+// stages of bf16 rows, one of fp32 rows), the consumers keep those stages from the producer,
+// each warp writes its z there and all consumer threads add them up at once; otherwise the
+// warps add into one buffer one after another.
 //
 // One launch runs iterations it0 .. it1-1.  Iteration it > 0 starts from the previous
 // iteration's partials, which every block sums in block order (z, then v = z / |z|); within a
@@ -391,6 +372,10 @@ __global__ void __launch_bounds__(kPowerThreads, (NV <= 5 || (!F32 && NV <= 6)) 
   const int r_beg = blockIdx.x * a.rows_per_block;
   const int r_end = min(p.rows, r_beg + a.rows_per_block);
   const int nst = (r_end - r_beg + kPowerWarps - 1) / kPowerWarps;
+  // The final step (stages jl and jl + 1) holds the warps' z when its stages have room for them:
+  // held_j is jl then, else -1.
+  const int held_j = ((nst - 1) & ~1) + 1 < nst || F32 ? (nst - 1) & ~1 : -1;
+  auto part_set = [&](int it) { return (it & 1) ? a.part[1] : a.part[0]; };
   if (threadIdx.x == 0) {
     for (int s = 0; s < a.stages; ++s) {
       mbar_init(full_bar(s), 1);
@@ -454,7 +439,7 @@ __global__ void __launch_bounds__(kPowerThreads, (NV <= 5 || (!F32 && NV <= 6)) 
             zc[k] = c < C ? x[c] : 0.f;
           }
         } else {
-          sum_partials(a.part[(it - 1) & 1] + static_cast<long long>(l) * a.nblk * C, a.nblk, C, threadIdx.x,
+          sum_partials(part_set(it - 1) + static_cast<long long>(l) * a.nblk * C, a.nblk, C, threadIdx.x,
                        kConsumers, zc);
           if (a.shift != nullptr) {
             // s y - z, y the previous pass's v (each thread reads and rewrites only its columns)
@@ -508,44 +493,89 @@ __global__ void __launch_bounds__(kPowerThreads, (NV <= 5 || (!F32 && NV <= 6)) 
           if (has1) tsq = fmaf(t1, t1, tsq);
         }
         __syncwarp();
-        if (lane == 0) {
+        if (lane == 0 && j != held_j) {
           mbar_arrive(empty_bar(s0));
           if (two) mbar_arrive(empty_bar(s1));
         }
       }
-      // the block's partial: the warps' z added into zs one warp after another
-      for (int w = 0; w < kPowerWarps; ++w) {
-        if (warp == w) {
+      // the block's partial of this iteration: the warps' z added in warp order
+      float* part = part_set(it) + (static_cast<long long>(l) * a.nblk + blockIdx.x) * C;
+      if (held_j >= 0) {
+        // once every warp has read its rows of the held stages, each warp's z goes there (warp w at
+        // slot w % wps of stage held_j + w / wps) ...
+        const int wps = F32 ? kPowerWarps : kPowerWarps / 2;  // warps' z per stage (8 C floats per two bf16 stages)
+        const int gl = gbase + held_j;
+        named_barrier_sync(1, kConsumers);
+        const int sw = (warp < wps ? gl : gl + 1) % a.stages;
+        float* zw = reinterpret_cast<float*>(ring + static_cast<size_t>(sw) * stage_bytes) + (warp % wps) * C;
 #pragma unroll
-          for (int i = 0; i < NV; ++i) {
-            const int c = 8 * lane + 256 * i;
-            if (c < C) {
-              ulonglong2* d = reinterpret_cast<ulonglong2*>(zs + c);
-              if (w == 0) {
-                d[0] = make_ulonglong2(z[i][0], z[i][1]);
-                d[1] = make_ulonglong2(z[i][2], z[i][3]);
-              } else {
-                const ulonglong2 e0 = d[0], e1 = d[1];
-                const uint64_t one = pack_f2(1.0f, 1.0f);
-                d[0] = make_ulonglong2(fma_f2(e0.x, one, z[i][0]), fma_f2(e0.y, one, z[i][1]));
-                d[1] = make_ulonglong2(fma_f2(e1.x, one, z[i][2]), fma_f2(e1.y, one, z[i][3]));
+        for (int i = 0; i < NV; ++i) {
+          const int c = 8 * lane + 256 * i;
+          if (c < C) {
+            ulonglong2* d = reinterpret_cast<ulonglong2*>(zw + c);
+            d[0] = make_ulonglong2(z[i][0], z[i][1]);
+            d[1] = make_ulonglong2(z[i][2], z[i][3]);
+          }
+        }
+        if (lane == 0) tq[warp] = tsq;
+        named_barrier_sync(1, kConsumers);
+        // ... then every consumer thread adds eight columns of the eight warps' z
+        const float* z0 = reinterpret_cast<const float*>(ring + static_cast<size_t>(gl % a.stages) * stage_bytes);
+        const float* z1 = reinterpret_cast<const float*>(ring + static_cast<size_t>((gl + 1) % a.stages) * stage_bytes);
+        for (int c = 8 * threadIdx.x; c < C; c += 8 * kConsumers) {
+          float4 lo = *reinterpret_cast<const float4*>(z0 + c), hi = *reinterpret_cast<const float4*>(z0 + c + 4);
+#pragma unroll
+          for (int w = 1; w < kPowerWarps; ++w) {
+            const float* src = (w < wps ? z0 : z1) + (w % wps) * C + c;
+            const float4 e = *reinterpret_cast<const float4*>(src), f = *reinterpret_cast<const float4*>(src + 4);
+            lo = make_float4(lo.x + e.x, lo.y + e.y, lo.z + e.z, lo.w + e.w);
+            hi = make_float4(hi.x + f.x, hi.y + f.y, hi.z + f.z, hi.w + f.w);
+          }
+          *reinterpret_cast<float4*>(part + c) = lo;
+          *reinterpret_cast<float4*>(part + c + 4) = hi;
+        }
+        // these generic accesses come before the producer's next bulk copies into the stages
+        fence_proxy_async_smem();
+      } else {
+        // the warps' z added into zs one warp after another
+        for (int w = 0; w < kPowerWarps; ++w) {
+          if (warp == w) {
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+              const int c = 8 * lane + 256 * i;
+              if (c < C) {
+                ulonglong2* d = reinterpret_cast<ulonglong2*>(zs + c);
+                if (w == 0) {
+                  d[0] = make_ulonglong2(z[i][0], z[i][1]);
+                  d[1] = make_ulonglong2(z[i][2], z[i][3]);
+                } else {
+                  const ulonglong2 e0 = d[0], e1 = d[1];
+                  const uint64_t one = pack_f2(1.0f, 1.0f);
+                  d[0] = make_ulonglong2(fma_f2(e0.x, one, z[i][0]), fma_f2(e0.y, one, z[i][1]));
+                  d[1] = make_ulonglong2(fma_f2(e1.x, one, z[i][2]), fma_f2(e1.y, one, z[i][3]));
+                }
               }
             }
+            if (lane == 0) tq[w] = tsq;
           }
-          if (lane == 0) tq[w] = tsq;
+          named_barrier_sync(1, kConsumers);
         }
-        named_barrier_sync(1, kConsumers);
+        for (int c = threadIdx.x; c < C; c += kConsumers) part[c] = zs[c];
       }
-      float* part = a.part[it & 1] + (static_cast<long long>(l) * a.nblk + blockIdx.x) * C;
-      for (int c = threadIdx.x; c < C; c += kConsumers) part[c] = zs[c];
       if (threadIdx.x == 0) {
         float acc = 0.f;
 #pragma unroll
         for (int k = 0; k < kPowerWarps; ++k) acc += tq[k];
         a.tsq_partial[static_cast<long long>(l) * a.nblk + blockIdx.x] = acc;
       }
-      __threadfence();
-      named_barrier_sync(1, kConsumers);  // zs is free again, and every store of the set is fenced
+      // Every store of the set is done (and zs or the held stages are free again).  Thread 0's
+      // release after this barrier publishes the whole block's stores (release is cumulative).
+      named_barrier_sync(1, kConsumers);
+      if (held_j >= 0 && lane == 0) {
+        const int gl = gbase + held_j;
+        mbar_arrive(empty_bar(gl % a.stages));
+        if (held_j + 1 < nst) mbar_arrive(empty_bar((gl + 1) % a.stages));
+      }
       if (threadIdx.x == 0) red_release_gpu_add(a.sync + l, 1u);
     }
   }
@@ -568,7 +598,7 @@ __global__ void __launch_bounds__(kPowerThreads, (NV <= 5 || (!F32 && NV <= 6)) 
     return;
   }
   float zc[kPowerCols];
-  sum_partials(a.part[(a.iters - 1) & 1] + static_cast<long long>(l) * a.nblk * C, a.nblk, C, threadIdx.x,
+  sum_partials(part_set(a.iters - 1) + static_cast<long long>(l) * a.nblk * C, a.nblk, C, threadIdx.x,
                kPowerThreads, zc);
   if (warp == 0) {
     const double tt = warp_sum_partials(a.tsq_partial + static_cast<long long>(l) * a.nblk, a.nblk, lane);

@@ -1,8 +1,8 @@
 """Host-side checks of the index arithmetic the elementwise and spectral kernels use (mirrors of
 the device code, no GPU): the strided row walk of the momentum and apply passes, the shared-memory
-layout of v in the streaming spectral passes, the row coverage of the column-slab pass and the
-block / stage split of the power pass.  Each mirror is compared with the plain definition
-(division, a dense loop) it replaces."""
+layout of v in the streaming spectral passes, the row coverage of the column-slab pass, the
+block / stage split of the power pass and where its warps' z meet at the end of an iteration.
+Each mirror is compared with the plain definition (division, a dense loop) it replaces."""
 import pytest
 
 
@@ -112,3 +112,56 @@ def test_power_pass_blocks_cover_rows_in_whole_stages(rows, want):
         assert nst * 8 >= end - beg > (nst - 1) * 8
         covered.extend(range(beg, end))
     assert covered == list(range(rows))
+
+
+# ---------------------------------------------------------------- power pass: warps' z in held stages
+def held_step(nst, f32):
+    """First stage of the final step when that step holds the eight warps' z, else -1."""
+    jl = (nst - 1) & ~1
+    return jl if (jl + 1 < nst or f32) else -1
+
+
+@pytest.mark.parametrize("f32", [False, True])
+@pytest.mark.parametrize("C", [8, 48, 256, 768, 1536, 2048])
+@pytest.mark.parametrize("nst", [1, 2, 3, 8, 35, 36])
+@pytest.mark.parametrize("stages", [2, 3, 7, 8])
+def test_power_pass_held_stages_take_every_warps_z(f32, C, nst, stages):
+    """At the end of an iteration of the streaming power pass, warp w writes its z (C floats,
+    eight columns per lane step) to slot w % wps of stage held_j + w / wps of the ring: the slots
+    are disjoint, lie inside their stage, the held stages are distinct ring slots, and the
+    consumer threads' eight-column reads cover every column of every warp exactly once."""
+    warps = 8
+    stage_bytes = warps * C * (4 if f32 else 2)
+    hj = held_step(nst, f32)
+    if hj < 0:
+        assert not f32 and nst % 2 == 1  # odd bf16 steps add the warps' z one after another
+        return
+    wps = warps if f32 else warps // 2
+    assert wps * C * 4 <= stage_bytes
+    for gbase in (0, 5 * nst, 17 * nst):
+        gl = gbase + hj
+        held = {gl % stages} | ({(gl + 1) % stages} if hj + 1 < nst else set())
+        assert len(held) == (2 if hj + 1 < nst else 1)
+        written = {}
+        for w in range(warps):
+            sw = (gl if w < wps else gl + 1) % stages
+            assert sw in held
+            for lane in range(32):
+                for i in range((C + 255) // 256):
+                    c = 8 * lane + 256 * i
+                    if c < C:
+                        for k in range(8):
+                            byte = (w % wps) * C * 4 + 4 * (c + k)
+                            assert byte + 4 <= stage_bytes
+                            key = (sw, byte)
+                            assert key not in written
+                            written[key] = (w, c + k)
+        assert len(written) == warps * C
+        reads = []
+        for t in range(256):
+            for c in range(8 * t, C, 8 * 256):
+                for w in range(warps):
+                    sw = (gl if w < wps else gl + 1) % stages
+                    for k in range(8):
+                        reads.append(written[(sw, (w % wps) * C * 4 + 4 * (c + k))])
+        assert sorted(reads) == sorted(written.values())
