@@ -948,34 +948,59 @@ __global__ void __launch_bounds__(kThreads, 2) colslab_kernel(const __grid_const
       if (threadIdx.x == 0) a.dsq[static_cast<long long>(l) * a.nslab + slab] = static_cast<float>(dtot);
       break;
     }
-    // phase 2: this slab's share of z = W d, a thread per row
+    // phase 2: this slab's share of z = W d, laid out like phase 1 (a row's columns over LPR
+    // lanes, 8 each, coalesced 16-byte loads, U2 rows in flight per lane: half as many for fp32
+    // rows, whose 8 columns take two loads); each row's lane products are added by an xor tree
+    // inside its row group.  The loop runs warp-uniform (rows past R contribute zeros) so that
+    // every lane takes part in the shuffles.
+    constexpr int U2 = F32 ? kSlabUnroll / 2 : kSlabUnroll;
     float* part = a.part[pass & 1] + (static_cast<long long>(l) * a.nslab + slab) * R;
-    for (int r = threadIdx.x; r < R && !abort_flag; r += kThreads) {
-      const uint4* src = reinterpret_cast<const uint4*>(W + (static_cast<long long>(r) * C + c0) * ES);
-      float z = 0.f;
+    float dk[8];
 #pragma unroll
-      for (int m = 0; m < S / 8; ++m) {
+    for (int t = 0; t < 8; ++t) dk[t] = ds[8 * k + t];
+    for (int rb = warp * RPW; rb < R && !abort_flag; rb += rstride * U2) {
+      uint4 raw[U2][F32 ? 2 : 1];
+#pragma unroll
+      for (int u = 0; u < U2; ++u) {
+        const int r = rb + rg + u * rstride;
+        if (r < R) {
+          const uint4* src = reinterpret_cast<const uint4*>(W + (static_cast<long long>(r) * C + c0 + 8 * k) * ES);
+#pragma unroll
+          for (int h = 0; h < (F32 ? 2 : 1); ++h) raw[u][h] = __ldcg(src + h);
+        } else {
+#pragma unroll
+          for (int h = 0; h < (F32 ? 2 : 1); ++h) raw[u][h] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U2; ++u) {
         float x[8];
         if (F32) {
-          const uint4 q0 = src[2 * m], q1 = src[2 * m + 1];
-          x[0] = __uint_as_float(q0.x); x[1] = __uint_as_float(q0.y); x[2] = __uint_as_float(q0.z);
-          x[3] = __uint_as_float(q0.w); x[4] = __uint_as_float(q1.x); x[5] = __uint_as_float(q1.y);
-          x[6] = __uint_as_float(q1.z); x[7] = __uint_as_float(q1.w);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            x[4 * h] = __uint_as_float(raw[u][h].x);
+            x[4 * h + 1] = __uint_as_float(raw[u][h].y);
+            x[4 * h + 2] = __uint_as_float(raw[u][h].z);
+            x[4 * h + 3] = __uint_as_float(raw[u][h].w);
+          }
         } else {
-          const uint4 q0 = src[m];
-          const uint32_t w4[4] = {q0.x, q0.y, q0.z, q0.w};
+          const uint32_t w4[4] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             x[2 * i] = __uint_as_float(w4[i] << 16);
             x[2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
           }
         }
+        float zz = 0.f;
 #pragma unroll
-        for (int t = 0; t < 8; ++t) z = fmaf(x[t], ds[8 * m + t], z);
+        for (int t = 0; t < 8; ++t) zz = fmaf(x[t], dk[t], zz);
+#pragma unroll
+        for (int o = 1; o < LPR; o <<= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
+        const int r = rb + rg + u * rstride;
+        if (k == 0 && r < R) part[r] = zz;
       }
-      part[r] = z;
     }
-    __threadfence();
+    // thread 0's release after the barrier publishes the whole block's partial (cumulative)
     __syncthreads();
     if (threadIdx.x == 0) red_release_gpu_add(a.sync + l, 1u);
   }

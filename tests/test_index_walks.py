@@ -90,6 +90,31 @@ def test_column_slab_rows_each_read_once(S, rows):
     assert seen == [1] * rows
 
 
+@pytest.mark.parametrize("S", [64, 128, 256])
+@pytest.mark.parametrize("unroll", [4, 8])
+@pytest.mark.parametrize("rows", [1, 3, 31, 64, 130, 768, 1000])
+def test_column_slab_phase2_rows_each_written_once(S, unroll, rows):
+    """Phase 2 of the column-slab pass walks the rows warp-uniformly: warp w starts at w * RPW,
+    steps by (warps x RPW x unroll), and row group g takes row start + g + u * (warps x RPW) for
+    u < unroll when it is below `rows`; every row's partial is written by exactly one lane."""
+    warps = 8
+    lpr = S // 8
+    rpw = 32 // lpr
+    rstride = warps * rpw
+    seen = [0] * rows
+    for w in range(warps):
+        rb = w * rpw
+        while rb < rows:
+            for lane in range(32):
+                g, k = lane // lpr, lane % lpr
+                for u in range(unroll):
+                    r = rb + g + u * rstride
+                    if k == 0 and r < rows:
+                        seen[r] += 1
+            rb += rstride * unroll
+    assert seen == [1] * rows
+
+
 # ---------------------------------------------------------------- power pass blocks and stages
 def power_blocks(rows, want):
     rpb = ((rows + want - 1) // want + 7) // 8 * 8
