@@ -870,8 +870,16 @@ __global__ void __launch_bounds__(kThreads, 2) colslab_kernel(const __grid_const
         const float* pp = a.part[(pass - 1) & 1] + static_cast<long long>(l) * a.nslab * R;
         const float s2 = a.shift[l] * a.shift[l];
         for (int r = threadIdx.x; r < R; r += kThreads) {
+          // the slabs' partials in slab order, eight loads in flight at a time
           float z = 0.f;
-          for (int b = 0; b < a.nslab; ++b) z += __ldcg(pp + static_cast<long long>(b) * R + r);
+          for (int b = 0; b < a.nslab; b += 8) {
+            float q[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) q[j] = b + j < a.nslab ? __ldcg(pp + static_cast<long long>(b + j) * R + r) : 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              if (b + j < a.nslab) z += q[j];
+          }
           const float v = fmaf(s2, ys[r], -z);
           ys[r] = v;
           ss += static_cast<double>(v) * v;
