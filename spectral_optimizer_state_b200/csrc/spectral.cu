@@ -195,15 +195,16 @@ __device__ __forceinline__ void raw_to_pairs(const Raw8w<F32>& r, uint64_t (&x)[
 // t = W[r, :] . v for each, then z += t W[r, :], on (even, odd) column pairs.  Each dot product
 // runs as two pair chains (the first and last four columns of every eight); the two rows' chains
 // and shuffle trees interleave.  The z update reads the stage again rather than hold the rows'
-// pairs across the trees (within the 96 registers two blocks per SM leave).
-template <bool F32, int NV>
+// pairs across the trees (within the 96 registers two blocks per SM leave).  FULL: cols is
+// exactly 256 * NV, so no column needs a bound check.
+template <bool F32, int NV, bool FULL>
 __device__ __forceinline__ void power_rows2(const uint8_t* row0, const uint8_t* row1, bool has1, const float* vs,
                                             int C, int lane, uint64_t (&z)[NV][4], float& t0, float& t1) {
   uint64_t a0 = 0, b0 = 0, a1 = 0, b1 = 0;  // (+0.0f, +0.0f) pairs
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int c = 8 * lane + 256 * i;
-    if (c < C) {
+    if (FULL || c < C) {
       const ulonglong2 lo = *reinterpret_cast<const ulonglong2*>(vs + 256 * i + 4 * lane);
       const ulonglong2 hi = *reinterpret_cast<const ulonglong2*>(vs + 256 * i + 128 + 4 * lane);
       Raw8w<F32> w;
@@ -240,7 +241,7 @@ __device__ __forceinline__ void power_rows2(const uint8_t* row0, const uint8_t* 
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int c = 8 * lane + 256 * i;
-    if (c < C) {
+    if (FULL || c < C) {
       uint64_t x[4];
       Raw8w<F32> w;
       load_raw_smem<F32>(row0, c, w);
@@ -484,7 +485,13 @@ __global__ void __launch_bounds__(kPowerThreads, (NV <= 5 || (!F32 && NV <= 6)) 
           const uint8_t* row0 = ring + static_cast<size_t>(s0) * stage_bytes + static_cast<size_t>(warp) * row_bytes;
           const uint8_t* row1 = ring + static_cast<size_t>(s1) * stage_bytes + static_cast<size_t>(warp) * row_bytes;
           float t0, t1;
-          power_rows2<F32, NV>(row0, row1, has1, vs, C, lane, z, t0, t1);
+          // rows of exactly 256 * NV columns up to 768 run without bound checks (measured faster
+          // there; wider rows keep them, which measured faster for 1536 columns and leaves 1024
+          // free of register spills)
+          if (NV <= 3 && C == 256 * NV)
+            power_rows2<F32, NV, true>(row0, row1, has1, vs, C, lane, z, t0, t1);
+          else
+            power_rows2<F32, NV, false>(row0, row1, has1, vs, C, lane, z, t0, t1);
           if (lane == 0) {
             p.y[l][r0] = t0;
             if (has1) p.y[l][r1] = t1;
