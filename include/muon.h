@@ -46,8 +46,11 @@
  *     pointers and sizes stay the same.  The first call of a shape grows
  *     them, which synchronises the device: made while `stream` is capturing,
  *     such a call returns MUON_ERR_ALLOC before queuing anything and leaves
- *     the capture intact (muon_last_cuda_error says why).  Make the same
- *     call once before capture.  A graph keeps the addresses of the
+ *     the capture intact (muon_last_cuda_error says why).  (One exception:
+ *     when the device refuses a spectral call's cooperative launch, e.g. with
+ *     another client holding SMs, a counter reset may already be queued
+ *     before its fallback finds it must grow.)  Make the same call once
+ *     before capture.  A graph keeps the addresses of the
  *     context's buffers, so once any call of a context has been captured the
  *     context never grows again: a later call that would need more returns
  *     MUON_ERR_ALLOC (use another context for it).  muon_step_groups_host
