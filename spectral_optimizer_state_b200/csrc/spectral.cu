@@ -588,9 +588,14 @@ __global__ void __launch_bounds__(kPowerThreads, (NV <= 5 || (!F32 && NV <= 6)) 
   }
   if (a.it1 < a.iters) return;
   // after the final iteration: the last block of this matrix to get here writes u, v and sigma
+  // (thread 0's fence after the barrier orders the block's stores of u, the partials and t^2
+  // before its count, for the last block's reads after its own count and fence)
   __syncthreads();
   if (abort_flag) return;
-  if (threadIdx.x == 0) s_last = atomicAdd(a.done + l, 1u) == static_cast<unsigned>(a.nblk - 1);
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(a.done + l, 1u) == static_cast<unsigned>(a.nblk - 1);
+  }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
