@@ -261,8 +261,8 @@ __device__ __forceinline__ void power_rows2(const uint8_t* row0, const uint8_t* 
 }
 
 // z[k] = sum over b = 0, 1, ... (in that order) of part[b][c_k], c_k = tid + k * nthr (zero past
-// cols; at most 8 columns per thread): every column of this thread at once, four partials ahead,
-// so the loads overlap.
+// cols; at most 8 columns per thread): every column of this thread at once, six partials per
+// round, so the loads overlap.
 __device__ __forceinline__ void sum_partials(const float* part, int nblk, int C, int tid, int nthr, float (&z)[8]) {
 #pragma unroll
   for (int k = 0; k < 8; ++k) z[k] = 0.f;
